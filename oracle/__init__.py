@@ -1,0 +1,157 @@
+"""CPU oracle for SparK channel pruning and recover-then-attend decode.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
+and the CPU-baseline / reference legs of ``bench.py`` may import this module.
+The product path never imports it and shares no code with it.
+
+The arithmetic lives in ``spark_oracle.c`` (plain C, fp64, no fast-math); this
+module only compiles it with gcc and marshals numpy arrays through ctypes.
+Every function cites the passage of the SparK pages it follows; see the C
+source header for the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "spark_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math, no FP contraction)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+               "-fno-fast-math", "-o", out, src, "-lm"]
+        subprocess.run(cmd, check=True)
+    return out
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        # ORACLE_LIB lets the planted-mistake tests run the pins against a
+        # deliberately broken copy of the oracle.
+        alt = os.environ.get("ORACLE_LIB")
+        _lib = _bind(ctypes.CDLL(alt if alt else build()))
+    return _lib
+
+
+def _bind(lib):
+    P = ctypes.c_void_p
+    L = ctypes.c_long
+    I = ctypes.c_int
+    lib.oracle_lambda_to_T.argtypes = [ctypes.c_float, I]
+    lib.oracle_lambda_to_T.restype = I
+    lib.oracle_qnorm.argtypes = [P, L, I, I, I, P]
+    lib.oracle_qnorm.restype = None
+    lib.oracle_prune.argtypes = [P, P, L, L, I, I, P, P, P]
+    lib.oracle_prune.restype = None
+    lib.oracle_recover_keys.argtypes = [P, P, P, P, L, L, I, I, P]
+    lib.oracle_recover_keys.restype = None
+    lib.oracle_decode.argtypes = [P, P, P, P, P, P, P, P, L, L, L, I, L, I, I, P]
+    lib.oracle_decode.restype = None
+    if hasattr(lib, "oracle_snapkv_scores"):
+        lib.oracle_snapkv_scores.argtypes = [P, P, L, I, I, L, I, P]
+        lib.oracle_snapkv_scores.restype = None
+        lib.oracle_snapkv_select.argtypes = [P, L, L, I, I, I, P]
+        lib.oracle_snapkv_select.restype = None
+    return lib
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def lambda_to_T(lam: float, D: int, lib=None) -> int:
+    """T = round((1 - lambda) * D), half away from zero (reading R7)."""
+    lib = lib or load()
+    return int(lib.oracle_lambda_to_T(ctypes.c_float(lam), D))
+
+
+def qnorm(q_obs, G: int, lib=None) -> np.ndarray:
+    """Window-query channel norms.  q_obs: [BH*G, W, D] (or [B, Hq, W, D]).
+    Returns qn [BH, D] fp32 (reading R1)."""
+    lib = lib or load()
+    q = _f32(q_obs)
+    W, D = q.shape[-2], q.shape[-1]
+    rows = q.size // (W * D)
+    assert rows % G == 0
+    BH = rows // G
+    qn = np.empty((BH, D), np.float32)
+    lib.oracle_qnorm(_ptr(q), BH, G, W, D, _ptr(qn))
+    return qn
+
+
+def prune(k, qn, T: int, lib=None):
+    """Top-T channel pruning.  k: [BH, S, D]; qn: [BH, D].
+    Returns (mask [BH, S, D/32] uint32, vals [BH, S, T] fp32,
+    stats [BH, 4] fp64 = {N, sum w, sum w^2, mu})."""
+    lib = lib or load()
+    k = _f32(k)
+    qn = _f32(qn)
+    D = k.shape[-1]
+    S = k.shape[-2]
+    BH = k.size // (S * D) if S > 0 else qn.size // D
+    nw = (D + 31) // 32
+    mask = np.zeros((BH, S, nw), np.uint32)
+    vals = np.zeros((BH, S, T), np.float32)
+    stats = np.zeros((BH, 4), np.float64)
+    lib.oracle_prune(_ptr(k), _ptr(qn), BH, S, D, T, _ptr(mask), _ptr(vals), _ptr(stats))
+    return mask, vals, stats
+
+
+def recover_keys(mask, vals, qn, stats, bh: int, lib=None) -> np.ndarray:
+    """Dense recovered key block K~ [S, D] (fp64) of one (b, h)."""
+    lib = lib or load()
+    mask = np.ascontiguousarray(mask, np.uint32)
+    vals = _f32(vals)
+    qn = _f32(qn)
+    stats = np.ascontiguousarray(stats, np.float64)
+    BH, S, _ = mask.shape
+    D = qn.shape[-1]
+    T = vals.shape[-1]
+    out = np.empty((S, D), np.float64)
+    lib.oracle_recover_keys(_ptr(mask), _ptr(vals), _ptr(qn), _ptr(stats), bh, S, D, T, _ptr(out))
+    return out
+
+
+def decode(q, mask, vals, qn, stats, v, k_tail=None, v_tail=None, n_tail: int = 0,
+           G: int = 1, lib=None) -> np.ndarray:
+    """Recover-then-attend decode.  q: [BH*G, D]; v: [BH, S, D];
+    k_tail/v_tail: [BH, cap, D].  Returns out [BH*G, D] fp32."""
+    lib = lib or load()
+    q = _f32(q)
+    mask = np.ascontiguousarray(mask, np.uint32)
+    vals = _f32(vals)
+    qn = _f32(qn)
+    stats = np.ascontiguousarray(stats, np.float64)
+    v = _f32(v)
+    BH, D = qn.shape
+    S = mask.shape[1]
+    T = vals.shape[-1]
+    if k_tail is None:
+        cap = max(n_tail, 1)
+        k_tail = np.zeros((BH, cap, D), np.float32)
+        v_tail = np.zeros((BH, cap, D), np.float32)
+    k_tail = _f32(k_tail)
+    v_tail = _f32(v_tail)
+    cap = k_tail.shape[1]
+    assert 0 <= n_tail <= cap
+    out = np.empty((BH * G, D), np.float32)
+    lib.oracle_decode(_ptr(q), _ptr(mask), _ptr(vals), _ptr(qn), _ptr(stats), _ptr(v),
+                      _ptr(k_tail), _ptr(v_tail), cap, n_tail, BH, G, S, D, T, _ptr(out))
+    return out

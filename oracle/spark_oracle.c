@@ -1,0 +1,231 @@
+/*
+ * spark_oracle.c -- plain, slow, obviously-correct CPU oracle for SparK
+ * channel pruning and recover-then-attend decode.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path
+ * (the CUDA library and its Python binding) never calls it, shares no code,
+ * header, table or helper with it, and fails loudly when its own CUDA
+ * library is missing.
+ *
+ * Sources (web pages on SparK, arXiv 2508.15212):
+ *   [W]  "KV Cache 还能再砍一刀：SparK 在通道维度上做了一件被忽略多年的事"
+ *        (paper walkthrough, ai-paper-analysis.pages.dev), sections 1, 3.1,
+ *        3.2, 3.3 (recovery steps 1-4 and the F table) and Fig. 3.
+ *   [A]  "AAAI 2026 AMD论文Spark方法揭秘" (AMD blog): decode runs standard
+ *        full attention after the pruned channels are rebuilt.
+ *
+ * Arithmetic: fp64 everywhere except where the reading below fixes fp32
+ * (the channel norm is rounded once to fp32, and the saliency is one fp32
+ * multiply, so that the integer outcome -- the mask -- is decided in the
+ * same precision on both sides).  Build with -ffp-contract=off and without
+ * fast-math.
+ *
+ * Readings where the pages are silent or disagree (each used everywhere):
+ *   R1  window-query channel norm: qn_j = sqrt(sum over the G query heads of
+ *       the group and the W window rows of q^2); [W] 3.1 writes ||q^j||_2 for
+ *       a channel of the query block, 3.2 replaces the query by the window.
+ *   R2  ||k^j_{i,t}||_2 for one key token is |k_t^j|.
+ *   R3  top-T ties go to the lower channel index.
+ *   R4  the statistic sampled by F is pooled per (batch, kv head) over the
+ *       pruned entries only (mu_pruned of [W] 3.3 step 1).
+ *   R5  recovered key k~ = w~ / qn_j with no sign ([W] 3.3 step 3); 0 when
+ *       qn_j == 0.
+ *   R6  softmax scale 1/sqrt(D); decode-time tail tokens are never pruned.
+ *   R7  T = round((1 - lambda) * D), half away from zero, in fp64.
+ *   R8  an empty context (no prefix, no tail) gives a zero output row.
+ *
+ * Layouts (row-major, all plain, none shared with the GPU path):
+ *   q_obs [BH*G][W][D]     k, v [BH][S][D]      qn [BH][D]  (fp32)
+ *   mask  [BH][S][ceil(D/32)] uint32, bit j%32 of word j/32 = channel kept
+ *   vals  [BH][S][T] fp32 (kept key values, ascending channel)
+ *   stats [BH][4] fp64 = {N_pruned, sum w, sum w^2, mu_pruned}
+ *   q, out [BH*G][D]; k_tail, v_tail [BH][tail_cap][D]
+ * Query head g of kv head h is row h*G + g (consecutive GQA grouping).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* R7: pruning ratio lambda -> number of kept channels T ([W] 4.1, Table 1
+ * caption of [A]: lambda is the fraction of key channels pruned). */
+int oracle_lambda_to_T(float lambda, int D)
+{
+    if (!(lambda >= 0.0f && lambda <= 1.0f) || D <= 0)
+        return -1;
+    return (int)llround((1.0 - (double)lambda) * (double)D);
+}
+
+/* R1: observation-window channel norm ([W] 3.1 saliency, 3.2 window). */
+void oracle_qnorm(const float *q_obs, long BH, int G, int W, int D, float *qn)
+{
+    for (long bh = 0; bh < BH; ++bh)
+        for (int j = 0; j < D; ++j) {
+            double acc = 0.0;
+            for (int g = 0; g < G; ++g)
+                for (int t = 0; t < W; ++t) {
+                    double x = q_obs[((bh * G + g) * (long)W + t) * D + j];
+                    acc += x * x;
+                }
+            qn[bh * D + j] = (float)sqrt(acc);
+        }
+}
+
+/* Proxy saliency of one entry, [W] 3.1: w = ||q^j||_2 * |k^j| as one fp32
+ * multiply (R2). */
+static float saliency(float qn_j, float k_tj)
+{
+    float a = fabsf(k_tj);
+    return qn_j * a;
+}
+
+typedef struct {
+    float w;
+    int j;
+} chan_score;
+
+/* Greedy order of the relaxed objective ([W] 3.1): larger saliency first,
+ * then lower channel index (R3). */
+static int by_saliency_desc(const void *pa, const void *pb)
+{
+    const chan_score *a = (const chan_score *)pa, *b = (const chan_score *)pb;
+    if (a->w > b->w) return -1;
+    if (a->w < b->w) return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+/* Per-token top-T channel selection + packing + pruned-score statistics.
+ * [W] 3.1 (relaxed objective max sum w z, sum z = T, solved greedily by
+ * sorting), 3.2 (per-token unstructured mask), 3.3 step 1 (cache keeps the
+ * pruned key, the mask and the score statistics). */
+void oracle_prune(const float *k, const float *qn, long BH, long S, int D,
+                  int T, uint32_t *mask, float *vals, double *stats)
+{
+    const int nw = (D + 31) / 32;
+    chan_score *order = (chan_score *)malloc(sizeof(chan_score) * (size_t)D);
+    unsigned char *keep = (unsigned char *)malloc((size_t)D);
+    float *w = (float *)malloc(sizeof(float) * (size_t)D);
+    for (long bh = 0; bh < BH; ++bh) {
+        double n = 0.0, sw = 0.0, sw2 = 0.0;
+        for (long t = 0; t < S; ++t) {
+            const float *krow = k + (bh * S + t) * D;
+            for (int j = 0; j < D; ++j) {
+                w[j] = saliency(qn[bh * D + j], krow[j]);
+                order[j].w = w[j];
+                order[j].j = j;
+            }
+            qsort(order, (size_t)D, sizeof(chan_score), by_saliency_desc);
+            memset(keep, 0, (size_t)D);
+            for (int r = 0; r < T; ++r)
+                keep[order[r].j] = 1;
+
+            uint32_t *mrow = mask + (bh * S + t) * nw;
+            for (int q = 0; q < nw; ++q)
+                mrow[q] = 0u;
+            float *vrow = vals + (bh * S + t) * (long)T;
+            int pos = 0;
+            for (int j = 0; j < D; ++j) {
+                if (keep[j]) {
+                    mrow[j / 32] |= 1u << (j % 32);
+                    vrow[pos++] = krow[j];
+                } else {
+                    double x = (double)w[j];
+                    n += 1.0;
+                    sw += x;
+                    sw2 += x * x;
+                }
+            }
+        }
+        stats[bh * 4 + 0] = n;
+        stats[bh * 4 + 1] = sw;
+        stats[bh * 4 + 2] = sw2;
+        stats[bh * 4 + 3] = (n > 0.0) ? sw / n : 0.0;
+    }
+    free(order);
+    free(keep);
+    free(w);
+}
+
+/* Recovery F = Degenerate, [W] 3.3 steps 2-4 and the F table: the sampled
+ * score is mu_pruned, and the key is back-solved from it as
+ * k~ = w~ / ||q^j||_2 (R5).  Kept channels are the stored key values.
+ * Writes the dense recovered key block Kt [S][D] (fp64) of one (b, h). */
+void oracle_recover_keys(const uint32_t *mask, const float *vals,
+                         const float *qn, const double *stats, long bh,
+                         long S, int D, int T, double *Kt)
+{
+    const int nw = (D + 31) / 32;
+    const double mu = stats[bh * 4 + 3];
+    for (long t = 0; t < S; ++t) {
+        const uint32_t *mrow = mask + (bh * S + t) * nw;
+        const float *vrow = vals + (bh * S + t) * (long)T;
+        int pos = 0;
+        for (int j = 0; j < D; ++j) {
+            int kept = (mrow[j / 32] >> (j % 32)) & 1u;
+            if (kept) {
+                Kt[t * D + j] = (double)vrow[pos++];
+            } else {
+                double qj = (double)qn[bh * D + j];
+                Kt[t * D + j] = (qj > 0.0) ? mu / qj : 0.0;
+            }
+        }
+    }
+}
+
+/* Decode: standard full attention over the recovered keys ([W] Fig. 3,
+ * [A]): for each query head, s_t = q . k~_t / sqrt(D) over the pruned
+ * prefix then the dense tail, softmax (max-subtracted, two passes), and
+ * out = sum_t p_t v_t.  Output rounded once to fp32. */
+void oracle_decode(const float *q, const uint32_t *mask, const float *vals,
+                   const float *qn, const double *stats, const float *v,
+                   const float *k_tail, const float *v_tail, long tail_cap,
+                   long n_tail, long BH, int G, long S, int D, int T,
+                   float *out)
+{
+    const long L = S + n_tail;
+    double *Kt = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * (size_t)D);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *acc = (double *)malloc(sizeof(double) * (size_t)D);
+    const double scale = 1.0 / sqrt((double)D);
+    for (long bh = 0; bh < BH; ++bh) {
+        oracle_recover_keys(mask, vals, qn, stats, bh, S, D, T, Kt);
+        for (long t = 0; t < n_tail; ++t)
+            for (int j = 0; j < D; ++j)
+                Kt[(S + t) * D + j] = (double)k_tail[(bh * tail_cap + t) * D + j];
+        for (int g = 0; g < G; ++g) {
+            const float *qrow = q + (bh * G + g) * (long)D;
+            float *orow = out + (bh * G + g) * (long)D;
+            if (L == 0) {
+                for (int d = 0; d < D; ++d)
+                    orow[d] = 0.0f;
+                continue;
+            }
+            double m = -INFINITY;
+            for (long t = 0; t < L; ++t) {
+                double dot = 0.0;
+                for (int j = 0; j < D; ++j)
+                    dot += (double)qrow[j] * Kt[t * D + j];
+                s[t] = dot * scale;
+                if (s[t] > m)
+                    m = s[t];
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; ++d)
+                acc[d] = 0.0;
+            for (long t = 0; t < L; ++t) {
+                double p = exp(s[t] - m);
+                const float *vrow = (t < S) ? v + (bh * S + t) * D
+                                            : v_tail + (bh * tail_cap + (t - S)) * D;
+                l += p;
+                for (int d = 0; d < D; ++d)
+                    acc[d] += p * (double)vrow[d];
+            }
+            for (int d = 0; d < D; ++d)
+                orow[d] = (float)(acc[d] / l);
+        }
+    }
+    free(Kt);
+    free(s);
+    free(acc);
+}

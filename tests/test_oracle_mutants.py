@@ -1,0 +1,53 @@
+"""Planted mistakes: each test copies the oracle's C source, plants one
+plausible mistake (a dropped term, a wrong sign or index, a transposed
+operand, a reversed tie rule), compiles the copy on the CPU and checks that
+the pin suite fails on it.  This shows the pins constrain every step of the
+oracle, not only the ones they were written for."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+
+MUTANTS = {
+    "tie_rule_reversed": ("return (a->j > b->j) - (a->j < b->j);",
+                          "return (a->j < b->j) - (a->j > b->j);"),
+    "qnorm_one_group_head": ("for (int g = 0; g < G; ++g)\n                for (int t = 0; t < W; ++t)",
+                             "for (int g = 0; g < 1; ++g)\n                for (int t = 0; t < W; ++t)"),
+    "qnorm_drops_window": ("for (int t = 0; t < W; ++t) {\n                    double x",
+                           "for (int t = 0; t < 1; ++t) {\n                    double x"),
+    "saliency_no_abs": ("float a = fabsf(k_tj);", "float a = k_tj;"),
+    "recovery_no_division": ("? mu / qj : 0.0;", "? mu : 0.0;"),
+    "recovery_sign_flip": ("? mu / qj : 0.0;", "? -mu / qj : 0.0;"),
+    "stats_over_kept": ("} else {\n                    double x = (double)w[j];",
+                        "}\n                {\n                    double x = (double)w[j];"),
+    "mean_wrong_denominator": ("? sw / n : 0.0;", "? sw / (n + 1.0) : 0.0;"),
+    "keeps_one_less": ("for (int r = 0; r < T; ++r)", "for (int r = 0; r < T - 1; ++r)"),
+    "vals_reversed": ("vrow[pos++] = krow[j];", "vrow[T - 1 - pos++] = krow[j];"),
+    "score_scale_1_over_D": ("1.0 / sqrt((double)D);", "1.0 / (double)D;"),
+    "gqa_transposed": ("const float *qrow = q + (bh * G + g) * (long)D;",
+                       "const float *qrow = q + ((long)g * BH + bh) * (long)D;"),
+    "tail_keys_from_values": ("(double)k_tail[(bh * tail_cap + t) * D + j];",
+                              "(double)v_tail[(bh * tail_cap + t) * D + j];"),
+    "lambda_truncates": ("return (int)llround((1.0 - (double)lambda) * (double)D);",
+                         "return (int)((1.0 - (double)lambda) * (double)D);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    before, after = MUTANTS[name]
+    src = open(os.path.join(ROOT, "oracle", "spark_oracle.c")).read()
+    assert src.count(before) == 1, f"mutation site for {name} not unique"
+    mutant_c = tmp_path / "mutant.c"
+    mutant_c.write_text(src.replace(before, after))
+    lib = oracle.build(force=True, src=str(mutant_c), out=str(tmp_path / "libmutant.so"))
+    env = dict(os.environ, ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", PINS, "-x", "-q", "-p", "no:cacheprovider"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
