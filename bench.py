@@ -1,0 +1,456 @@
+"""Benchmark of the SparK hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+window-norm + top-T channel pruning + pruned-saliency statistics over every
+(layer, kv head) of the prompt (spark_prune), one unpruned key/value appended
+to the dense tail (spark_tail_append), and one decode-attention step over the
+pruned cache plus tail for every layer (spark_decode_attn: split-K kernel and
+log-sum-exp combine).  Default workload: the pages' long-context Llama-3.1-8B
+shape -- B=1, 32 layers x 8 kv heads x GQA 4, D=128, S=131072, bf16,
+lambda=0.8 (T=26).
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the CPU oracle (the
+only reference this method has) on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from channel_pruned_decode_b200.synth import (WORKLOADS, make_decode_step, make_prefill,  # noqa: E402
+                                              scaled)
+
+METRIC = "decode-attn KV tokens·heads/s & HBM GB/s (frac of 8 TB/s); spark_prune GB/s"
+UNIT = "KV token·heads/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _workload_desc(wl, T):
+    return (f"{wl.name}: B={wl.B} L={wl.L} Hkv={wl.Hkv} G={wl.G} S={wl.S} D={wl.D} W={wl.W} "
+            f"lambda={wl.lam} (T={T}) {wl.dtype}; prune all layers + tail append + 1 decode step")
+
+
+def _byte_model(wl, T, n_tail):
+    """Algorithmic HBM bytes per launch of the two heavy calls."""
+    es = 2 if wl.dtype == "bf16" else 4
+    BH, S, D, G = wl.BH, wl.S, wl.D, wl.G
+    prune = BH * S * (D * es + 16 + T * es) + BH * G * wl.W * D * es + BH * (D * 4 + 32)
+    decode = (BH * S * (16 + T * es + D * es) + BH * n_tail * 2 * D * es
+              + BH * G * D * (es + 4) + BH * (D * 4 + 32))
+    return {"prune": prune, "decode": decode, "per_token_head_prune": D * es + 16 + T * es,
+            "per_token_head_decode": 16 + T * es + D * es}
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+        except Exception:
+            bus = str(device_index)
+        self.bus = bus
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.bus, f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# -------------------------------------------------------------- GPU arm
+class Job:
+    """Device buffers and the step of one rank."""
+
+    def __init__(self, wl, dev, host_inputs: bool = False):
+        import channel_pruned_decode_b200 as sp
+        self.sp = sp
+        self.wl = wl
+        self.dev = dev
+        self.T = sp.spark_lambda_to_T(wl.lam, wl.D)
+        pre = make_prefill(wl, dev)
+        self.k, self.v, self.q_obs = pre["k"], pre["v"], pre["q_obs"]
+        stp = make_decode_step(wl, 0, dev)
+        self.q, self.k_new, self.v_new = stp["q"], stp["k_new"], stp["v_new"]
+        R, H, S, D, G = wl.rows, wl.Hkv, wl.S, wl.D, wl.G
+        self.cap = wl.tail_cap
+        self.kt = torch.zeros((R, H, self.cap, D), dtype=wl.torch_dtype, device=dev)
+        self.vt = torch.zeros_like(self.kt)
+        self.kc = sp.KCache.empty(R, H, S, D, self.T, wl.torch_dtype, device=dev)
+        self.wsp = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_PRUNE, R, H, G, S, D, self.T, 0), dev)
+        self.wsd = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_DECODE, R, H, G, S, D, self.T,
+                                                         self.cap), dev)
+        self.out = torch.empty((R, wl.Hq, D), dtype=torch.float32, device=dev)
+        self.n_tail = 0
+        self.launches_per_step = 6  # qnorm, prune, stats, tail append, decode, combine
+
+    def step(self, stream, ev=None):
+        sp, wl = self.sp, self.wl
+        slot = 0  # one decode step per bench step: the tail holds this step's token
+        if ev is not None:
+            ev[0].record(stream)
+        sp.spark_prune(self.k, self.q_obs, wl.G, wl.W, self.kc, self.wsp, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        sp.spark_tail_append(self.k_new, self.v_new, self.kt, self.vt, wl.rows, wl.Hkv, wl.D, self.cap,
+                             slot, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        sp.spark_decode_attn(self.q, self.kc, self.v, self.kt, self.vt, self.cap, slot + 1, wl.G,
+                             self.out, self.wsd, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+
+def _barrier(dist_on):
+    if dist_on:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            recs = json.load(f)
+    except Exception:
+        return None
+    rec = recs.get(f"{kernel}@{workload}")
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except Exception:
+        return None
+    return rec["bytes_per_launch"] if h == rec["source_sha"] else None
+
+
+def cpu_baseline(wl, job, units: int | None = None):
+    """The CPU oracle, as it stands, on a bounded sample of the workload:
+    prune + decode of whole (layer, kv head) units, threads over units."""
+    import concurrent.futures as cf
+
+    import numpy as np
+
+    import oracle
+
+    lib = oracle.load()
+    BH, S, D, G = wl.BH, wl.S, wl.D, wl.G
+    cores = os.cpu_count() or 1
+    units = units or min(BH, cores)
+    sel = list(range(0, BH, max(1, BH // units)))[:units]
+    k = job.k.reshape(BH, S, D)
+    v = job.v.reshape(BH, S, D)
+    qo = job.q_obs.reshape(BH * G, wl.W, D)
+    q = job.q.reshape(BH * G, D)
+    data = []
+    for b in sel:
+        data.append((k[b:b + 1].float().cpu().numpy(), v[b:b + 1].float().cpu().numpy(),
+                     qo[b * G:(b + 1) * G].float().cpu().numpy(), q[b * G:(b + 1) * G].float().cpu().numpy()))
+
+    def one(d):
+        kk, vv, qq, q1 = d
+        qn = oracle.qnorm(qq, G, lib=lib)
+        m, vals, st = oracle.prune(kk, qn, job.T, lib=lib)
+        return oracle.decode(q1, m, vals, qn, st, vv, G=G, lib=lib)
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=min(cores, len(data))) as ex:
+        list(ex.map(one, data))
+    dt = time.perf_counter() - t0
+    return {"value": len(data) * S / dt, "unit": UNIT, "cores": min(cores, len(data)), "kind": "oracle",
+            "sample": f"{len(data)} of {BH} (layer, kv head) units, full S={S}: prune + 1 decode step, "
+                      f"{dt:.1f} s wall"}
+
+
+def run_gpu(args):
+    dist_on = args.gpus > 1
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if dist_on:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = WORKLOADS[args.workload]
+    job = Job(wl, dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            job.step(stream)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    _barrier(dist_on)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            job.step(stream, evs[i])
+        end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    _barrier(dist_on)
+    ms_local = start.elapsed_time(end)
+    prune_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    decode_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    append_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    ms = _max_over_ranks(ms_local, dist_on)
+    st = job.sp.spark_device_status(job.wsd)
+    st |= job.sp.spark_device_status(job.wsp)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timed region")
+
+    token_heads = wl.BH * (wl.S + 1)
+    ms_per_step = ms / args.steps
+    value = world * token_heads / (ms_per_step / 1e3)
+    bm = _byte_model(wl, job.T, 1)
+    peak, peak_kind = _peaks()
+    prune_gbs = bm["prune"] / (prune_ms / 1e3) / 1e9
+    decode_gbs = bm["decode"] / (decode_ms / 1e3) / 1e9
+    dom = "prune" if prune_ms >= decode_ms else "decode"
+    dom_ms = prune_ms if dom == "prune" else decode_ms
+    achieved = bm[dom] / (dom_ms / 1e3) / 1e9
+    kernel_name = {"prune": "prune_kernel", "decode": "decode_kernel"}[dom]
+    traffic = _traffic_record(kernel_name, wl.name)
+
+    e2e = None
+    if not args.no_e2e:  # every rank: the e2e timing has its own barrier and max
+        e2e = run_e2e(job, wl, min(args.steps, args.e2e_steps), dist_on, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, job)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded N(0,1) x per-channel LogNormal(0,1) outlier scales)",
+            "config": {"workload": _workload_desc(wl, job.T), "B": wl.B, "layers": wl.L, "Hkv": wl.Hkv,
+                       "G": wl.G, "S": wl.S, "D": wl.D, "W": wl.W, "lambda": wl.lam, "T": job.T,
+                       "parallelism": f"replicas x{world} (independent (layer, head) work per GPU)",
+                       "l2": "inputs (K, V: 17.2 GB) exceed the 126 MB L2; no flush needed"},
+            "decode": {"us_per_step": decode_ms * 1e3, "gbs": decode_gbs,
+                       "frac_8tbs": decode_gbs / NOMINAL_HBM_GBS, f"frac_{peak_kind}": decode_gbs / peak,
+                       "token_heads_per_s": world * token_heads / (decode_ms / 1e3),
+                       "bytes_per_step": bm["decode"]},
+            "prune": {"us_per_step": prune_ms * 1e3, "gbs": prune_gbs, "frac_8tbs": prune_gbs / NOMINAL_HBM_GBS,
+                      f"frac_{peak_kind}": prune_gbs / peak, "bytes_per_step": bm["prune"]},
+            "tail_append_us": append_ms * 1e3,
+            "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic,
+                         "bytes_per_launch": bm[dom],
+                         "timing": "CUDA events around the entry point on its stream "
+                                   "(the two small kernels launched with it included)"},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": job.launches_per_step * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(job, wl, steps, dist_on, world):
+    """Same metric through the public API with pinned HOST inputs: every step
+    copies K, V, window queries and the decode query/new key/value to the
+    device, runs the step and reads the output back."""
+    import psutil
+    need = sum(t.numel() * t.element_size() for t in (job.k, job.v, job.q_obs, job.q, job.k_new, job.v_new))
+    if psutil.virtual_memory().available < 2.5 * need:
+        return {"value": None, "unit": UNIT, "skipped": f"host RAM < 2.5 x {need / 1e9:.1f} GB"}
+    hk = torch.empty(job.k.shape, dtype=job.k.dtype, pin_memory=True)
+    hv = torch.empty(job.v.shape, dtype=job.v.dtype, pin_memory=True)
+    hk.copy_(job.k)
+    hv.copy_(job.v)
+    small = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t), t)
+             for t in (job.q_obs, job.q, job.k_new, job.v_new)]
+    hout = torch.empty(job.out.shape, dtype=job.out.dtype, pin_memory=True)
+    stream = torch.cuda.Stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def one():
+        job.k.copy_(hk, non_blocking=True)
+        job.v.copy_(hv, non_blocking=True)
+        for h, d in small:
+            d.copy_(h, non_blocking=True)
+        job.step(stream)
+        hout.copy_(job.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        one()
+    torch.cuda.synchronize()
+    _barrier(dist_on)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            one()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(start.elapsed_time(end), dist_on) / steps
+    h2d = need
+    d2h = hout.numel() * hout.element_size()
+    return {"value": world * wl.BH * (wl.S + 1) / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+# -------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import concurrent.futures as cf
+
+    import oracle
+    lib = oracle.load()
+    wl = WORKLOADS[args.workload]
+    T = oracle.lambda_to_T(wl.lam, wl.D, lib=lib)
+    cores = os.cpu_count() or 1
+    S, D, G = wl.S, wl.D, wl.G
+    # one step = `cores` (kv head) units of the first S_s prompt tokens: prune +
+    # one decode step each; bounded so that K + W steps take a few minutes
+    S_s = min(S, 16384)
+    wl1 = scaled(wl, L=1, B=1, S=S_s)
+    pre = make_prefill(wl1, "cpu")
+    stp = make_decode_step(wl1, 0, "cpu")
+    units = []
+    for u in range(cores):
+        h = u % wl.Hkv
+        units.append((pre["k"][0, h:h + 1].float().numpy(), pre["v"][0, h:h + 1].float().numpy(),
+                      pre["q_obs"][0, h * G:(h + 1) * G].float().numpy(),
+                      stp["q"][0, h * G:(h + 1) * G].float().numpy()))
+
+    def one(d):
+        kk, vv, qq, q1 = d
+        qn = oracle.qnorm(qq, G, lib=lib)
+        m, vals, st = oracle.prune(kk, qn, T, lib=lib)
+        return oracle.decode(q1, m, vals, qn, st, vv, G=G, lib=lib)
+
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        for _ in range(args.warmup):
+            list(ex.map(one, units))
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            list(ex.map(one, units))
+        dt = time.perf_counter() - t0
+    value = args.steps * len(units) * (S_s + 1) / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": _workload_desc(wl, T)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {len(units)} kv-head units of the first {S_s} of "
+                                   f"S={S} prompt tokens, prune + 1 decode step (threads over units)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="spark", choices=["spark", "reference"])
+    ap.add_argument("--workload", default="long", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,14 @@
+"""SparK on B200: query-aware unstructured key-cache channel pruning at
+prefill and recover-then-attend decode attention, as hand-written sm_100a
+CUDA kernels behind a C ABI (include/spark.h), with a thin ctypes binding.
+
+Method: SparK (arXiv 2508.15212), as described by the paper walkthrough
+"KV Cache 还能再砍一刀：SparK 在通道维度上做了一件被忽略多年的事" (sections
+3.1-3.3, Fig. 3) and the AMD blog "AAAI 2026 AMD论文Spark方法揭秘".
+"""
+from .binding import (  # noqa: F401
+    KCache, SparkError, lib, spark_cache_bytes, spark_cache_sizes, spark_decode_attn,
+    spark_device_status, spark_lambda_to_T, spark_prune, spark_tail_append, spark_workspace_bytes,
+    status_str, workspace, SPARK_BF16, SPARK_F32, SPARK_OP_DECODE, SPARK_OP_PRUNE,
+    SPARK_F_DEGENERATE, SPARK_F_GAUSSIAN, SPARK_F_EXPONENTIAL, EXPORTS,
+)

@@ -1,0 +1,198 @@
+"""Thin ctypes binding of libspark.so (include/spark.h).
+
+Argument marshalling only: every step of pruning and decode runs in the CUDA
+kernels of libspark.so.  torch tensors supply device memory and streams.
+There is no CPU fallback: loading fails loudly when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspark.so")
+
+SPARK_OK = 0
+SPARK_ERR_ARG = 1
+SPARK_ERR_UNSUPPORTED = 2
+SPARK_ERR_CUDA = 3
+SPARK_ERR_TIMEOUT = 4
+SPARK_ERR_WORKSPACE = 5
+SPARK_F32 = 0
+SPARK_BF16 = 1
+SPARK_F_DEGENERATE = 0
+SPARK_F_GAUSSIAN = 1
+SPARK_F_EXPONENTIAL = 2
+SPARK_OP_PRUNE = 0
+SPARK_OP_DECODE = 1
+
+EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
+           "spark_prune", "spark_decode_attn", "spark_tail_append", "spark_device_status",
+           "spark_status_str")
+
+
+class SparkError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+class spark_kcache(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("S", ctypes.c_int), ("D", ctypes.c_int),
+                ("T", ctypes.c_int), ("dtype", ctypes.c_int), ("mask", ctypes.c_void_p),
+                ("vals", ctypes.c_void_p), ("qn", ctypes.c_void_p), ("stats", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libspark.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"SparK CUDA library not found at {_LIB_PATH}; build it with "
+                               "`python -m channel_pruned_decode_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.spark_lambda_to_T.argtypes = [ctypes.c_float, I]
+        L.spark_lambda_to_T.restype = I
+        L.spark_cache_sizes.argtypes = [I, I, I, I, I, I, ctypes.POINTER(Z)]
+        L.spark_cache_sizes.restype = Z
+        L.spark_cache_bytes.argtypes = [I, I, I, I, I, I]
+        L.spark_cache_bytes.restype = Z
+        L.spark_workspace_bytes.argtypes = [I, I, I, I, I, I, I, I]
+        L.spark_workspace_bytes.restype = Z
+        L.spark_prune.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P, Z, P]
+        L.spark_prune.restype = I
+        L.spark_decode_attn.argtypes = [P, ctypes.POINTER(spark_kcache), P, P, P, I, I, I, I,
+                                        ctypes.c_ulonglong, P, P, Z, P]
+        L.spark_decode_attn.restype = I
+        L.spark_tail_append.argtypes = [P, P, P, P, I, I, I, I, I, I, P]
+        L.spark_tail_append.restype = I
+        L.spark_device_status.argtypes = [P, ctypes.POINTER(I), I, P]
+        L.spark_device_status.restype = I
+        L.spark_status_str.argtypes = [I]
+        L.spark_status_str.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().spark_status_str(status).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != SPARK_OK:
+        raise SparkError(rc, where)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return SPARK_BF16
+    if t == torch.float32:
+        return SPARK_F32
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ------------------------------------------------------------------ sizes
+def spark_lambda_to_T(lam: float, D: int = 128) -> int:
+    return int(lib().spark_lambda_to_T(ctypes.c_float(lam), D))
+
+
+def spark_cache_sizes(B, Hkv, S, D, T, dtype) -> tuple[int, list[int]]:
+    sizes = (ctypes.c_size_t * 4)()
+    total = lib().spark_cache_sizes(B, Hkv, S, D, T, dtype, sizes)
+    return int(total), [int(x) for x in sizes]
+
+
+def spark_cache_bytes(B, Hkv, S, D, T, dtype) -> int:
+    return int(lib().spark_cache_bytes(B, Hkv, S, D, T, dtype))
+
+
+def spark_workspace_bytes(op, B, Hkv, G, S, D, T, n_tail) -> int:
+    return int(lib().spark_workspace_bytes(op, B, Hkv, G, S, D, T, n_tail))
+
+
+# ------------------------------------------------------------------ cache
+@dataclass
+class KCache:
+    """Device tensors of the packed key cache (layout of include/spark.h)."""
+    B: int
+    Hkv: int
+    S: int
+    D: int
+    T: int
+    dtype: torch.dtype
+    mask: torch.Tensor    # uint32 bits stored as int32 [B, Hkv, S, 4]
+    vals: torch.Tensor    # [B, Hkv, S32 * T] interleaved by 32-token groups
+    qn: torch.Tensor      # fp32 [B, Hkv, D]
+    stats: torch.Tensor   # fp64 [B, Hkv, 4]
+
+    @staticmethod
+    def empty(B, Hkv, S, D, T, dtype, device="cuda") -> "KCache":
+        S32 = (S + 31) // 32 * 32
+        return KCache(B, Hkv, S, D, T, dtype,
+                      torch.empty((B, Hkv, S, 4), dtype=torch.int32, device=device),
+                      torch.empty((B, Hkv, S32 * T), dtype=dtype, device=device),
+                      torch.empty((B, Hkv, D), dtype=torch.float32, device=device),
+                      torch.empty((B, Hkv, 4), dtype=torch.float64, device=device))
+
+    def struct(self) -> spark_kcache:
+        return spark_kcache(self.B, self.Hkv, self.S, self.D, self.T, _dtype_code(self.dtype),
+                            _ptr(self.mask), _ptr(self.vals), _ptr(self.qn), _ptr(self.stats))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.mask, self.vals, self.qn, self.stats))
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Zero-initialised workspace (the status word must start at zero)."""
+    n = (max(nbytes, 256) + 255) // 256 * 256
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------- entry points
+def spark_prune(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, kc: KCache,
+                ws: torch.Tensor, stream=None) -> None:
+    s = kc.struct()
+    rc = lib().spark_prune(_ptr(k), _ptr(q_obs), G, W, ctypes.byref(s), _ptr(ws),
+                           ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_prune")
+
+
+def spark_decode_attn(q: torch.Tensor, kc: KCache, v: torch.Tensor, k_tail, v_tail, tail_cap: int,
+                      n_tail: int, G: int, out: torch.Tensor, ws: torch.Tensor,
+                      recovery: int = SPARK_F_DEGENERATE, seed: int = 0, stream=None) -> None:
+    s = kc.struct()
+    rc = lib().spark_decode_attn(_ptr(q), ctypes.byref(s), _ptr(v), _ptr(k_tail), _ptr(v_tail), tail_cap,
+                                 n_tail, G, recovery, seed, _ptr(out), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_decode_attn")
+
+
+def spark_tail_append(k_new, v_new, k_tail, v_tail, B, Hkv, D, tail_cap, slot, stream=None) -> None:
+    rc = lib().spark_tail_append(_ptr(k_new), _ptr(v_new), _ptr(k_tail), _ptr(v_tail), B, Hkv, D,
+                                 tail_cap, slot, _dtype_code(k_new.dtype), _stream(stream))
+    _check(rc, "spark_tail_append")
+
+
+def spark_device_status(ws: torch.Tensor, clear: bool = False, stream=None) -> int:
+    st = ctypes.c_int(0)
+    rc = lib().spark_device_status(_ptr(ws), ctypes.byref(st), int(clear), _stream(stream))
+    _check(rc, "spark_device_status")
+    return st.value

@@ -1,0 +1,196 @@
+// C ABI entry points of the SparK sm_100a library: argument validation,
+// cache layout arithmetic, workspace sizing, the tail-append kernel and the
+// device status word.  The compute kernels live in prune.cu and decode.cu.
+#include "spark_internal.cuh"
+
+#include <math.h>
+
+namespace spark {
+cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const spark_kcache &kc,
+                         void *ws, cudaStream_t st);
+cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const void *k_tail,
+                          const void *v_tail, int tail_cap, int n_tail, int G, float *out, void *ws,
+                          const DecodeGeom &geo, cudaStream_t st);
+
+static int elem_size(int dtype) {
+    return dtype == SPARK_F32 ? 4 : (dtype == SPARK_BF16 ? 2 : 0);
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+static int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+// shape checks shared by prune and decode; returns SPARK_OK or an error
+static int check_cache(const spark_kcache *kc) {
+    if (!kc) return SPARK_ERR_ARG;
+    if (kc->B < 0 || kc->Hkv < 0 || kc->S < 0) return SPARK_ERR_ARG;
+    if (elem_size(kc->dtype) == 0) return SPARK_ERR_ARG;
+    if (kc->D != kD) return SPARK_ERR_UNSUPPORTED;
+    if (kc->T < 0 || kc->T > kc->D) return SPARK_ERR_ARG;
+    if ((long)kc->B * kc->Hkv == 0) return SPARK_OK;
+    if (!kc->qn || !kc->stats || !aligned16(kc->qn) || !aligned16(kc->stats)) return SPARK_ERR_ARG;
+    if (kc->S > 0) {
+        if (!kc->mask || !aligned16(kc->mask)) return SPARK_ERR_ARG;
+        if (kc->T > 0 && (!kc->vals || !aligned16(kc->vals))) return SPARK_ERR_ARG;
+    }
+    return SPARK_OK;
+}
+
+__global__ void tail_append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                                   uint4 *__restrict__ k_tail, uint4 *__restrict__ v_tail,
+                                   int row_vec, int tail_cap, int slot) {
+    const long bh = blockIdx.x;
+    const int i = threadIdx.x;
+    if (i < row_vec) {
+        const size_t dst = ((size_t)bh * tail_cap + slot) * row_vec + i;
+        k_tail[dst] = k_new[(size_t)bh * row_vec + i];
+        v_tail[dst] = v_new[(size_t)bh * row_vec + i];
+    }
+}
+
+}  // namespace spark
+
+using namespace spark;
+
+extern "C" {
+
+int spark_lambda_to_T(float lambda, int D) {
+    if (!(lambda >= 0.0f && lambda <= 1.0f) || D <= 0) return -1;
+    return (int)llround((1.0 - (double)lambda) * (double)D);
+}
+
+size_t spark_cache_sizes(int B, int Hkv, int S, int D, int T, int dtype, size_t sizes[4]) {
+    const int es = elem_size(dtype);
+    if (B < 0 || Hkv < 0 || S < 0 || D != kD || T < 0 || T > D || es == 0) return 0;
+    const size_t BH = (size_t)B * Hkv;
+    const size_t S32 = ((size_t)S + 31) / 32 * 32;
+    size_t sz[4];
+    sz[0] = BH * S * kMaskWords * sizeof(uint32_t);
+    sz[1] = BH * S32 * T * es;
+    sz[2] = BH * D * sizeof(float);
+    sz[3] = BH * 4 * sizeof(double);
+    size_t total = 0;
+    for (int i = 0; i < 4; ++i) {
+        if (sizes) sizes[i] = sz[i];
+        total += round256(sz[i]);
+    }
+    return total;
+}
+
+size_t spark_cache_bytes(int B, int Hkv, int S, int D, int T, int dtype) {
+    return spark_cache_sizes(B, Hkv, S, D, T, dtype, nullptr);
+}
+
+size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D, int T, int n_tail) {
+    if (B < 0 || Hkv < 0 || S < 0 || D != kD || T < 0 || T > D || G < 1 || n_tail < 0) return 0;
+    const long BH = (long)B * Hkv;
+    if (op == SPARK_OP_PRUNE) return round256(prune_workspace(BH, S));
+    if (op == SPARK_OP_DECODE) {
+        if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
+        // the geometry depends on the element size only through the stage
+        // size; take the larger of the two so one workspace serves both
+        const DecodeGeom g2 = decode_geometry(BH, S, T, 2, G, num_sms());
+        const DecodeGeom g4 = decode_geometry(BH, S, T, 4, G, num_sms());
+        const size_t a = decode_workspace(BH, g2, G), b = decode_workspace(BH, g4, G);
+        return round256(a > b ? a : b);
+    }
+    return 0;
+}
+
+int spark_prune(const void *k, const void *q_obs, int G, int W, const spark_kcache *out,
+                void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_cache(out);
+    if (rc != SPARK_OK) return rc;
+    if (G < 1 || W < 1) return SPARK_ERR_ARG;
+    const long BH = (long)out->B * out->Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
+    if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < prune_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_prune(k, q_obs, G, W, *out, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, const void *k_tail,
+                      const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
+                      unsigned long long seed, float *out, void *workspace, size_t ws_bytes,
+                      void *stream) {
+    (void)seed;
+    int rc = check_cache(kc);
+    if (rc != SPARK_OK) return rc;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return G < 1 ? SPARK_ERR_ARG : SPARK_ERR_UNSUPPORTED;
+    if (recovery != SPARK_F_DEGENERATE) {
+        if (recovery == SPARK_F_GAUSSIAN || recovery == SPARK_F_EXPONENTIAL) return SPARK_ERR_UNSUPPORTED;
+        return SPARK_ERR_ARG;
+    }
+    if (tail_cap < 0 || n_tail < 0 || n_tail > tail_cap) return SPARK_ERR_ARG;
+    const long BH = (long)kc->B * kc->Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!q || !aligned16(q) || !out || !aligned16(out)) return SPARK_ERR_ARG;
+    if (kc->S > 0 && (!v || !aligned16(v))) return SPARK_ERR_ARG;
+    if (tail_cap > 0 && (!k_tail || !v_tail || !aligned16(k_tail) || !aligned16(v_tail)))
+        return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    const int es = elem_size(kc->dtype);
+    const DecodeGeom geo = decode_geometry(BH, kc->S, kc->T, es, G, num_sms());
+    if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_decode(q, *kc, v, k_tail, v_tail, tail_cap, n_tail, G, out, workspace, geo,
+                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_tail_append(const void *k_new, const void *v_new, void *k_tail, void *v_tail, int B, int Hkv,
+                      int D, int tail_cap, int slot, int dtype, void *stream) {
+    const int es = elem_size(dtype);
+    if (es == 0 || B < 0 || Hkv < 0) return SPARK_ERR_ARG;
+    if (D != kD) return SPARK_ERR_UNSUPPORTED;
+    if (tail_cap < 1 || slot < 0 || slot >= tail_cap) return SPARK_ERR_ARG;
+    const long BH = (long)B * Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!k_new || !v_new || !k_tail || !v_tail) return SPARK_ERR_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_tail) || !aligned16(v_tail))
+        return SPARK_ERR_ARG;
+    const int row_vec = D * es / 16;
+    tail_append_kernel<<<(unsigned)BH, 32 * ((row_vec + 31) / 32), 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), static_cast<uint4 *>(k_tail),
+        static_cast<uint4 *>(v_tail), row_vec, tail_cap, slot);
+    return cudaGetLastError() == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_device_status(void *workspace, int *status, int clear, void *stream) {
+    if (!workspace || !status) return SPARK_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return SPARK_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SPARK_ERR_CUDA;
+    *status = (word & kDevTimeout) ? SPARK_ERR_TIMEOUT : SPARK_OK;
+    if (clear && word) {
+        if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return SPARK_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return SPARK_ERR_CUDA;
+    }
+    return SPARK_OK;
+}
+
+const char *spark_status_str(int status) {
+    switch (status) {
+    case SPARK_OK: return "ok";
+    case SPARK_ERR_ARG: return "invalid argument";
+    case SPARK_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SPARK_ERR_CUDA: return "CUDA error";
+    case SPARK_ERR_TIMEOUT: return "device-side wait timed out";
+    case SPARK_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,146 @@
+// Internal helpers of the SparK sm_100a library: element access, async bulk
+// copies with mbarrier completion, bounded waits, and the launch geometry
+// that both the entry points and the workspace-size query must agree on.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "spark.h"
+
+namespace spark {
+
+constexpr int kD = 128;               // head dimension the kernels are built for
+constexpr int kMaskWords = kD / 32;   // 128-bit channel mask per token
+constexpr int kWsHeader = 256;        // status word + padding at workspace start
+constexpr uint32_t kDevTimeout = 1u;  // status bit: a bounded wait ran out
+
+// ----------------------------------------------------------------- prune
+constexpr int kPruneThreads = 128;    // 4 lanes per token, 32 tokens per group
+constexpr int kPruneGroups = 8;       // 32-token groups per CTA (256 tokens)
+
+inline int prune_chunks(int S) {
+    const int per = 32 * kPruneGroups;
+    return S > 0 ? (S + per - 1) / per : 0;
+}
+
+inline size_t prune_workspace(long BH, int S) {
+    return kWsHeader + (size_t)BH * (size_t)prune_chunks(S) * 2 * sizeof(double);
+}
+
+// ---------------------------------------------------------------- decode
+constexpr int kDecThreads = 128;
+constexpr int kNT = 64;               // tokens per pipeline tile
+constexpr int kMaxStages = 6;
+
+struct DecodeGeom {
+    int chunk;        // prefix tokens per unit (multiple of kNT)
+    int n_pre;        // prefix units per (row, kv head)
+    int units;        // n_pre + 1 (last unit = dense tail)
+    int nstage;       // pipeline depth
+    int ctas_per_sm;  // occupancy the smem budget was sized for
+    size_t smem;      // dynamic shared memory per CTA
+};
+
+__host__ __device__ inline size_t dec_stage_bytes(int T, int es) {
+    return (size_t)kNT * 16 + (size_t)kNT * T * es + (size_t)kNT * kD * es;
+}
+
+inline size_t dec_fixed_bytes(int G) {
+    // q' table, c table, Qc, p buffer, per-warp maxima, mbarriers, padding
+    return (size_t)kD * G * 4 + kD * 4 + 64 + (size_t)kNT * G * 4 +
+           4 * G * 4 + kMaxStages * 8 + 256;
+}
+
+inline size_t dec_epilogue_bytes(int G) {
+    // per token-subset partial accumulators (8 subsets) and l sums
+    return (size_t)8 * G * kD * 4 + (size_t)8 * G * 4;
+}
+
+DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms);
+
+inline size_t decode_workspace(long BH, const DecodeGeom &g, int G) {
+    return kWsHeader + (size_t)BH * g.units * G * (kD + 2) * sizeof(float);
+}
+
+// ------------------------------------------------------- element access
+template <typename E> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float to_f(float x) { return x; }
+    static constexpr int size = 4;
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static constexpr int size = 2;
+};
+
+// ------------------------------------------------------------- PTX glue
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after ~1 s of device
+// time.  Returns false on timeout (the caller records it and winds down).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 0; it < (1u << 26); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u && global_ns() - t0 > 1000000000ull) return false;
+    }
+    return false;
+}
+
+// Async bulk copy global -> shared, completion counted on `bar` (bytes).
+// Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// order-preserving float <-> int map for integer warp max reductions
+__device__ __forceinline__ int f2ord(float f) {
+    int i = __float_as_int(f);
+    return i ^ ((i >> 31) & 0x7fffffff);
+}
+__device__ __forceinline__ float ord2f(int i) {
+    return __int_as_float(i ^ ((i >> 31) & 0x7fffffff));
+}
+
+}  // namespace spark

@@ -1,0 +1,185 @@
+/*
+ * spark.h -- C ABI of a B200 (sm_100a) library for SparK: query-aware,
+ * unstructured key-cache channel pruning at prefill and recover-then-attend
+ * decode attention over the pruned cache.
+ *
+ * Method sources (web pages on SparK, arXiv 2508.15212):
+ *   [W]  "KV Cache 还能再砍一刀：SparK 在通道维度上做了一件被忽略多年的事"
+ *        (paper walkthrough): section 1 (KV size 2*B*S*L*N*D), 3.1 (pruning
+ *        objective, its channel-independent relaxation and the proxy
+ *        saliency w = ||q^j||_2 * ||k^j||_2 solved by greedy top-T), 3.2
+ *        (observation-window queries), 3.3 (cache = pruned key + mask +
+ *        score statistics; recovery F samples a score and back-solves
+ *        k~ = w~ / ||q^j||_2; F table: Degenerate / Gaussian / Exponential),
+ *        Fig. 3 (prefill prunes, decode recovers then runs full attention).
+ *   [A]  "AAAI 2026 AMD论文Spark方法揭秘" (AMD blog): lambda is the fraction of
+ *        key channels pruned; decode runs standard full attention.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees, synchronises or prints.  Every launch
+ *     is asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - Tensors are dense row-major; pointers must be 16-byte aligned.
+ *   - dtype: SPARK_F32 (fp32) or SPARK_BF16 (bf16) for keys, values and
+ *     queries.  D must be 128.  Saliency, norms and attention arithmetic run
+ *     in fp32 (norm accumulated in fp64), statistics in fp64.
+ *   - Argument errors are returned synchronously (SPARK_ERR_ARG,
+ *     SPARK_ERR_UNSUPPORTED, SPARK_ERR_WORKSPACE) and nothing is launched.
+ *     A failed launch returns SPARK_ERR_CUDA.  Errors detected on the device
+ *     (a bounded wait that ran out) set a sticky bit in the first 4 bytes of
+ *     the workspace; read it with spark_device_status().
+ *   - "B" is the flattened batch: callers with L layers pass B*L rows.
+ *     Query head g of kv head h is head h*G + g (consecutive GQA groups).
+ */
+#ifndef SPARK_H
+#define SPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPARK_API __attribute__((visibility("default")))
+#else
+#define SPARK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPARK_OK = 0,
+    SPARK_ERR_ARG = 1,          /* bad pointer, size, alignment or shape      */
+    SPARK_ERR_UNSUPPORTED = 2,  /* valid request this build does not run      */
+    SPARK_ERR_CUDA = 3,         /* a CUDA call failed (launch, attribute)     */
+    SPARK_ERR_TIMEOUT = 4,      /* device-side bounded wait ran out           */
+    SPARK_ERR_WORKSPACE = 5     /* workspace NULL, misaligned or too small    */
+} spark_status;
+
+typedef enum { SPARK_F32 = 0, SPARK_BF16 = 1 } spark_dtype;
+
+/* Recovery function F of [W] 3.3 (F table). */
+typedef enum {
+    SPARK_F_DEGENERATE = 0,   /* w~ = mu_pruned                              */
+    SPARK_F_GAUSSIAN = 1,     /* w~ ~ N(mu, sigma^2)   (not built: UNSUPPORTED) */
+    SPARK_F_EXPONENTIAL = 2   /* w~ ~ Exp(1/mu)        (not built: UNSUPPORTED) */
+} spark_recovery;
+
+typedef enum { SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1 } spark_op;
+
+/*
+ * The packed key cache of [W] 3.3 step 1 / Fig. 3: per token the kept key
+ * values and a channel mask; per (row, kv head) the window-query channel
+ * norms and the statistics of the pruned saliencies.  All device memory,
+ * owned by the caller, sized with spark_cache_sizes().
+ *
+ *   mask  uint32 [B][Hkv][S][4]: bit (j % 32) of word (j / 32) is set iff
+ *         channel j of that token is kept.  Exactly T bits per token.
+ *   vals  dtype, per (b, h) a block of S32*T elements (S32 = S rounded up
+ *         to a multiple of 32), grouped by 32 tokens: kept value i (in
+ *         ascending channel order) of token t sits at element
+ *         ((t / 32) * T + i) * 32 + (t % 32) of the block.  Slots of the
+ *         padding tokens t >= S are unspecified.
+ *   qn    fp32 [B][Hkv][D]: window-query channel norm (see spark_prune).
+ *   stats fp64 [B][Hkv][4]: {N_pruned, sum w, sum w^2, mu_pruned} over the
+ *         pruned (token, channel) entries of that head; mu = 0 when N = 0.
+ */
+typedef struct spark_kcache {
+    int B, Hkv, S, D, T, dtype;
+    uint32_t *mask;
+    void *vals;
+    float *qn;
+    double *stats;
+} spark_kcache;
+
+/* Kept channels for pruning ratio lambda ([A] Table 1 caption, [W] 4.1):
+ * T = round((1 - lambda) * D), halves away from zero, in fp64.
+ * Returns -1 when lambda is outside [0, 1] (or NaN) or D <= 0. */
+SPARK_API int spark_lambda_to_T(float lambda, int D);
+
+/* Byte sizes of the four cache regions {mask, vals, qn, stats} (written to
+ * sizes[0..3]) and their total when packed back to back at 256-byte
+ * aligned offsets (the return value).  Returns 0 on bad arguments.
+ * The pages' dense KV size is 2*B*S*L*N*D elements ([W] 1); the pruned key
+ * cache replaces the key half by 16 + T*es bytes per token-head. */
+SPARK_API size_t spark_cache_sizes(int B, int Hkv, int S, int D, int T, int dtype,
+                         size_t sizes[4]);
+
+/* Total bytes of the packed cache (same as spark_cache_sizes' return). */
+SPARK_API size_t spark_cache_bytes(int B, int Hkv, int S, int D, int T, int dtype);
+
+/* Workspace bytes that `op` needs for the given shape (device memory,
+ * 256-byte aligned, caller-owned; its first 4 bytes hold the device status
+ * word and must be zero before first use).  For SPARK_OP_DECODE pass the
+ * tail capacity as n_tail.  Depends on the current device's SM count.
+ * Returns 0 on bad arguments. */
+SPARK_API size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D,
+                             int T, int n_tail);
+
+/*
+ * Prefill channel pruning ([W] 3.1, 3.2, 3.3 step 1).
+ *   k      [B][Hkv][S][D] dtype    prompt keys (post-RoPE)
+ *   q_obs  [B][Hkv*G][W][D] dtype  observation-window queries
+ *   out    cache descriptor; out->B, Hkv, S, D, T, dtype select the shape
+ *          and out->mask/vals/qn/stats receive the result.
+ * Computes
+ *   qn[b,h,j] = sqrt(sum_{g<G} sum_{t<W} q_obs[b,h*G+g,t,j]^2)   (fp64 sum of
+ *               the squares in (g, t) order, rounded once to fp32)
+ *   w[t,j]    = qn[b,h,j] * |k[b,h,t,j]|                          (one fp32 mul)
+ * keeps, per token, the T channels of largest w (ties -> lower channel),
+ * writes mask and the kept values (bit-exact copies of k), and reduces
+ * N = S*(D-T), sum w and sum w^2 over the pruned entries and
+ * mu_pruned = sum w / N into stats.
+ * Requires D == 128, 0 <= T <= 128, G >= 1, W >= 1, S >= 0 and a
+ * workspace of spark_workspace_bytes(SPARK_OP_PRUNE, ...) bytes.
+ * Inputs with NaN or infinity give unspecified masks.
+ */
+SPARK_API int spark_prune(const void *k, const void *q_obs, int G, int W,
+                const spark_kcache *out, void *workspace, size_t ws_bytes,
+                void *stream);
+
+/*
+ * Decode attention over the pruned cache plus a dense tail ([W] 3.3 steps
+ * 2-4, Fig. 3, [A]).
+ *   q       [B][Hkv*G][D] dtype       this step's queries
+ *   kc      the cache written by spark_prune
+ *   v       [B][Hkv][S][D] dtype      prompt values (dense, unpruned)
+ *   k_tail, v_tail  [B][Hkv][tail_cap][D] dtype  keys/values appended at
+ *           decode time (never pruned); the first n_tail rows are used.
+ *           May be NULL when tail_cap == 0.
+ *   out     [B][Hkv*G][D] fp32
+ * For each query head: the pruned channels of every prefix token are
+ * rebuilt by F (Degenerate: k~_j = mu_pruned / qn_j, 0 when qn_j == 0),
+ * then out = softmax(q . K~^T / sqrt(D)) V over prefix + tail, a split-K
+ * (flash-decoding) pass followed by a log-sum-exp combine.  An empty
+ * context (S + n_tail == 0) gives zeros.  `seed` is reserved for the
+ * sampling recoveries.  Requires the decode workspace size for tail_cap.
+ */
+SPARK_API int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v,
+                      const void *k_tail, const void *v_tail, int tail_cap,
+                      int n_tail, int G, int recovery, unsigned long long seed,
+                      float *out, void *workspace, size_t ws_bytes,
+                      void *stream);
+
+/*
+ * Append one unpruned decode-time key/value per (row, kv head) into the
+ * dense tail at row `slot` (configs that "append unpruned new keys").
+ *   k_new, v_new [B][Hkv][D] dtype;  k_tail, v_tail [B][Hkv][tail_cap][D].
+ * Requires 0 <= slot < tail_cap and D == 128.
+ */
+SPARK_API int spark_tail_append(const void *k_new, const void *v_new, void *k_tail,
+                      void *v_tail, int B, int Hkv, int D, int tail_cap,
+                      int slot, int dtype, void *stream);
+
+/* Synchronise `stream`, read the device status word at the start of
+ * `workspace` into *status (SPARK_OK or SPARK_ERR_TIMEOUT) and, when
+ * clear != 0, reset it to zero.  Returns SPARK_ERR_CUDA if a copy fails. */
+SPARK_API int spark_device_status(void *workspace, int *status, int clear, void *stream);
+
+/* Static description of a status code. */
+SPARK_API const char *spark_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPARK_H */

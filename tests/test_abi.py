@@ -1,0 +1,149 @@
+"""Host-side checks of the C ABI library (no GPU needed): it builds and
+loads, exports exactly what include/spark.h declares, and its host logic
+(lambda -> T, cache layout sizes, workspace sizes, argument validation)
+behaves as documented.  No compute call is made."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from channel_pruned_decode_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spark.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from channel_pruned_decode_b200 import build
+    build.build()
+    return B.lib()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return set(re.findall(r"SPARK_API\s+[\w\s\*]*?\b(spark_\w+)\s*\(", txt))
+
+
+def test_exports_match_header(L):
+    decl = _declared()
+    assert decl == set(B.EXPORTS)
+    for name in decl:
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", B._LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln and "spark" in ln}
+    assert exported == decl
+
+
+@pytest.mark.parametrize("lam", [0.0, 0.1, 0.25, 0.3, 0.5, 0.58, 0.8, 0.9, 1.0, -0.01, 1.01])
+def test_lambda_to_T_matches_oracle(L, lam):
+    assert B.spark_lambda_to_T(lam, 128) == oracle.lambda_to_T(lam, 128)
+
+
+def test_cache_sizes_layout():
+    for (b, h, s, t, dt, es) in [(1, 8, 32768, 64, B.SPARK_BF16, 2), (2, 2, 513, 26, B.SPARK_F32, 4),
+                                 (1, 1, 0, 0, B.SPARK_BF16, 2)]:
+        total, sz = B.spark_cache_sizes(b, h, s, 128, t, dt)
+        s32 = (s + 31) // 32 * 32
+        assert sz == [b * h * s * 16, b * h * s32 * t * es, b * h * 128 * 4, b * h * 32]
+        assert total == sum((x + 255) // 256 * 256 for x in sz)
+        assert B.spark_cache_bytes(b, h, s, 128, t, dt) == total
+    assert B.spark_cache_bytes(1, 1, 16, 64, 8, B.SPARK_BF16) == 0       # D != 128
+    assert B.spark_cache_bytes(1, 1, 16, 128, 129, B.SPARK_BF16) == 0    # T > D
+    assert B.spark_cache_bytes(1, 1, 16, 128, 8, 7) == 0                 # dtype
+
+
+def test_storage_reduction_arithmetic():
+    # key bytes per token-head: 16-byte mask + T kept bf16 values vs 256 dense.
+    # lambda 0.5 -> 144 B (43.75 % smaller key, 21.9 % smaller K+V);
+    # lambda 0.8 -> 68 B (73.4 % smaller key, 36.7 % smaller K+V) -- the pages
+    # quote ~50 % key / ~25 % total and ~40 % total without the mask overhead.
+    S = 1 << 15
+    for lam, key_red, kv_red in [(0.5, 0.4375, 0.21875), (0.8, 0.734375, 0.3671875)]:
+        T = B.spark_lambda_to_T(lam, 128)
+        _, sz = B.spark_cache_sizes(1, 1, S, 128, T, B.SPARK_BF16)
+        per_tok = (sz[0] + sz[1]) / S
+        assert 1 - per_tok / 256 == pytest.approx(key_red)
+        assert 1 - (per_tok + 256) / 512 == pytest.approx(kv_red)
+
+
+def test_workspace_sizes():
+    assert B.spark_workspace_bytes(B.SPARK_OP_PRUNE, 1, 8, 4, 32768, 128, 64, 0) >= 256 + 8 * 128 * 16
+    assert B.spark_workspace_bytes(B.SPARK_OP_DECODE, 1, 8, 4, 32768, 128, 64, 256) > 256
+    assert B.spark_workspace_bytes(B.SPARK_OP_DECODE, 1, 8, 3, 32768, 128, 64, 256) == 0  # G
+    assert B.spark_workspace_bytes(B.SPARK_OP_PRUNE, 1, 8, 4, 32768, 96, 64, 0) == 0      # D
+    assert B.spark_workspace_bytes(9, 1, 8, 4, 32768, 128, 64, 0) == 0                   # op
+
+
+def _kc(**kw):
+    d = dict(B=1, Hkv=2, S=64, D=128, T=32, dtype=B.SPARK_BF16, mask=16, vals=16, qn=16, stats=16)
+    d.update(kw)
+    return B.spark_kcache(**d)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(D=64), B.SPARK_ERR_UNSUPPORTED),
+    (dict(T=129), B.SPARK_ERR_ARG),
+    (dict(T=-1), B.SPARK_ERR_ARG),
+    (dict(dtype=5), B.SPARK_ERR_ARG),
+    (dict(mask=None), B.SPARK_ERR_ARG),
+    (dict(vals=24), B.SPARK_ERR_ARG),   # misaligned
+    (dict(S=-1), B.SPARK_ERR_ARG),
+])
+def test_prune_rejects_bad_cache(L, kw, want):
+    kc = _kc(**kw)
+    rc = L.spark_prune(16, 16, 4, 32, ctypes.byref(kc), 256, 1 << 20, None)
+    assert rc == want
+
+
+def test_prune_rejects_bad_args(L):
+    kc = _kc()
+    assert L.spark_prune(16, 16, 0, 32, ctypes.byref(kc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert L.spark_prune(16, 16, 4, 0, ctypes.byref(kc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert L.spark_prune(None, 16, 4, 32, ctypes.byref(kc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert L.spark_prune(16, 16, 4, 32, ctypes.byref(kc), None, 1 << 20, None) == B.SPARK_ERR_WORKSPACE
+    assert L.spark_prune(16, 16, 4, 32, ctypes.byref(kc), 256, 16, None) == B.SPARK_ERR_WORKSPACE
+    assert L.spark_prune(16, 16, 4, 32, None, 256, 1 << 20, None) == B.SPARK_ERR_ARG
+
+
+def test_decode_rejects_bad_args(L):
+    kc = _kc()
+    call = lambda **k: L.spark_decode_attn(
+        k.get("q", 16), ctypes.byref(kc), k.get("v", 16), k.get("kt", 16), k.get("vt", 16),
+        k.get("cap", 8), k.get("n", 0), k.get("G", 4), k.get("rec", 0), 0, k.get("out", 16),
+        k.get("ws", 256), 1 << 20, None)
+    assert call(G=3) == B.SPARK_ERR_UNSUPPORTED
+    assert call(G=0) == B.SPARK_ERR_ARG
+    assert call(rec=B.SPARK_F_GAUSSIAN) == B.SPARK_ERR_UNSUPPORTED
+    assert call(rec=9) == B.SPARK_ERR_ARG
+    assert call(n=9) == B.SPARK_ERR_ARG          # n_tail > tail_cap
+    assert call(cap=-1) == B.SPARK_ERR_ARG
+    assert call(q=None) == B.SPARK_ERR_ARG
+    assert call(out=8) == B.SPARK_ERR_ARG        # misaligned
+    assert call(kt=None) == B.SPARK_ERR_ARG      # tail_cap > 0 needs tail buffers
+    assert call(ws=None) == B.SPARK_ERR_WORKSPACE
+
+
+def test_tail_append_rejects_bad_args(L):
+    f = L.spark_tail_append
+    assert f(16, 16, 16, 16, 1, 2, 64, 8, 0, B.SPARK_BF16, None) == B.SPARK_ERR_UNSUPPORTED
+    assert f(16, 16, 16, 16, 1, 2, 128, 8, 8, B.SPARK_BF16, None) == B.SPARK_ERR_ARG   # slot
+    assert f(16, 16, 16, 16, 1, 2, 128, 0, 0, B.SPARK_BF16, None) == B.SPARK_ERR_ARG   # cap
+    assert f(None, 16, 16, 16, 1, 2, 128, 8, 0, B.SPARK_BF16, None) == B.SPARK_ERR_ARG
+    assert f(16, 16, 16, 16, 1, 2, 128, 8, 0, 3, None) == B.SPARK_ERR_ARG
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert B.status_str(s)
+    assert B.status_str(99) == "unknown status"
+
+
+def test_empty_batch_is_a_no_op(L):
+    kc = _kc(B=0)
+    assert L.spark_prune(None, None, 4, 32, ctypes.byref(kc), None, 0, None) == B.SPARK_OK
