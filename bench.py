@@ -74,6 +74,8 @@ class ClockSampler:
         self.path = None
         try:
             bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            dom, rest = bus.split(":", 1)
+            bus = dom.zfill(8) + ":" + rest  # nvidia-smi's 8-digit PCI domain form
         except Exception:
             bus = str(device_index)
         self.bus = bus
@@ -249,6 +251,8 @@ def run_gpu(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     wl = WORKLOADS[args.workload]
+    if args.layers:
+        wl = scaled(wl, L=args.layers)
     job = Job(wl, dev)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -441,6 +445,7 @@ def main():
     ap.add_argument("--impl", default="spark", choices=["spark", "reference"])
     ap.add_argument("--workload", default="long", choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
