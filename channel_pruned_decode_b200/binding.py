@@ -29,7 +29,7 @@ SPARK_OP_PRUNE = 0
 SPARK_OP_DECODE = 1
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
-           "spark_prune", "spark_decode_attn", "spark_tail_append", "spark_device_status",
+           "spark_prune", "spark_prune_noalloc", "spark_decode_attn", "spark_tail_append", "spark_device_status",
            "spark_status_str")
 
 
@@ -67,6 +67,8 @@ def lib():
         L.spark_workspace_bytes.restype = Z
         L.spark_prune.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P, Z, P]
         L.spark_prune.restype = I
+        L.spark_prune_noalloc.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P]
+        L.spark_prune_noalloc.restype = I
         L.spark_decode_attn.argtypes = [P, ctypes.POINTER(spark_kcache), P, P, P, I, I, I, I,
                                         ctypes.c_ulonglong, P, P, Z, P]
         L.spark_decode_attn.restype = I
@@ -173,6 +175,15 @@ def spark_prune(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, kc: KCache
     rc = lib().spark_prune(_ptr(k), _ptr(q_obs), G, W, ctypes.byref(s), _ptr(ws),
                            ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_prune")
+
+
+def spark_prune_noalloc(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, kc: KCache,
+                        stream=None) -> None:
+    """spark_prune for callers that cannot allocate a workspace: the library's
+    fixed 4 MiB per-device scratch array stands in for it (see spark.h)."""
+    s = kc.struct()
+    rc = lib().spark_prune_noalloc(_ptr(k), _ptr(q_obs), G, W, ctypes.byref(s), _stream(stream))
+    _check(rc, "spark_prune_noalloc")
 
 
 def spark_decode_attn(q: torch.Tensor, kc: KCache, v: torch.Tensor, k_tail, v_tail, tail_cap: int,

@@ -139,6 +139,32 @@ SPARK_API int spark_prune(const void *k, const void *q_obs, int G, int W,
                 void *stream);
 
 /*
+ * spark_prune without a workspace.  Not part of the SparK method: the paper
+ * has no counterpart; this is a calling convention for this library.
+ *
+ * For callers that cannot allocate device memory where they prune -- e.g. a
+ * serving engine whose memory pool owns the whole device after start-up and
+ * forbids allocations on the request path, or a plugin host that hands an op
+ * only its input and output buffers.  Computes exactly what spark_prune
+ * computes, with the same arguments minus the workspace; the caller still
+ * owns k, q_obs and every cache buffer.
+ *
+ * Scratch: a 4 MiB array in device memory that every GPU loading this
+ * library holds until the process exits.  The call needs
+ * 256 + 16 * B * Hkv * ceil(S / 256) bytes of it and returns
+ * SPARK_ERR_WORKSPACE (launching nothing) when that exceeds 4 MiB, i.e.
+ * when B * Hkv * ceil(S / 256) > 262128.
+ * The first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (that device must be current); make that first call
+ * before any stream capture.  All calls share the array and it keeps the
+ * last call's contents (every value a call reads it writes first), so calls
+ * whose kernels overlap on the GPU -- on different streams, or from several
+ * host threads -- race and must be serialised by the caller.
+ */
+SPARK_API int spark_prune_noalloc(const void *k, const void *q_obs, int G, int W,
+                                  const spark_kcache *out, void *stream);
+
+/*
  * Decode attention over the pruned cache plus a dense tail ([W] 3.3 steps
  * 2-4, Fig. 3, [A]).
  *   q       [B][Hkv*G][D] dtype       this step's queries
