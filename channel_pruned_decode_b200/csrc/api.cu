@@ -142,6 +142,7 @@ int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, cons
     if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
     const int es = elem_size(kc->dtype);
     const DecodeGeom geo = decode_geometry(BH, kc->S, kc->T, es, G, num_sms());
+    if (BH * (long)geo.units >= (1L << 31)) return SPARK_ERR_UNSUPPORTED;  // 32-bit item indices
     if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
     cudaError_t e = launch_decode(q, *kc, v, k_tail, v_tail, tail_cap, n_tail, G, out, workspace, geo,
                                   static_cast<cudaStream_t>(stream));

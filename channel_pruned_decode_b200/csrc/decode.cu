@@ -4,7 +4,7 @@
 // steps 2-4 and the F table (Degenerate: the sampled score is mu_pruned and
 // the key is back-solved as k~_j = mu_pruned / ||q^j||_2), Fig. 3 (decode runs
 // standard full attention over the recovered keys); AMD blog "AAAI 2026
-// AMD论文Spark方法揭秘" (same).  Flash-decoding split-K with a log-sum-exp
+// AMD论文Spark方法揭秘" (same).  Split-K flash decoding with a log-sum-exp
 // combine is the standard way to run that attention on one GPU.
 //
 // Score algebra.  With c_j = mu / qn_j (0 when qn_j = 0) the recovered key is
@@ -14,17 +14,24 @@
 // the T kept values, which is all the cache holds.  Identical to the dense
 // recover-then-attend form in real arithmetic; fp32 rounding differs.
 //
-// decode_kernel: one CTA per (unit, row, kv head).  Units 0..n_pre-1 each own
-// a contiguous chunk of prompt tokens; unit n_pre owns the dense tail.  A
-// prompt chunk is streamed in 64-token tiles by cp.async.bulk copies
-// (mask 16 B/token, interleaved kept values T*es B/token, dense V 256 B/token)
-// into an nstage-deep shared-memory ring completed on mbarriers, with bounded
-// waits.  Per tile: two threads per token walk the set bits of their 64-bit
-// half of the mask and accumulate q'_g (k_j - c_j) for the G heads of the
-// group (q' pre-scaled by log2(e)/sqrt(D)); a CTA-wide max updates the running
-// max; p = 2^(s - m) goes to shared memory; then 16 channel-groups x 8 token
-// subsets accumulate p * V in fp32.  Each unit writes (acc[G][D], m, l).
-// combine_kernel merges the units of a (row, head) in a fixed order.
+// decode_kernel: a persistent grid, one CTA per SM, whose warps are
+// independent flash-decoding workers.  Work items are (row, kv head, chunk of
+// prompt tokens) plus one dense-tail item per head; warp w of the grid takes
+// items w, w + #warps, ...  Each warp streams its items' 32-token tiles: the
+// mask (16 B/token) and one 32-token group of interleaved kept values
+// (T*es B/token) by cp.async.bulk copies, issued by its lane 0 into its own
+// ring of shared-memory stages and completed on per-stage mbarriers (bounded
+// waits); the dense V rows (256 B/token) by coalesced 8-byte loads straight
+// into registers, issued before the tile's q.k~ so that they land under it.
+// No CTA-wide barrier is on the path.  Per tile:
+//   q.k~     lane = token; the lane walks exactly T set bits of its 128-bit
+//            mask and accumulates q'_g (k_j - c_j) for the G heads of the
+//            group from the q' / c tables (q' = q * log2(e)/sqrt(D));
+//   softmax  warp max (integer REDUX on an order-preserving map) updates the
+//            running max; p = 2^(s - m) goes to shared memory as fp32 pairs;
+//   P.V      lane = 4 value channels; packed fp32x2 FMAs over the tokens.
+// At the end of an item the warp writes (acc[G][D], m, l) for it;
+// combine_kernel merges a head's items in a fixed order.
 #include "spark_internal.cuh"
 
 #include <algorithm>
@@ -40,8 +47,10 @@ struct DecArgs {
     const void *v;
     const void *k_tail;
     const void *v_tail;
-    float *part;       // [BH][units][G][D + 2]: acc[D], m, l
+    float *acc;        // [BH][units][G][D]
+    float *ml;         // [BH][units][G][2]
     uint32_t *status;  // device status word
+    long BH;
     int S;
     long S32;
     int T;
@@ -51,27 +60,61 @@ struct DecArgs {
     int n_pre;
     int units;
     int nstage;
+    int nwarp;
+    size_t warp_bytes;
 };
 
-// 8 consecutive channels of a V (or K) row as fp32
-template <typename E> struct Row8;
-template <> struct Row8<__nv_bfloat16> {
-    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&x)[8]) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(p);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            x[2 * i] = __uint_as_float(w[i] << 16);
-            x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-        }
+// log2(e) / sqrt(128): folds the softmax scale and the exp -> exp2 change
+// into the query.
+constexpr float kQScale = 0.12751743074602467f;
+
+// 4 consecutive channels of a key row (dense tail) as fp32
+template <typename E> struct Row4;
+template <> struct Row4<__nv_bfloat16> {
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&x)[4]) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        x[0] = __uint_as_float(u.x << 16);
+        x[1] = __uint_as_float(u.x & 0xffff0000u);
+        x[2] = __uint_as_float(u.y << 16);
+        x[3] = __uint_as_float(u.y & 0xffff0000u);
     }
 };
-template <> struct Row8<float> {
-    __device__ __forceinline__ static void load(const float *p, float (&x)[8]) {
+template <> struct Row4<float> {
+    __device__ __forceinline__ static void load(const float *p, float (&x)[4]) {
         const float4 a = *reinterpret_cast<const float4 *>(p);
-        const float4 b = *reinterpret_cast<const float4 *>(p + 4);
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+};
+
+// This lane's 4 value channels of a batch of consecutive tokens, in
+// registers: 32 tokens for bf16, 16 for fp32 (64 registers either way).
+template <typename E> struct VRegs;
+template <> struct VRegs<__nv_bfloat16> {
+    static constexpr int kTok = 32;
+    uint2 v[kTok];
+    // row0 points at channel 4*lane of the batch's first token
+    __device__ __forceinline__ void load(const __nv_bfloat16 *row0, int n) {
+#pragma unroll
+        for (int t = 0; t < kTok; ++t)
+            v[t] = (t < n) ? __ldcs(reinterpret_cast<const uint2 *>(row0 + (size_t)t * kD)) : make_uint2(0u, 0u);
+    }
+    __device__ __forceinline__ void get(int t, float2 &x01, float2 &x23) const {
+        x01 = make_float2(__uint_as_float(v[t].x << 16), __uint_as_float(v[t].x & 0xffff0000u));
+        x23 = make_float2(__uint_as_float(v[t].y << 16), __uint_as_float(v[t].y & 0xffff0000u));
+    }
+};
+template <> struct VRegs<float> {
+    static constexpr int kTok = 16;
+    float4 v[kTok];
+    __device__ __forceinline__ void load(const float *row0, int n) {
+#pragma unroll
+        for (int t = 0; t < kTok; ++t)
+            v[t] = (t < n) ? __ldcs(reinterpret_cast<const float4 *>(row0 + (size_t)t * kD))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __device__ __forceinline__ void get(int t, float2 &x01, float2 &x23) const {
+        x01 = make_float2(v[t].x, v[t].y);
+        x23 = make_float2(v[t].z, v[t].w);
     }
 };
 
@@ -94,336 +137,407 @@ template <int G> struct QVec {
     }
 };
 
-// log2(e) / sqrt(128): folds the softmax scale and the exp -> exp2 change
-// into the query.
-constexpr float kQScale = 0.12751743074602467f;
-
+// Per-warp shared memory: tables, p buffer, mbarriers, then the stage ring.
 template <typename E, int G>
-struct Smem {
-    float *tabq;   // [kD][G]
-    float *tabc;   // [kD]
-    float *qc;     // [G] (16 floats reserved)
-    float *pbuf;   // [kNT][G]
-    float *wmax;   // [4][G]
+struct WarpSmem {
+    float *tabq;   // [kD][G]   q' per channel
+    float *tabc;   // [kD]      c_j = mu / qn_j
+    float *pdup;   // [kWT][G][2] p duplicated into fp32 pairs
+    float *qc;     // [G] Qc = sum_j q'_j c_j of the current head
     uint64_t *bars;
     unsigned char *stages;
-    size_t stage_bytes;
-    int T;
-    __device__ __forceinline__ uint32_t *smask(int st) const {
-        return reinterpret_cast<uint32_t *>(stages + (size_t)st * stage_bytes);
+    uint32_t stage_bytes;
+    __device__ __forceinline__ const uint32_t *smask(int st) const {
+        return reinterpret_cast<const uint32_t *>(stages + (size_t)st * stage_bytes);
     }
-    __device__ __forceinline__ E *svals(int st) const {
-        return reinterpret_cast<E *>(stages + (size_t)st * stage_bytes + kNT * 16);
-    }
-    __device__ __forceinline__ E *sV(int st) const {
-        return reinterpret_cast<E *>(stages + (size_t)st * stage_bytes + kNT * 16 +
-                                     (size_t)kNT * T * sizeof(E));
+    __device__ __forceinline__ const E *svals(int st) const {
+        return reinterpret_cast<const E *>(stages + (size_t)st * stage_bytes + kWT * 16);
     }
 };
 
-// One tile's softmax update + P.V accumulation, shared by the prompt and the
-// tail paths.  s[] holds this thread's token scores (thread pair per token,
-// both halves hold the same sums).  Returns false when the CTA must stop.
-template <typename E, int G, typename VRow>
-__device__ __forceinline__ void softmax_pv(const Smem<E, G> &sm, const float (&s)[G], int n,
-                                           float (&m_run)[G], float (&acc)[G][8], float (&lsum)[G],
-                                           VRow vrow) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tt = tid >> 1, h = tid & 1;
+// flash-decoding state of one warp for the item in progress
+template <int G>
+struct Flash {
+    float m[G];       // running max (log2 domain), warp-uniform
+    float l[G];       // this lane's share of the running sum
+    float2 acc[G][2]; // this lane's 4 value channels, as fp32 pairs
+    __device__ __forceinline__ void reset() {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const int mx = __reduce_max_sync(0xffffffffu, f2ord(s[g]));
-        if (lane == 0) sm.wmax[warp * G + g] = ord2f(mx);
+        for (int g = 0; g < G; ++g) {
+            m[g] = -INFINITY;
+            l[g] = 0.f;
+            acc[g][0] = make_float2(0.f, 0.f);
+            acc[g][1] = make_float2(0.f, 0.f);
+        }
     }
-    __syncthreads();
-    float alpha[G];
+};
+
+// Online-softmax update for one tile: s[] is this lane's token score (-inf
+// for lanes past the tile end).  Leaves p (duplicated pairs) in shared
+// memory and rescales the accumulators when the running max moved.
+template <typename E, int G>
+__device__ __forceinline__ void tile_softmax(const WarpSmem<E, G> &ws, Flash<G> &f, const float (&s)[G]) {
+    const int lane = threadIdx.x & 31;
+    float alpha[G], p[G];
     bool rescale = false;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        float mt = sm.wmax[g];
-#pragma unroll
-        for (int w = 1; w < kDecThreads / 32; ++w) mt = fmaxf(mt, sm.wmax[w * G + g]);
-        const float m_new = fmaxf(m_run[g], mt);
-        alpha[g] = (m_new == -INFINITY) ? 1.f : exp2f(m_run[g] - m_new);
+        const float mt = ord2f(__reduce_max_sync(0xffffffffu, f2ord(s[g])));
+        const float m_new = fmaxf(f.m[g], mt);
+        alpha[g] = (m_new == -INFINITY) ? 1.f : exp2f(f.m[g] - m_new);
         rescale |= (alpha[g] != 1.f);
-        m_run[g] = m_new;
+        f.m[g] = m_new;
+        p[g] = (m_new == -INFINITY) ? 0.f : exp2f(s[g] - m_new);
+        f.l[g] = fmaf(f.l[g], alpha[g], p[g]);
     }
-    if (h == 0) {
+    float *pd = ws.pdup + lane * G * 2;
+    if constexpr (G == 1) {
+        *reinterpret_cast<float2 *>(pd) = make_float2(p[0], p[0]);
+    } else {
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-            sm.pbuf[tt * G + g] = (m_run[g] == -INFINITY) ? 0.f : exp2f(s[g] - m_run[g]);
+        for (int g = 0; g < G; g += 2)
+            *reinterpret_cast<float4 *>(pd + 2 * g) = make_float4(p[g], p[g], p[g + 1], p[g + 1]);
     }
-    __syncthreads();
     if (rescale) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            lsum[g] *= alpha[g];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[g][c] *= alpha[g];
+            const float2 a2 = make_float2(alpha[g], alpha[g]);
+            f.acc[g][0] = __fmul2_rn(f.acc[g][0], a2);
+            f.acc[g][1] = __fmul2_rn(f.acc[g][1], a2);
         }
     }
-    const int cg = tid & 15, ts = tid >> 4;
-#pragma unroll 2
-    for (int kk = 0; kk < kNT / 8; ++kk) {
-        const int t2 = ts * (kNT / 8) + kk;
-        if (t2 < n) {
-            QVec<G> p;
-            p.load(sm.pbuf + t2 * G);
-            float x[8];
-            Row8<E>::load(vrow(t2) + 8 * cg, x);
+    __syncwarp();
+}
+
+// P.V over tokens [t_lo, t_lo + VRegs::kTok) of the tile (those < n), V rows
+// from registers, p from shared memory.
+template <typename E, int G>
+__device__ __forceinline__ void tile_pv(const WarpSmem<E, G> &ws, Flash<G> &f, const VRegs<E> &vr, int t_lo,
+                                        int n) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                lsum[g] += p.v[g];
+    for (int t = 0; t < VRegs<E>::kTok; ++t) {
+        if (t_lo + t < n) {
+            float2 x01, x23;
+            vr.get(t, x01, x23);
+            const float *pd = ws.pdup + (t_lo + t) * G * 2;
+            if constexpr (G == 1) {
+                const float2 pp = *reinterpret_cast<const float2 *>(pd);
+                f.acc[0][0] = __ffma2_rn(pp, x01, f.acc[0][0]);
+                f.acc[0][1] = __ffma2_rn(pp, x23, f.acc[0][1]);
+            } else {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[g][c] = fmaf(p.v[g], x[c], acc[g][c]);
+                for (int g = 0; g < G; g += 2) {
+                    const float4 pp = *reinterpret_cast<const float4 *>(pd + 2 * g);
+                    const float2 pa = make_float2(pp.x, pp.y), pb = make_float2(pp.z, pp.w);
+                    f.acc[g][0] = __ffma2_rn(pa, x01, f.acc[g][0]);
+                    f.acc[g][1] = __ffma2_rn(pa, x23, f.acc[g][1]);
+                    f.acc[g + 1][0] = __ffma2_rn(pb, x01, f.acc[g + 1][0]);
+                    f.acc[g + 1][1] = __ffma2_rn(pb, x23, f.acc[g + 1][1]);
+                }
             }
         }
     }
 }
 
-template <typename E, int G>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(DecArgs a) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int unit = blockIdx.x % a.units;
-    const long bh = blockIdx.x / a.units;
-    const int es = (int)sizeof(E);
-
-    Smem<E, G> sm;
-    sm.T = a.T;
-    sm.tabq = reinterpret_cast<float *>(smem_raw);
-    sm.tabc = sm.tabq + kD * G;
-    sm.qc = sm.tabc + kD;
-    sm.pbuf = sm.qc + 16;
-    sm.wmax = sm.pbuf + kNT * G;
-    {
-        uintptr_t p = reinterpret_cast<uintptr_t>(sm.wmax + 4 * G);
-        p = (p + 7) & ~uintptr_t(7);
-        sm.bars = reinterpret_cast<uint64_t *>(p);
-        p = reinterpret_cast<uintptr_t>(sm.bars + kMaxStages);
-        p = (p + 127) & ~uintptr_t(127);
-        sm.stages = reinterpret_cast<unsigned char *>(p);
-    }
-    sm.stage_bytes = dec_stage_bytes(a.T, es);
-
-    const bool tail_unit = (unit == a.n_pre);
-
-    // ---- tables: q' (scaled query), c_j = mu / qn_j, Qc = sum_j q'_j c_j
-    {
-        const int j = tid;
-        const E *q = static_cast<const E *>(a.q) + (size_t)bh * G * kD;
-        const double mu = a.stats[bh * 4 + 3];
-        const float qnj = a.qn[bh * kD + j];
-        const float c = (!tail_unit && qnj > 0.f) ? (float)(mu / (double)qnj) : 0.f;
-        sm.tabc[j] = c;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float qq = Elem<E>::to_f(q[(size_t)g * kD + j]) * kQScale;
-            sm.tabq[j * G + g] = qq;
-            float prod = qq * c;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) prod += __shfl_xor_sync(0xffffffffu, prod, o);
-            if (lane == 0) sm.wmax[(tid >> 5) * G + g] = prod;
-        }
-        if (tid == 0) {
-            for (int st = 0; st < a.nstage; ++st) mbar_init(smem_u32(sm.bars + st), 1);
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        }
-        __syncthreads();
-        if (tid < G) {
-            float s = 0.f;
-            for (int w = 0; w < kDecThreads / 32; ++w) s += sm.wmax[w * G + tid];
-            sm.qc[tid] = s;
-        }
-        __syncthreads();
-    }
-
-    float m_run[G], lsum[G], acc[G][8];
+// Write one item's partial state (acc[G][D], m, l) to the workspace.
+template <int G>
+__device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, Flash<G> &f) {
+    const int lane = threadIdx.x & 31;
+    const size_t row = (size_t)bh * a.units + u;
+    float *acc = a.acc + row * G * kD;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        m_run[g] = -INFINITY;
-        lsum[g] = 0.f;
+        *reinterpret_cast<float4 *>(acc + g * kD + 4 * lane) =
+            make_float4(f.acc[g][0].x, f.acc[g][0].y, f.acc[g][1].x, f.acc[g][1].y);
+        float l = f.l[g];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[g][c] = 0.f;
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) {
+            a.ml[(row * G + g) * 2 + 0] = f.m[g];
+            a.ml[(row * G + g) * 2 + 1] = l;
+        }
     }
+}
+
+// warps per CTA the kernel is compiled for: 16 (128 registers) up to G = 4,
+// 12 (168 registers) for G = 8
+__host__ __device__ constexpr int dec_max_warps(int G) { return G > 4 ? 12 : kMaxWarps; }
+
+template <typename E, int G>
+__global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= a.nwarp) return;
+    const int es = (int)sizeof(E);
+    constexpr int kVB = VRegs<E>::kTok;
+
+    WarpSmem<E, G> ws;
+    {
+        unsigned char *base = smem_raw + (size_t)warp * a.warp_bytes;
+        ws.tabq = reinterpret_cast<float *>(base);
+        ws.tabc = ws.tabq + kD * G;
+        ws.pdup = ws.tabc + kD;
+        ws.qc = ws.pdup + kWT * G * 2;
+        ws.bars = reinterpret_cast<uint64_t *>(ws.qc + 16);
+        ws.stages = base + dec_table_bytes(G);
+        ws.stage_bytes = (uint32_t)dec_stage_bytes(a.T, es);
+    }
+    if (lane == 0) {
+        for (int st = 0; st < a.nstage; ++st) mbar_init(smem_u32(ws.bars + st), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+
+    // Items 0 .. BH*n_pre-1 are prompt chunks (row-major over (head, chunk)),
+    // then one dense-tail item per head, so the small tail items fill the idle
+    // warps of the last round.  Warps are numbered CTA-fastest so that
+    // consecutive items land on different SMs.  Item indices fit in 32 bits
+    // (BH * units < 2^31 is checked on the host).
+    const int nwt = gridDim.x * a.nwarp;
+    const int gw = warp * gridDim.x + blockIdx.x;
+    const int n_items = (int)(a.BH * a.units);
+    const int n_prompt = (int)(a.BH * a.n_pre);
+    auto item_head = [&](int item) -> int { return item < n_prompt ? item / a.n_pre : item - n_prompt; };
+    auto item_unit = [&](int item) -> int { return item < n_prompt ? item % a.n_pre : a.n_pre; };
+
+    // ---- tile stream of this warp: prompt tiles of its items, in order
+    struct Cursor {
+        int item;
+        int tile;
+    };
+    auto item_tiles = [&](int item) -> int {
+        const int u = item_unit(item);
+        if (u >= a.n_pre) return 0;  // dense-tail items are not streamed
+        const long t0 = (long)u * a.chunk;
+        const long t1 = min((long)a.S, t0 + a.chunk);
+        return t1 > t0 ? (int)((t1 - t0 + kWT - 1) / kWT) : 0;
+    };
+    auto settle = [&](Cursor &c) {  // move to the next tile that exists
+        while (c.item < n_items && c.tile >= item_tiles(c.item)) {
+            c.item += nwt;
+            c.tile = 0;
+        }
+    };
+    const E *gvals = static_cast<const E *>(a.vals);
+    const E *gv = static_cast<const E *>(a.v);
+    auto issue = [&](int st, const Cursor &c) {
+        const long bh = item_head(c.item);
+        const int u = item_unit(c.item);
+        const long t0 = (long)u * a.chunk + (long)c.tile * kWT;
+        const long t1 = min((long)a.S, (long)u * a.chunk + a.chunk);
+        const int n = (int)min((long)kWT, t1 - t0);
+        const uint32_t mb = (uint32_t)n * 16u;
+        const uint32_t vb = (uint32_t)kWT * (uint32_t)a.T * (uint32_t)es;  // one whole 32-token group
+        const uint32_t bar = smem_u32(ws.bars + st);
+        unsigned char *dst = ws.stages + (size_t)st * ws.stage_bytes;
+        mbar_expect_tx(bar, mb + vb);
+        bulk_g2s(smem_u32(dst), a.mask + ((size_t)bh * a.S + t0) * kMaskWords, mb, bar);
+        if (vb) bulk_g2s(smem_u32(dst + kWT * 16), gvals + (size_t)bh * a.S32 * a.T + (size_t)t0 * a.T, vb, bar);
+    };
+
+    Cursor ic{gw, 0};
+    settle(ic);
+    int issued = 0, consumed = 0;
+    if (lane == 0) {
+        Cursor c = ic;
+        for (int st = 0; st < a.nstage && c.item < n_items; ++st) {
+            issue(st, c);
+            ++c.tile;
+            settle(c);
+        }
+    }
+    for (int st = 0; st < a.nstage && ic.item < n_items; ++st) {  // all lanes track the cursor
+        ++issued;
+        ++ic.tile;
+        settle(ic);
+    }
+
+    Flash<G> f;
+    VRegs<E> vr;
+    int tab_bh = -1;
     bool failed = false;
-    const int tt = tid >> 1, h = tid & 1;
 
-    if (!tail_unit) {
-        const long t_begin = (long)unit * a.chunk;
-        const long t_end = min((long)a.S, t_begin + a.chunk);
-        const int ntiles = t_end > t_begin ? (int)((t_end - t_begin + kNT - 1) / kNT) : 0;
-        const uint32_t *gmask = a.mask + (size_t)bh * a.S * kMaskWords;
-        const E *gvals = static_cast<const E *>(a.vals) + (size_t)bh * a.S32 * a.T;
-        const E *gv = static_cast<const E *>(a.v) + (size_t)bh * a.S * kD;
+    for (int item = gw; item < n_items && !failed; item += nwt) {
+        const int bh = item_head(item);
+        const int u = item_unit(item);
+        const bool tail = (u == a.n_pre);
+        if (tail && a.n_tail == 0) {
+            f.reset();
+            write_partial<G>(a, bh, u, f);
+            continue;
+        }
+        // ---- tables of this head: q' (scaled query), c_j = mu / qn_j, Qc
+        if (bh != tab_bh) {
+            const E *q = static_cast<const E *>(a.q) + (size_t)bh * G * kD;
+            const double mu = a.stats[bh * 4 + 3];
+            float part[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) part[g] = 0.f;
+#pragma unroll
+            for (int i = 0; i < kD / 32; ++i) {
+                const int j = lane + 32 * i;
+                const float qnj = a.qn[bh * kD + j];
+                const float c = qnj > 0.f ? (float)(mu / (double)qnj) : 0.f;
+                ws.tabc[j] = c;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float qq = Elem<E>::to_f(q[(size_t)g * kD + j]) * kQScale;
+                    ws.tabq[j * G + g] = qq;
+                    part[g] = fmaf(qq, c, part[g]);
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) part[g] += __shfl_xor_sync(0xffffffffu, part[g], o);
+                if (lane == 0) ws.qc[g] = part[g];
+            }
+            tab_bh = bh;
+            __syncwarp();
+        }
+        f.reset();
 
-        auto issue = [&](int i) {
-            const int st = i % a.nstage;
-            const long t0 = t_begin + (long)i * kNT;
-            const int n = (int)min((long)kNT, t_end - t0);
-            const uint32_t mb = (uint32_t)n * 16u;
-            const uint32_t vb = (uint32_t)((n + 31) / 32) * 32u * (uint32_t)a.T * (uint32_t)es;
-            const uint32_t Vb = (uint32_t)n * kD * (uint32_t)es;
-            const uint32_t bar = smem_u32(sm.bars + st);
-            mbar_expect_tx(bar, mb + vb + Vb);
-            bulk_g2s(smem_u32(sm.smask(st)), gmask + t0 * kMaskWords, mb, bar);
-            if (vb) bulk_g2s(smem_u32(sm.svals(st)), gvals + t0 * a.T, vb, bar);
-            bulk_g2s(smem_u32(sm.sV(st)), gv + t0 * kD, Vb, bar);
-        };
-        if (tid == 0)
-            for (int i = 0; i < min(a.nstage, ntiles); ++i) issue(i);
+        if (tail) {
+            // ---- dense tail: keys and values read from global memory
+            const E *kt = static_cast<const E *>(a.k_tail) + (size_t)bh * a.tail_cap * kD;
+            const E *vt = static_cast<const E *>(a.v_tail) + (size_t)bh * a.tail_cap * kD;
+            for (int t0 = 0; t0 < a.n_tail; t0 += kWT) {
+                const int n = min(kWT, a.n_tail - t0);
+                vr.load(vt + (size_t)t0 * kD + 4 * lane, n);
+                float s[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) s[g] = 0.f;
+                if (lane < n) {
+                    const E *krow = kt + (size_t)(t0 + lane) * kD;
+#pragma unroll 4
+                    for (int j4 = 0; j4 < kD; j4 += 4) {
+                        float x[4];
+                        Row4<E>::load(krow + j4, x);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            QVec<G> qv;
+                            qv.load(ws.tabq + (j4 + c) * G);
+#pragma unroll
+                            for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x[c], s[g]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) s[g] = (lane < n) ? s[g] : -INFINITY;
+                tile_softmax<E, G>(ws, f, s);
+                for (int tb = 0; tb < n; tb += kVB) {
+                    if (tb > 0) vr.load(vt + (size_t)(t0 + tb) * kD + 4 * lane, n - tb);
+                    tile_pv<E, G>(ws, f, vr, tb, n);
+                }
+                __syncwarp();
+            }
+            write_partial<G>(a, bh, u, f);
+            continue;
+        }
 
-        int consumed = 0;
-        for (int i = 0; i < ntiles; ++i) {
-            const int st = i % a.nstage;
-            const long t0 = t_begin + (long)i * kNT;
-            const int n = (int)min((long)kNT, t_end - t0);
-            bool ok = mbar_wait_bounded(smem_u32(sm.bars + st), (uint32_t)((i / a.nstage) & 1));
-            if (!__syncthreads_and(ok)) {
+        // ---- prompt tokens of this item, one 32-token tile at a time
+        const int ntiles = item_tiles(item);
+        const long t_item = (long)u * a.chunk;
+        const long t_end = min((long)a.S, t_item + a.chunk);
+        const E *vbase = gv + (size_t)bh * a.S * kD + 4 * lane;
+        for (int tile = 0; tile < ntiles; ++tile) {
+            const long t0 = t_item + (long)tile * kWT;
+            const int n = (int)min((long)kWT, t_end - t0);
+            // this tile's first V rows go to registers under the q.k~ below
+            vr.load(vbase + (size_t)t0 * kD, n);
+
+            const int st = (int)(consumed % a.nstage);
+            const uint32_t par = (uint32_t)((consumed / a.nstage) & 1);
+            // every lane waits; the warp agrees on the outcome so that no lane
+            // leaves the shuffles and REDUX below on its own
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(ws.bars + st), par))) {
                 failed = true;
                 break;
             }
-            consumed = i + 1;
+            const bool valid = lane < n;
 
-            // ---- scores: two threads per token, 64 channels each
+            // q . k~ over the T kept channels of this lane's token
             float s[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) s[g] = 0.f;
-            const bool valid = tt < n;
-            if (valid && a.T > 0) {
-                const uint4 mw = *reinterpret_cast<const uint4 *>(sm.smask(st) + tt * kMaskWords);
-                uint32_t wa = h ? mw.z : mw.x;
-                uint32_t wb = h ? mw.w : mw.y;
-                int pos = h ? (__popc(mw.x) + __popc(mw.y)) : 0;
-                const E *vcol = sm.svals(st) + (tt >> 5) * 32 * a.T + (tt & 31);
-                const int jb = 64 * h;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t cur = half ? wb : wa;
-                    const int jbase = jb + 32 * half;
-                    while (cur) {
-                        const int b = __ffs(cur) - 1;
-                        cur &= cur - 1u;
-                        const int j = jbase + b;
-                        // a mask with more than T bits (a cache never written by
-                        // spark_prune) must not index past this stage
-                        const float kv = Elem<E>::to_f(vcol[min(pos, a.T - 1) * 32]);
-                        ++pos;
-                        const float x = kv - sm.tabc[j];
-                        QVec<G> qv;
-                        qv.load(sm.tabq + j * G);
-#pragma unroll
-                        for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                s[g] += __shfl_xor_sync(0xffffffffu, s[g], 1);
-                s[g] = valid ? s[g] + sm.qc[g] : -INFINITY;
-            }
-            const E *sV = sm.sV(st);
-            softmax_pv<E, G>(sm, s, n, m_run, acc, lsum, [&](int t2) { return sV + (size_t)t2 * kD; });
-            __syncthreads();  // stage and p buffer free
-            if (tid == 0 && i + a.nstage < ntiles) {
-                fence_proxy_async_smem();
-                issue(i + a.nstage);
-            }
-        }
-        if (failed) {
-            if (tid == 0) {
-                atomicOr(a.status, kDevTimeout);
-                // let copies already in flight land before the CTA exits
-                const int issued = min(ntiles, consumed + a.nstage);
-                for (int i = consumed; i < issued; ++i)
-                    (void)mbar_wait_bounded(smem_u32(sm.bars + (i % a.nstage)),
-                                            (uint32_t)((i / a.nstage) & 1));
-            }
-            return;
-        }
-    } else {
-        // ---- dense tail: keys and values read straight from global memory
-        const E *kt = static_cast<const E *>(a.k_tail) + (size_t)bh * a.tail_cap * kD;
-        const E *vt = static_cast<const E *>(a.v_tail) + (size_t)bh * a.tail_cap * kD;
-        for (int t0 = 0; t0 < a.n_tail; t0 += kNT) {
-            const int n = min(kNT, a.n_tail - t0);
-            float s[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g) s[g] = 0.f;
-            const bool valid = tt < n;
-            if (valid) {
-                const E *krow = kt + (size_t)(t0 + tt) * kD + 64 * h;
+            if (a.T > 0) {
+                const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
+                uint32_t w1 = mw.y, w2 = mw.z, w3 = mw.w;
+                uint32_t cur = mw.x;
+                int wi = 0;
+                const E *vp = ws.svals(st) + lane;
 #pragma unroll 2
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    float x[8];
-                    Row8<E>::load(krow + 8 * c8, x);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        QVec<G> qv;
-                        qv.load(sm.tabq + (64 * h + 8 * c8 + c) * G);
-#pragma unroll
-                        for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x[c], s[g]);
+                for (int i = 0; i < a.T; ++i) {
+                    while (cur == 0u && wi < 3) {
+                        ++wi;
+                        cur = (wi == 1) ? w1 : ((wi == 2) ? w2 : w3);
                     }
+                    // a mask with fewer than T bits (a cache never written by
+                    // spark_prune, or a lane past n) still indexes in bounds
+                    const int j = (32 * wi + __ffs(cur) - 1) & (kD - 1);
+                    cur &= cur - 1u;
+                    const float x = Elem<E>::to_f(vp[i * kWT]) - ws.tabc[j];
+                    QVec<G> qv;
+                    qv.load(ws.tabq + j * G);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }
             }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                s[g] += __shfl_xor_sync(0xffffffffu, s[g], 1);
-                s[g] = valid ? s[g] : -INFINITY;
+            // the stage is read: hand it to the tile nstage ahead
+            __syncwarp();
+            ++consumed;
+            if (ic.item < n_items) {
+                if (lane == 0) {
+                    fence_proxy_async_smem();
+                    issue(st, ic);
+                }
+                ++issued;
+                ++ic.tile;
+                settle(ic);
             }
-            const E *vbase = vt + (size_t)t0 * kD;
-            softmax_pv<E, G>(sm, s, n, m_run, acc, lsum, [&](int t2) { return vbase + (size_t)t2 * kD; });
-            __syncthreads();
+#pragma unroll
+            for (int g = 0; g < G; ++g) s[g] = valid ? s[g] + ws.qc[g] : -INFINITY;
+            tile_softmax<E, G>(ws, f, s);
+            for (int tb = 0; tb < n; tb += kVB) {
+                if (tb > 0) vr.load(vbase + (size_t)(t0 + tb) * kD, n - tb);
+                tile_pv<E, G>(ws, f, vr, tb, n);
+            }
+            __syncwarp();  // p buffer free
         }
+        if (!failed) write_partial<G>(a, bh, u, f);
     }
 
-    // ---- epilogue: reduce the 8 token subsets in a fixed order
-    float *red = reinterpret_cast<float *>(sm.stages);  // [8][G][kD] then [8][G]
-    float *lred = red + 8 * G * kD;
-    const int cg = tid & 15, ts = tid >> 4;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) red[(ts * G + g) * kD + 8 * cg + c] = acc[g][c];
-        if (cg == 0) lred[ts * G + g] = lsum[g];
-    }
-    __syncthreads();
-    float *out = a.part + ((size_t)bh * a.units + unit) * G * (kD + 2);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float o = 0.f;
-#pragma unroll
-        for (int k2 = 0; k2 < 8; ++k2) o += red[(k2 * G + g) * kD + tid];
-        out[g * (kD + 2) + tid] = o;
-    }
-    if (tid < G) {
-        float l = 0.f;
-        for (int k2 = 0; k2 < 8; ++k2) l += lred[k2 * G + tid];
-        out[tid * (kD + 2) + kD] = m_run[tid];
-        out[tid * (kD + 2) + kD + 1] = l;
+    if (failed) {
+        if (lane == 0) {
+            atomicOr(a.status, kDevTimeout);
+            // let copies already in flight land before the warp exits
+            for (int i = consumed; i < issued; ++i)
+                (void)mbar_wait_bounded(smem_u32(ws.bars + (int)(i % a.nstage)),
+                                        (uint32_t)((i / a.nstage) & 1));
+        }
+        __syncwarp();
     }
 }
 
 template <int G>
-__global__ void __launch_bounds__(kD) combine_kernel(const float *__restrict__ part, int units,
+__global__ void __launch_bounds__(kD) combine_kernel(const float *__restrict__ acc,
+                                                     const float *__restrict__ ml, int units,
                                                      float *__restrict__ out) {
     const long row = blockIdx.x;  // (bh, g)
     const long bh = row / G;
     const int g = (int)(row % G);
     const int d = threadIdx.x;
-    const size_t ustride = (size_t)G * (kD + 2);
-    const float *base = part + (size_t)bh * units * ustride + (size_t)g * (kD + 2);
     float M = -INFINITY;
-    for (int u = 0; u < units; ++u) M = fmaxf(M, base[u * ustride + kD]);
+    for (int u = 0; u < units; ++u) M = fmaxf(M, ml[(((size_t)bh * units + u) * G + g) * 2]);
     float L = 0.f, o = 0.f;
     if (M != -INFINITY) {
         for (int u = 0; u < units; ++u) {
-            const float mu = base[u * ustride + kD];
-            const float lu = base[u * ustride + kD + 1];
+            const size_t r = ((size_t)bh * units + u) * G + g;
+            const float mu = ml[r * 2], lu = ml[r * 2 + 1];
             if (lu > 0.f) {
                 const float w = exp2f(mu - M);
                 L = fmaf(lu, w, L);
-                o = fmaf(base[u * ustride + d], w, o);
+                o = fmaf(acc[r * kD + d], w, o);
             }
         }
     }
@@ -433,42 +547,42 @@ __global__ void __launch_bounds__(kD) combine_kernel(const float *__restrict__ p
 DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms) {
     DecodeGeom g{};
     const size_t stage = dec_stage_bytes(T, es);
-    const size_t fixed = dec_fixed_bytes(G);
-    const size_t epi = dec_epilogue_bytes(G);
-    const size_t per_sm = 228 * 1024, per_cta_max = 227 * 1024;
-    g.ctas_per_sm = 1;
-    g.nstage = 2;
-    for (int cpsm = 3; cpsm >= 1; --cpsm) {
-        const size_t lim = std::min(per_cta_max, per_sm / cpsm - 1024);
-        if (lim <= fixed) continue;
-        const int ns = (int)std::min<size_t>(kMaxStages, (lim - fixed) / stage);
-        if (ns >= (cpsm > 1 ? 3 : 2)) {
-            g.ctas_per_sm = cpsm;
-            g.nstage = ns;
-            break;
-        }
-    }
-    g.smem = fixed + std::max((size_t)g.nstage * stage, epi);
+    const size_t table = dec_table_bytes(G);
+    const size_t budget = 227 * 1024;
+    const int max_w = dec_max_warps(G);
+    auto warps_for = [&](int ns) {
+        const size_t wb = (table + ns * stage + 127) / 128 * 128;
+        return (int)std::min<size_t>(max_w, budget / wb);
+    };
+    // a 4-deep ring if all warps still fit, else 3 deep with >= 3/4 of them,
+    // else 2 deep with as many warps as fit
+    if (warps_for(4) >= max_w) g.nstage = 4;
+    else if (warps_for(3) >= max_w * 3 / 4) g.nstage = 3;
+    else g.nstage = 2;
+    g.nwarp = std::max(1, warps_for(g.nstage));
+    g.warp_bytes = (table + g.nstage * stage + 127) / 128 * 128;
+    g.smem = g.warp_bytes * g.nwarp;
+    g.ctas = num_sms;
 
+    const long nwt = (long)g.ctas * g.nwarp;
     if (S <= 0 || BH <= 0) {
-        g.chunk = kNT;
+        g.chunk = kWT;
         g.n_pre = 0;
     } else {
-        const long slots = (long)num_sms * g.ctas_per_sm;
-        const long overhead = 512;  // per-unit fixed cost in token equivalents
+        const long overhead = 128;  // per-item cost in token equivalents
         double best = 1e300;
-        for (int w = 1; w <= 256; ++w) {
-            long n_pre = std::max(1L, (w * slots) / BH);
-            long chunk = ((S + n_pre - 1) / n_pre + kNT - 1) / kNT * kNT;
+        for (int w = 1; w <= 512; ++w) {
+            long n_pre = std::max(1L, (w * nwt) / BH);
+            long chunk = ((S + n_pre - 1) / n_pre + kWT - 1) / kWT * kWT;
             n_pre = (S + chunk - 1) / chunk;
-            const long waves = (BH * n_pre + slots - 1) / slots;
+            const long waves = (BH * n_pre + nwt - 1) / nwt;
             const double cost = (double)waves * (double)(chunk + overhead);
             if (cost < best) {
                 best = cost;
                 g.chunk = (int)chunk;
                 g.n_pre = (int)n_pre;
             }
-            if (chunk == kNT) break;
+            if (chunk == kWT) break;
         }
     }
     g.units = g.n_pre + 1;
@@ -476,29 +590,29 @@ DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms) {
 }
 
 template <typename E, int G>
-static cudaError_t launch_decode_t(const DecArgs &a0, long BH, const DecodeGeom &geo, float *out,
-                                   cudaStream_t st) {
+static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, float *out, cudaStream_t st) {
     DecArgs a = a0;
     a.chunk = geo.chunk;
     a.n_pre = geo.n_pre;
     a.units = geo.units;
     a.nstage = geo.nstage;
+    a.nwarp = geo.nwarp;
+    a.warp_bytes = geo.warp_bytes;
     auto kern = decode_kernel<E, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)geo.smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(BH * geo.units), kDecThreads, geo.smem, st>>>(a);
-    combine_kernel<G><<<(unsigned)(BH * G), kD, 0, st>>>(a.part, geo.units, out);
+    kern<<<geo.ctas, geo.nwarp * 32, geo.smem, st>>>(a);
+    combine_kernel<G><<<(unsigned)(a.BH * G), kD, 0, st>>>(a.acc, a.ml, geo.units, out);
     return cudaGetLastError();
 }
 
 template <typename E>
-static cudaError_t dispatch_g(const DecArgs &a, long BH, const DecodeGeom &geo, int G, float *out,
-                              cudaStream_t st) {
+static cudaError_t dispatch_g(const DecArgs &a, const DecodeGeom &geo, int G, float *out, cudaStream_t st) {
     switch (G) {
-    case 1: return launch_decode_t<E, 1>(a, BH, geo, out, st);
-    case 2: return launch_decode_t<E, 2>(a, BH, geo, out, st);
-    case 4: return launch_decode_t<E, 4>(a, BH, geo, out, st);
-    case 8: return launch_decode_t<E, 8>(a, BH, geo, out, st);
+    case 1: return launch_decode_t<E, 1>(a, geo, out, st);
+    case 2: return launch_decode_t<E, 2>(a, geo, out, st);
+    case 4: return launch_decode_t<E, 4>(a, geo, out, st);
+    case 8: return launch_decode_t<E, 8>(a, geo, out, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -518,14 +632,16 @@ cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, 
     a.k_tail = k_tail;
     a.v_tail = v_tail;
     a.status = static_cast<uint32_t *>(ws);
-    a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
+    a.acc = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
+    a.ml = a.acc + (size_t)BH * geo.units * G * kD;
+    a.BH = BH;
     a.S = kc.S;
     a.S32 = ((long)kc.S + 31) / 32 * 32;
     a.T = kc.T;
     a.tail_cap = tail_cap;
     a.n_tail = n_tail;
-    if (kc.dtype == SPARK_BF16) return dispatch_g<__nv_bfloat16>(a, BH, geo, G, out, st);
-    return dispatch_g<float>(a, BH, geo, G, out, st);
+    if (kc.dtype == SPARK_BF16) return dispatch_g<__nv_bfloat16>(a, geo, G, out, st);
+    return dispatch_g<float>(a, geo, G, out, st);
 }
 
 }  // namespace spark

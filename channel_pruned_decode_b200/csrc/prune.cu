@@ -109,33 +109,63 @@ __device__ __forceinline__ int quad_sum(int v) {
     return v;
 }
 
+// Count of the quad's keys >= mid, from the packed bf16-truncated keys
+// (the upper 16 bits of the fp32 saliency, two per register).  Truncation is
+// monotone, so this is the integer count over the 16-bit keys.  `mid` is 0 or
+// a normal bf16 pattern (>= 0x80), so no subnormal is ever compared; keys
+// below 0x80 (zero or subnormal saliency) are below every probe.  One packed
+// compare and one packed add per two channels; counts <= 32 per lane are
+// exact in bf16.
+__device__ __forceinline__ int quad_count16(const uint32_t (&kp)[16], uint32_t mid) {
+    const uint32_t mm = mid * 0x10001u;
+    const __nv_bfloat162 m2 = *reinterpret_cast<const __nv_bfloat162 *>(&mm);
+    const __nv_bfloat162 z = __float2bfloat162_rn(0.f);
+    __nv_bfloat162 a0 = z, a1 = z, a2 = z, a3 = z;
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+        a0 = __hadd2(a0, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 0]), m2));
+        a1 = __hadd2(a1, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 1]), m2));
+        a2 = __hadd2(a2, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 2]), m2));
+        a3 = __hadd2(a3, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 3]), m2));
+    }
+    a0 = __hadd2(__hadd2(a0, a1), __hadd2(a2, a3));
+    const int c = (int)(__low2float(a0) + __high2float(a0));
+    return quad_sum(c);
+}
+
+__device__ __forceinline__ int quad_count32(const uint32_t (&key)[32], uint32_t mid) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) c += (key[i] >= mid) ? 1 : 0;
+    return quad_sum(c);
+}
+
 // Mask word (32 channels) of this lane's quarter of the token: the T largest
-// keys over the quad, ties to the lower channel index.
-__device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], int T, int s) {
+// exact fp32 keys over the quad, ties to the lower channel index.
+//
+// Phase 1 searches the T-th largest 16-bit key with packed counts, starting
+// at the previous token's threshold `tau16` and galloping outward until the
+// bracket closes, then bisecting; it ends either with a probe that leaves
+// exactly T keys above it (the usual case) or with the 16-bit tie band
+// [tau16, tau16+1) holding the boundary.  Phase 2 bisects the exact 32-bit
+// keys inside that band.  Both loops have warp-uniform trip counts (quads
+// that are done idle), so the quad shuffles always see the full warp.
+__device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
+                                                 int s, uint32_t &tau16) {
     if (T <= 0) return 0u;
     if (T >= kD) return 0xffffffffu;
-    uint32_t kmax = 0u, kmin = 0xffffffffu;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        kmax = max(kmax, key[i]);
-        kmin = min(kmin, key[i]);
-    }
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 1));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, 2));
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, 1));
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, 2));
 
-    // invariant: count(key >= lo) >= T > count(key >= hi); keys are < 2^31
-    uint32_t lo = kmin, hi = kmax + 1u;
+    // ---- phase 1: 16-bit keys.  count(>= lo) >= T > count(>= hi)
+    constexpr uint32_t kTop = 0x7f81u;  // above +inf: nothing reaches it
+    uint32_t lo = 0u, hi = kTop;
     int c_hi = 0;
     bool exact = false;
-    bool done = (hi - lo <= 1u);
-    while (__any_sync(0xffffffffu, !done)) {  // warp-uniform trip count
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        int c = 0;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) c += (key[i] >= mid) ? 1 : 0;
-        c = quad_sum(c);
+    bool done = false;
+    uint32_t step = 64u;
+    uint32_t mid = min(max(tau16, 1u), kTop - 1u);
+    while (__any_sync(0xffffffffu, !done)) {
+        const uint32_t probe = (mid > 0u && mid < 0x80u) ? 0x80u : mid;
+        const int c = quad_count16(kp, probe);
         if (!done) {
             if (c >= T) {
                 lo = mid;
@@ -145,25 +175,60 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], int 
                 c_hi = c;
             }
             if (hi - lo <= 1u) done = true;
+            // next probe: gallop away from an unknown side, else bisect
+            if (hi == kTop) {
+                mid = min(lo + step, kTop - 1u);
+                step <<= 1;
+            } else if (lo == 0u) {
+                mid = hi > step ? hi - step : hi >> 1;
+                mid = max(mid, 1u);
+                step <<= 1;
+            } else {
+                mid = lo + ((hi - lo) >> 1);
+            }
         }
     }
-    // exact: exactly T keys are >= lo.  Otherwise lo is the T-th largest key,
-    // c_hi keys are above it, and T - c_hi of the keys equal to lo are kept in
-    // channel order.
-    const uint32_t thr = exact ? lo : lo + 1u;
+    tau16 = lo;
+
+    // ---- phase 2: exact keys inside the band of 16-bit key == lo.  Quads
+    // whose phase 1 was exact skip it (done2) but stay in the uniform loop.
+    // When exact, exactly T keys have a 16-bit key >= lo (lo >= 1; no 16-bit
+    // key lies in [1, 0x80)), i.e. an fp32 key >= max(lo, 0x80) << 16.
+    uint32_t lo32 = exact ? (max(lo, 0x80u) << 16) : ((lo == 0u) ? 0u : (lo << 16));
+    uint32_t hi32 = (lo == 0u) ? 0x00800000u : ((lo + 1u) << 16);
+    bool exact32 = exact;
+    bool done2 = exact || (hi32 - lo32 <= 1u);
+    while (__any_sync(0xffffffffu, !done2)) {
+        const uint32_t mid32 = lo32 + ((hi32 - lo32) >> 1);
+        const int c = quad_count32(key, mid32);
+        if (!done2) {
+            if (c >= T) {
+                lo32 = mid32;
+                if (c == T) { exact32 = true; done2 = true; }
+            } else {
+                hi32 = mid32;
+                c_hi = c;
+            }
+            if (hi32 - lo32 <= 1u) done2 = true;
+        }
+    }
+    // exact32: exactly T keys are >= lo32.  Otherwise lo32 is the T-th largest
+    // key, c_hi keys are above it, and the first T - c_hi keys equal to it (in
+    // channel order over the quad) are kept.
+    const uint32_t thr = exact32 ? lo32 : lo32 + 1u;
     uint32_t m = 0u;
     int e = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         m |= (key[i] >= thr ? 1u : 0u) << i;
-        e += (key[i] == lo) ? 1 : 0;
+        e += (key[i] == lo32) ? 1 : 0;
     }
     int r = quad_excl_scan(e, s);
-    if (!exact) {
+    if (!exact32) {
         const int need = T - c_hi;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            if (key[i] == lo) {
+            if (key[i] == lo32) {
                 if (r < need) m |= 1u << i;
                 ++r;
             }
@@ -171,14 +236,16 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], int 
     }
     return m;
 }
-
 template <typename E>
 __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
                  E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks) {
     using Raw = typename RawT<E>::type;
     __shared__ __align__(16) Raw vtile[2][kD * 32];  // [kept index][token in group]
-    __shared__ double red[2][kPruneThreads];
+    __shared__ double red[2][kPruneThreads / 32];
+    // window-query norms of this head, one padded row per quarter (stride 36
+    // floats): the 4 quarters' 16-byte reads fall in distinct banks
+    __shared__ __align__(16) float qs[4 * 36];
 
     const long bh = blockIdx.x / n_chunks;
     const int chunk = blockIdx.x % n_chunks;
@@ -187,55 +254,69 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     const int tl = warp * 8 + (lane >> 2);  // token within the 32-token group
     const long S32 = ((long)S + 31) / 32 * 32;
 
-    float qv[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) qv[i] = __ldg(qn + bh * kD + 32 * s + i);
+    if (tid < kD) qs[(tid >> 5) * 36 + (tid & 31)] = __ldg(qn + bh * kD + tid);
+    __syncthreads();
 
+    // the first token of each quad starts its threshold search at 1.0
+    uint32_t tau16 = 0x3f80u;
     double acc_w = 0.0, acc_w2 = 0.0;
+    const long g_first = (long)chunk * kPruneGroups;
+    KSlice<E> ks, ks_next;
+    {
+        const long t = g_first * 32 + tl;
+        if (t < S) ks.load(k + ((size_t)bh * S + t) * kD + 32 * s);
+        else ks.zero();
+    }
     for (int gi = 0; gi < kPruneGroups; ++gi) {
-        const long grp = (long)chunk * kPruneGroups + gi;
+        const long grp = g_first + gi;
         const long t0 = grp * 32;
         if (t0 >= S) break;  // uniform across the CTA
         const long t = t0 + tl;
         const bool valid = t < S;
+        // prefetch the next group's slice while this one is selected
+        {
+            const long tn = t + 32;
+            if (gi + 1 < kPruneGroups && tn < S) ks_next.load(k + ((size_t)bh * S + tn) * kD + 32 * s);
+            else ks_next.zero();
+        }
 
-        KSlice<E> ks;
-        if (valid)
-            ks.load(k + ((size_t)bh * S + t) * kD + 32 * s);
-        else
-            ks.zero();
-
+        // exact fp32 saliency keys and their packed 16-bit truncations
         uint32_t key[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            key[i] = __float_as_uint(__fmul_rn(qv[i], __uint_as_float(ks.abs_bits(i))));
+        for (int c = 0; c < 8; ++c) {
+            const float4 q4 = *reinterpret_cast<const float4 *>(qs + s * 36 + 4 * c);
+            const float qq[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                key[4 * c + e] = __float_as_uint(__fmul_rn(qq[e], __uint_as_float(ks.abs_bits(4 * c + e))));
+        }
+        uint32_t kp[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) kp[i] = __byte_perm(key[2 * i], key[2 * i + 1], 0x7632);
 
-        const uint32_t m = select_top_t(key, T, s);
+        const uint32_t m = select_top_t(key, kp, T, s, tau16);
         if (valid) mask[((size_t)bh * S + t) * kMaskWords + s] = m;
 
-        // pruned-saliency sums (fp32 over this lane's 32 channels, fp64 across tokens)
-        float sw = 0.f, sw2 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float w = __uint_as_float(key[i]);
-            const bool pr = !((m >> i) & 1u);
-            sw = __fadd_rn(sw, pr ? w : 0.f);
-            sw2 = __fmaf_rn(pr ? w : 0.f, w, sw2);
-        }
-        if (valid) {
-            acc_w = __dadd_rn(acc_w, (double)sw);
-            acc_w2 = __dadd_rn(acc_w2, (double)sw2);
-        }
-
-        // pack kept values in ascending channel order into the staging tile
+        // pruned-saliency sums (fp32 over this lane's 32 channels, fp64 across
+        // tokens) and the kept values, in ascending channel order, into the
+        // staging tile
         Raw *vt = vtile[gi & 1];
         int pos = quad_excl_scan(__popc(m), s);
+        float sw = 0.f, sw2 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             if ((m >> i) & 1u) {
                 vt[pos * 32 + tl] = (Raw)ks.raw(i);
                 ++pos;
+            } else {
+                const float w = __uint_as_float(key[i]);
+                sw = __fadd_rn(sw, w);
+                sw2 = __fmaf_rn(w, w, sw2);
             }
+        }
+        if (valid) {
+            acc_w = __dadd_rn(acc_w, (double)sw);
+            acc_w2 = __dadd_rn(acc_w2, (double)sw2);
         }
         __syncthreads();
         // 32 tokens x T values, contiguous in the interleaved layout
@@ -243,14 +324,23 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
         uint4 *dst = reinterpret_cast<uint4 *>(vals + (size_t)bh * S32 * T + (size_t)t0 * T);
         const uint4 *src = reinterpret_cast<const uint4 *>(vt);
         for (int vi = tid; vi < nvec; vi += kPruneThreads) __stcs(dst + vi, src[vi]);
+        ks = ks_next;
     }
 
-    red[0][tid] = acc_w;
-    red[1][tid] = acc_w2;
+    // fixed-order reduction: xor tree inside each warp, then warps in order
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        acc_w = __dadd_rn(acc_w, __shfl_xor_sync(0xffffffffu, acc_w, o));
+        acc_w2 = __dadd_rn(acc_w2, __shfl_xor_sync(0xffffffffu, acc_w2, o));
+    }
+    if (lane == 0) {
+        red[0][warp] = acc_w;
+        red[1][warp] = acc_w2;
+    }
     __syncthreads();
     if (tid == 0) {
         double a = 0.0, b = 0.0;
-        for (int i = 0; i < kPruneThreads; ++i) {
+        for (int i = 0; i < kPruneThreads / 32; ++i) {
             a = __dadd_rn(a, red[0][i]);
             b = __dadd_rn(b, red[1][i]);
         }
@@ -259,20 +349,30 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     }
 }
 
+// One warp per (row, kv head): lanes sum the chunk partials in a fixed order,
+// then a fixed xor tree.
 __global__ void stats_kernel(const double *__restrict__ partial, int n_chunks, long BH, int S, int T,
                              double *__restrict__ stats) {
-    const long bh = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long bh = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
     if (bh >= BH) return;
     double a = 0.0, b = 0.0;
-    for (int c = 0; c < n_chunks; ++c) {
+    for (int c = lane; c < n_chunks; c += 32) {
         a = __dadd_rn(a, partial[((size_t)bh * n_chunks + c) * 2 + 0]);
         b = __dadd_rn(b, partial[((size_t)bh * n_chunks + c) * 2 + 1]);
     }
-    const double n = (double)S * (double)(kD - T);
-    stats[bh * 4 + 0] = n;
-    stats[bh * 4 + 1] = a;
-    stats[bh * 4 + 2] = b;
-    stats[bh * 4 + 3] = n > 0.0 ? a / n : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a = __dadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+        b = __dadd_rn(b, __shfl_xor_sync(0xffffffffu, b, o));
+    }
+    if (lane == 0) {
+        const double n = (double)S * (double)(kD - T);
+        stats[bh * 4 + 0] = n;
+        stats[bh * 4 + 1] = a;
+        stats[bh * 4 + 2] = b;
+        stats[bh * 4 + 3] = n > 0.0 ? a / n : 0.0;
+    }
 }
 
 template <typename E>
@@ -288,7 +388,7 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
             static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
             nch);
     }
-    stats_kernel<<<(unsigned)((BH + 127) / 128), 128, 0, st>>>(partial, nch, BH, kc.S, kc.T, kc.stats);
+    stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.S, kc.T, kc.stats);
     return cudaGetLastError();
 }
 

@@ -30,36 +30,39 @@ inline size_t prune_workspace(long BH, int S) {
 }
 
 // ---------------------------------------------------------------- decode
-constexpr int kDecThreads = 128;
-constexpr int kNT = 64;               // tokens per pipeline tile
-constexpr int kMaxStages = 6;
+// Each warp of a persistent CTA is an independent flash-decoding worker.  Its
+// ring of shared-memory stages holds the mask and kept values of one 32-token
+// tile each; the tile's dense V rows go straight to registers.
+constexpr int kWT = 32;               // tokens per warp tile
+constexpr int kMaxWarps = 16;         // warps per CTA
+constexpr int kMaxStagesW = 4;        // ring depth per warp
 
 struct DecodeGeom {
-    int chunk;        // prefix tokens per unit (multiple of kNT)
-    int n_pre;        // prefix units per (row, kv head)
-    int units;        // n_pre + 1 (last unit = dense tail)
-    int nstage;       // pipeline depth
-    int ctas_per_sm;  // occupancy the smem budget was sized for
-    size_t smem;      // dynamic shared memory per CTA
+    int chunk;        // prefix tokens per work item (multiple of kWT)
+    int n_pre;        // prefix items per (row, kv head)
+    int units;        // n_pre + 1 (the last item of a head is its dense tail)
+    int nstage;       // stages per warp
+    int nwarp;        // warps per CTA
+    int ctas;         // persistent grid size
+    size_t warp_bytes;  // shared memory of one warp (tables + ring)
+    size_t smem;        // dynamic shared memory per CTA
 };
 
+// mask (16 B/token) + one 32-token group of kept values
 __host__ __device__ inline size_t dec_stage_bytes(int T, int es) {
-    return (size_t)kNT * 16 + (size_t)kNT * T * es + (size_t)kNT * kD * es;
+    return (size_t)kWT * 16 + (size_t)kWT * T * es;
 }
 
-inline size_t dec_fixed_bytes(int G) {
-    // q' table, c table, Qc, p buffer, per-warp maxima, mbarriers, padding
-    return (size_t)kD * G * 4 + kD * 4 + 64 + (size_t)kNT * G * 4 +
-           4 * G * 4 + kMaxStages * 8 + 256;
-}
-
-inline size_t dec_epilogue_bytes(int G) {
-    // per token-subset partial accumulators (8 subsets) and l sums
-    return (size_t)8 * G * kD * 4 + (size_t)8 * G * 4;
+// q' table [kD][G], c table [kD], duplicated p buffer [kWT][G][2], Qc [16],
+// mbarriers, rounded to 128 bytes so that the stages start aligned
+__host__ __device__ inline size_t dec_table_bytes(int G) {
+    const size_t b = (size_t)kD * G * 4 + kD * 4 + (size_t)kWT * G * 8 + 64 + kMaxStagesW * 8;
+    return (b + 127) / 128 * 128;
 }
 
 DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms);
 
+// partials: acc [BH][units][G][D] fp32, then (m, l) [BH][units][G][2] fp32
 inline size_t decode_workspace(long BH, const DecodeGeom &g, int G) {
     return kWsHeader + (size_t)BH * g.units * G * (kD + 2) * sizeof(float);
 }
