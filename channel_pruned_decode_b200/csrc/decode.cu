@@ -94,9 +94,14 @@ template <> struct VRegs<__nv_bfloat16> {
     uint2 v[kTok];
     // row0 points at channel 4*lane of the batch's first token
     __device__ __forceinline__ void load(const __nv_bfloat16 *row0, int n) {
+        if (n >= kTok) {
 #pragma unroll
-        for (int t = 0; t < kTok; ++t)
-            v[t] = (t < n) ? __ldcs(reinterpret_cast<const uint2 *>(row0 + (size_t)t * kD)) : make_uint2(0u, 0u);
+            for (int t = 0; t < kTok; ++t) v[t] = __ldcs(reinterpret_cast<const uint2 *>(row0 + (size_t)t * kD));
+        } else {
+#pragma unroll
+            for (int t = 0; t < kTok; ++t)
+                v[t] = (t < n) ? __ldcs(reinterpret_cast<const uint2 *>(row0 + (size_t)t * kD)) : make_uint2(0u, 0u);
+        }
     }
     __device__ __forceinline__ void get(int t, float2 &x01, float2 &x23) const {
         x01 = make_float2(__uint_as_float(v[t].x << 16), __uint_as_float(v[t].x & 0xffff0000u));
@@ -107,10 +112,15 @@ template <> struct VRegs<float> {
     static constexpr int kTok = 16;
     float4 v[kTok];
     __device__ __forceinline__ void load(const float *row0, int n) {
+        if (n >= kTok) {
 #pragma unroll
-        for (int t = 0; t < kTok; ++t)
-            v[t] = (t < n) ? __ldcs(reinterpret_cast<const float4 *>(row0 + (size_t)t * kD))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int t = 0; t < kTok; ++t) v[t] = __ldcs(reinterpret_cast<const float4 *>(row0 + (size_t)t * kD));
+        } else {
+#pragma unroll
+            for (int t = 0; t < kTok; ++t)
+                v[t] = (t < n) ? __ldcs(reinterpret_cast<const float4 *>(row0 + (size_t)t * kD))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
     __device__ __forceinline__ void get(int t, float2 &x01, float2 &x23) const {
         x01 = make_float2(v[t].x, v[t].y);
@@ -211,12 +221,12 @@ __device__ __forceinline__ void tile_softmax(const WarpSmem<E, G> &ws, Flash<G> 
 
 // P.V over tokens [t_lo, t_lo + VRegs::kTok) of the tile (those < n), V rows
 // from registers, p from shared memory.
-template <typename E, int G>
-__device__ __forceinline__ void tile_pv(const WarpSmem<E, G> &ws, Flash<G> &f, const VRegs<E> &vr, int t_lo,
-                                        int n) {
+template <typename E, int G, bool kFull>
+__device__ __forceinline__ void tile_pv_impl(const WarpSmem<E, G> &ws, Flash<G> &f, const VRegs<E> &vr,
+                                             int t_lo, int n) {
 #pragma unroll
     for (int t = 0; t < VRegs<E>::kTok; ++t) {
-        if (t_lo + t < n) {
+        if (kFull || t_lo + t < n) {
             float2 x01, x23;
             vr.get(t, x01, x23);
             const float *pd = ws.pdup + (t_lo + t) * G * 2;
@@ -239,6 +249,13 @@ __device__ __forceinline__ void tile_pv(const WarpSmem<E, G> &ws, Flash<G> &f, c
     }
 }
 
+template <typename E, int G>
+__device__ __forceinline__ void tile_pv(const WarpSmem<E, G> &ws, Flash<G> &f, const VRegs<E> &vr, int t_lo,
+                                        int n) {
+    if (t_lo + VRegs<E>::kTok <= n) tile_pv_impl<E, G, true>(ws, f, vr, t_lo, n);
+    else tile_pv_impl<E, G, false>(ws, f, vr, t_lo, n);
+}
+
 // Write one item's partial state (acc[G][D], m, l) to the workspace.
 template <int G>
 __device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, Flash<G> &f) {
@@ -259,9 +276,10 @@ __device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, 
     }
 }
 
-// warps per CTA the kernel is compiled for: 16 (128 registers) up to G = 4,
-// 12 (168 registers) for G = 8
-__host__ __device__ constexpr int dec_max_warps(int G) { return G > 4 ? 12 : kMaxWarps; }
+// warps per CTA the kernel is compiled for: 16 (128 registers) for G <= 2,
+// 12 (168 registers, no spills) for G >= 4 -- measured faster than 16
+// spilling warps on the G = 4 workloads
+__host__ __device__ constexpr int dec_max_warps(int G) { return G > 2 ? 12 : kMaxWarps; }
 
 template <typename E, int G>
 __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArgs a) {
@@ -301,28 +319,37 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
     auto item_unit = [&](int item) -> int { return item < n_prompt ? item % a.n_pre : a.n_pre; };
 
     // ---- tile stream of this warp: prompt tiles of its items, in order
-    struct Cursor {
-        int item;
-        int tile;
-    };
-    auto item_tiles = [&](int item) -> int {
-        const int u = item_unit(item);
+    auto item_tiles = [&](int u) -> int {
         if (u >= a.n_pre) return 0;  // dense-tail items are not streamed
         const long t0 = (long)u * a.chunk;
         const long t1 = min((long)a.S, t0 + a.chunk);
         return t1 > t0 ? (int)((t1 - t0 + kWT - 1) / kWT) : 0;
     };
+    // issue cursor: the next prompt tile to copy, with its item decoded once
+    struct Cursor {
+        int item, tile, ntiles, bh, u;
+    };
+    auto enter = [&](Cursor &c) {
+        c.tile = 0;
+        if (c.item < n_items) {
+            c.bh = item_head(c.item);
+            c.u = item_unit(c.item);
+            c.ntiles = item_tiles(c.u);
+        } else {
+            c.ntiles = 0;
+        }
+    };
     auto settle = [&](Cursor &c) {  // move to the next tile that exists
-        while (c.item < n_items && c.tile >= item_tiles(c.item)) {
+        while (c.item < n_items && c.tile >= c.ntiles) {
             c.item += nwt;
-            c.tile = 0;
+            enter(c);
         }
     };
     const E *gvals = static_cast<const E *>(a.vals);
     const E *gv = static_cast<const E *>(a.v);
     auto issue = [&](int st, const Cursor &c) {
-        const long bh = item_head(c.item);
-        const int u = item_unit(c.item);
+        const long bh = c.bh;
+        const int u = c.u;
         const long t0 = (long)u * a.chunk + (long)c.tile * kWT;
         const long t1 = min((long)a.S, (long)u * a.chunk + a.chunk);
         const int n = (int)min((long)kWT, t1 - t0);
@@ -335,7 +362,8 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         if (vb) bulk_g2s(smem_u32(dst + kWT * 16), gvals + (size_t)bh * a.S32 * a.T + (size_t)t0 * a.T, vb, bar);
     };
 
-    Cursor ic{gw, 0};
+    Cursor ic{gw, 0, 0, 0, 0};
+    enter(ic);
     settle(ic);
     int issued = 0, consumed = 0;
     if (lane == 0) {
@@ -436,7 +464,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         }
 
         // ---- prompt tokens of this item, one 32-token tile at a time
-        const int ntiles = item_tiles(item);
+        const int ntiles = item_tiles(u);
         const long t_item = (long)u * a.chunk;
         const long t_end = min((long)a.S, t_item + a.chunk);
         const E *vbase = gv + (size_t)bh * a.S * kD + 4 * lane;

@@ -25,6 +25,8 @@
 // All reductions have a fixed order, so reruns are bit-identical.
 #include "spark_internal.cuh"
 
+#include <cuda_fp16.h>
+
 namespace spark {
 
 template <typename E>
@@ -109,24 +111,23 @@ __device__ __forceinline__ int quad_sum(int v) {
     return v;
 }
 
-// Count of the quad's keys >= mid, from the packed bf16-truncated keys
-// (the upper 16 bits of the fp32 saliency, two per register).  Truncation is
-// monotone, so this is the integer count over the 16-bit keys.  `mid` is 0 or
-// a normal bf16 pattern (>= 0x80), so no subnormal is ever compared; keys
-// below 0x80 (zero or subnormal saliency) are below every probe.  One packed
-// compare and one packed add per two channels; counts <= 32 per lane are
-// exact in bf16.
+// Count of the quad's keys >= mid over the packed 16-bit keys.  A key16 is
+// the upper half of the fp32 saliency (a positive bf16 pattern), clamped to
+// 0x7bff: read as fp16 bit patterns these stay in the same order, and fp16
+// packed compare + add (one instruction each per two channels) count them.
+// `mid` is 0 or >= 0x400 (a normal fp16 pattern); keys below 0x400 sit below
+// every probe.  Counts <= 32 per lane are exact in fp16.
 __device__ __forceinline__ int quad_count16(const uint32_t (&kp)[16], uint32_t mid) {
     const uint32_t mm = mid * 0x10001u;
-    const __nv_bfloat162 m2 = *reinterpret_cast<const __nv_bfloat162 *>(&mm);
-    const __nv_bfloat162 z = __float2bfloat162_rn(0.f);
-    __nv_bfloat162 a0 = z, a1 = z, a2 = z, a3 = z;
+    const __half2 m2 = *reinterpret_cast<const __half2 *>(&mm);
+    const __half2 z = __float2half2_rn(0.f);
+    __half2 a0 = z, a1 = z, a2 = z, a3 = z;
 #pragma unroll
     for (int i = 0; i < 16; i += 4) {
-        a0 = __hadd2(a0, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 0]), m2));
-        a1 = __hadd2(a1, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 1]), m2));
-        a2 = __hadd2(a2, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 2]), m2));
-        a3 = __hadd2(a3, __hge2(*reinterpret_cast<const __nv_bfloat162 *>(&kp[i + 3]), m2));
+        a0 = __hadd2(a0, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 0]), m2));
+        a1 = __hadd2(a1, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 1]), m2));
+        a2 = __hadd2(a2, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 2]), m2));
+        a3 = __hadd2(a3, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 3]), m2));
     }
     a0 = __hadd2(__hadd2(a0, a1), __hadd2(a2, a3));
     const int c = (int)(__low2float(a0) + __high2float(a0));
@@ -156,7 +157,7 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     if (T >= kD) return 0xffffffffu;
 
     // ---- phase 1: 16-bit keys.  count(>= lo) >= T > count(>= hi)
-    constexpr uint32_t kTop = 0x7f81u;  // above +inf: nothing reaches it
+    constexpr uint32_t kTop = 0x7c00u;  // above the clamp: nothing reaches it
     uint32_t lo = 0u, hi = kTop;
     int c_hi = 0;
     bool exact = false;
@@ -164,7 +165,7 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     uint32_t step = 64u;
     uint32_t mid = min(max(tau16, 1u), kTop - 1u);
     while (__any_sync(0xffffffffu, !done)) {
-        const uint32_t probe = (mid > 0u && mid < 0x80u) ? 0x80u : mid;
+        const uint32_t probe = (mid > 0u && mid < 0x400u) ? 0x400u : mid;
         const int c = quad_count16(kp, probe);
         if (!done) {
             if (c >= T) {
@@ -192,10 +193,12 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
 
     // ---- phase 2: exact keys inside the band of 16-bit key == lo.  Quads
     // whose phase 1 was exact skip it (done2) but stay in the uniform loop.
-    // When exact, exactly T keys have a 16-bit key >= lo (lo >= 1; no 16-bit
-    // key lies in [1, 0x80)), i.e. an fp32 key >= max(lo, 0x80) << 16.
-    uint32_t lo32 = exact ? (max(lo, 0x80u) << 16) : ((lo == 0u) ? 0u : (lo << 16));
-    uint32_t hi32 = (lo == 0u) ? 0x00800000u : ((lo + 1u) << 16);
+    // Bands in fp32 key space: [0, 0x400 << 16) for lo == 0 (every probe
+    // below 0x400 acts as 0x400), [0x7bff << 16, 2^31) for the clamp value,
+    // [lo << 16, (lo + 1) << 16) otherwise.  When exact, exactly T keys have a
+    // 16-bit key >= lo, i.e. an fp32 key >= max(lo, 0x400) << 16.
+    uint32_t lo32 = exact ? (max(lo, 0x400u) << 16) : ((lo == 0u) ? 0u : (lo << 16));
+    uint32_t hi32 = (lo == 0u) ? (0x400u << 16) : ((lo >= 0x7bffu) ? 0x80000000u : ((lo + 1u) << 16));
     bool exact32 = exact;
     bool done2 = exact || (hi32 - lo32 <= 1u);
     while (__any_sync(0xffffffffu, !done2)) {
@@ -217,20 +220,21 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     // channel order over the quad) are kept.
     const uint32_t thr = exact32 ? lo32 : lo32 + 1u;
     uint32_t m = 0u;
-    int e = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        m |= (key[i] >= thr ? 1u : 0u) << i;
-        e += (key[i] == lo32) ? 1 : 0;
-    }
-    int r = quad_excl_scan(e, s);
-    if (!exact32) {
-        const int need = T - c_hi;
+    for (int i = 0; i < 32; ++i) m |= (key[i] >= thr ? 1u : 0u) << i;
+    if (__any_sync(0xffffffffu, !exact32)) {  // warp-uniform: the scan below shuffles
+        int e = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (key[i] == lo32) {
-                if (r < need) m |= 1u << i;
-                ++r;
+        for (int i = 0; i < 32; ++i) e += (key[i] == lo32) ? 1 : 0;
+        int r = quad_excl_scan(e, s);
+        if (!exact32) {
+            const int need = T - c_hi;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (key[i] == lo32) {
+                    if (r < need) m |= 1u << i;
+                    ++r;
+                }
             }
         }
     }
@@ -257,8 +261,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     if (tid < kD) qs[(tid >> 5) * 36 + (tid & 31)] = __ldg(qn + bh * kD + tid);
     __syncthreads();
 
-    // the first token of each quad starts its threshold search at 1.0
-    uint32_t tau16 = 0x3f80u;
+    uint32_t tau16 = 0x3f80u;  // reset from the first token's keys below
     double acc_w = 0.0, acc_w2 = 0.0;
     const long g_first = (long)chunk * kPruneGroups;
     KSlice<E> ks, ks_next;
@@ -291,9 +294,29 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
                 key[4 * c + e] = __float_as_uint(__fmul_rn(qq[e], __uint_as_float(ks.abs_bits(4 * c + e))));
         }
         uint32_t kp[16];
+        {
+            const uint32_t cap = 0x7bff7bffu;
+            const __half2 cap2 = *reinterpret_cast<const __half2 *>(&cap);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) kp[i] = __byte_perm(key[2 * i], key[2 * i + 1], 0x7632);
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t pr = __byte_perm(key[2 * i], key[2 * i + 1], 0x7632);
+                const __half2 c = __hmin2(*reinterpret_cast<const __half2 *>(&pr), cap2);
+                kp[i] = *reinterpret_cast<const uint32_t *>(&c);
+            }
+        }
 
+        if (gi == 0) {
+            // first token of this quad: start 1.5 octaves (192 key16 units)
+            // below its largest key instead of at a fixed guess
+            __half2 mx = *reinterpret_cast<const __half2 *>(&kp[0]);
+#pragma unroll
+            for (int i = 1; i < 16; ++i) mx = __hmax2(mx, *reinterpret_cast<const __half2 *>(&kp[i]));
+            const uint32_t mb = *reinterpret_cast<const uint32_t *>(&mx);
+            uint32_t m16 = max(mb & 0xffffu, mb >> 16);
+            m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
+            m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
+            tau16 = m16 > 192u ? m16 - 192u : 1u;
+        }
         const uint32_t m = select_top_t(key, kp, T, s, tau16);
         if (valid) mask[((size_t)bh * S + t) * kMaskWords + s] = m;
 
