@@ -30,6 +30,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
+from channel_pruned_decode_b200 import dist as sd  # noqa: E402
 from channel_pruned_decode_b200.synth import (WORKLOADS, make_decode_step, make_prefill,  # noqa: E402
                                               scaled)
 
@@ -163,18 +164,11 @@ class Job:
 
 
 def _barrier(dist_on):
-    if dist_on:
-        import torch.distributed as dist
-        dist.barrier()
+    sd.barrier()
 
 
 def _max_over_ranks(x: float, dist_on: bool) -> float:
-    if not dist_on:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return sd.max_over_ranks(x, device="cuda") if dist_on else float(x)
 
 
 def _traffic_record(kernel: str, workload: str):
@@ -237,17 +231,12 @@ def cpu_baseline(wl, job, units: int | None = None):
 
 def run_gpu(args):
     dist_on = args.gpus > 1
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    # one process per GPU; every rank runs its own replica of the workload
+    # (independent (layer, batch, head) units: no data-path collective)
     if dist_on:
-        import datetime
-
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        rank, world = sd.init("nccl")
     else:
+        rank, world = 0, 1
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     wl = WORKLOADS[args.workload]
@@ -336,9 +325,7 @@ def run_gpu(args):
             "gpu_launches": job.launches_per_step * args.steps,
         }
         print(json.dumps(line), flush=True)
-    if dist_on:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    sd.finalize()
 
 
 def run_e2e(job, wl, steps, dist_on, world):

@@ -60,11 +60,12 @@ def _bind(lib):
     lib.oracle_recover_keys.restype = None
     lib.oracle_decode.argtypes = [P, P, P, P, P, P, P, P, L, L, L, I, L, I, I, P]
     lib.oracle_decode.restype = None
-    if hasattr(lib, "oracle_snapkv_scores"):
-        lib.oracle_snapkv_scores.argtypes = [P, P, L, I, I, L, I, P]
-        lib.oracle_snapkv_scores.restype = None
-        lib.oracle_snapkv_select.argtypes = [P, L, L, I, I, I, P]
-        lib.oracle_snapkv_select.restype = None
+    lib.oracle_snapkv_scores.argtypes = [P, P, L, I, I, L, I, P]
+    lib.oracle_snapkv_scores.restype = None
+    lib.oracle_snapkv_pool.argtypes = [P, L, L, I, P]
+    lib.oracle_snapkv_pool.restype = None
+    lib.oracle_snapkv_select.argtypes = [P, L, L, I, I, P]
+    lib.oracle_snapkv_select.restype = None
     return lib
 
 
@@ -155,3 +156,36 @@ def decode(q, mask, vals, qn, stats, v, k_tail=None, v_tail=None, n_tail: int = 
     lib.oracle_decode(_ptr(q), _ptr(mask), _ptr(vals), _ptr(qn), _ptr(stats), _ptr(v),
                       _ptr(k_tail), _ptr(v_tail), cap, n_tail, BH, G, S, D, T, _ptr(out))
     return out
+
+
+def snapkv_scores(q_obs, k, G: int, lib=None) -> np.ndarray:
+    """Summed window-attention probabilities of the prefix tokens (reading
+    R11).  q_obs: [BH*G, W, D]; k: [BH, S, D].  Returns [BH, S-W] fp64."""
+    lib = lib or load()
+    q = _f32(q_obs)
+    k = _f32(k)
+    BH, S, D = k.shape
+    W = q.shape[-2]
+    out = np.zeros((BH, max(S - W, 0)), np.float64)
+    lib.oracle_snapkv_scores(_ptr(q), _ptr(k), BH, G, W, S, D, _ptr(out))
+    return out
+
+
+def snapkv_pool(scores, pool: int, lib=None) -> np.ndarray:
+    """1-D max-pool of the scores along tokens (reading R12)."""
+    lib = lib or load()
+    sc = np.ascontiguousarray(scores, np.float64)
+    BH, P = sc.shape
+    out = np.empty_like(sc)
+    lib.oracle_snapkv_pool(_ptr(sc), BH, P, pool, _ptr(out))
+    return out
+
+
+def snapkv_select(pooled, S: int, W: int, keep: int, lib=None) -> np.ndarray:
+    """Kept token indices [BH, keep] in original order (reading R13)."""
+    lib = lib or load()
+    pl = np.ascontiguousarray(pooled, np.float64)
+    BH = pl.shape[0]
+    idx = np.empty((BH, keep), np.int64)
+    lib.oracle_snapkv_select(_ptr(pl), BH, S, W, keep, _ptr(idx))
+    return idx

@@ -229,3 +229,104 @@ void oracle_decode(const float *q, const uint32_t *mask, const float *vals,
     free(s);
     free(acc);
 }
+
+/*
+ * SnapKV-style token eviction pre-pass, which [W] stacks SparK on (sections 2
+ * and 4.1: SnapKV / PyramidKV bases; 3.2: SparK reuses SnapKV's observation
+ * window).  The pages give no detail of SnapKV itself; the reading used here:
+ *   R11 the W window queries are the last W prompt positions p = S-W+w; each
+ *       of the G*W (query head, window row) pairs attends causally over keys
+ *       0..p with scale 1/sqrt(D); the score of a prefix token t < P = S-W is
+ *       the sum of its probabilities over the G*W rows;
+ *   R12 scores are max-pooled along t with kernel `pool` (odd), stride 1 and
+ *       half-width padding that never wins (max over the in-range window);
+ *   R13 keep-W prefix tokens with the largest pooled score (ties -> lower t)
+ *       plus all W window tokens are kept, in original order.
+ */
+void oracle_snapkv_scores(const float *q_obs, const float *k, long BH, int G, int W,
+                          long S, int D, double *scores /* [BH][S-W] */)
+{
+    const long P = S - W;
+    const double scale = 1.0 / sqrt((double)D);
+    double *logit = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+    for (long bh = 0; bh < BH; ++bh) {
+        double *sc = scores + bh * (P > 0 ? P : 0);
+        for (long t = 0; t < P; ++t)
+            sc[t] = 0.0;
+        for (int g = 0; g < G; ++g)
+            for (int w = 0; w < W; ++w) {
+                const float *q = q_obs + ((bh * G + g) * (long)W + w) * D;
+                const long p = P + w; /* this query's position */
+                double m = -INFINITY;
+                for (long t = 0; t <= p; ++t) {
+                    const float *kr = k + (bh * S + t) * D;
+                    double dot = 0.0;
+                    for (int j = 0; j < D; ++j)
+                        dot += (double)q[j] * (double)kr[j];
+                    logit[t] = dot * scale;
+                    if (logit[t] > m)
+                        m = logit[t];
+                }
+                double l = 0.0;
+                for (long t = 0; t <= p; ++t)
+                    l += exp(logit[t] - m);
+                for (long t = 0; t < P; ++t)
+                    sc[t] += exp(logit[t] - m) / l;
+            }
+    }
+    free(logit);
+}
+
+void oracle_snapkv_pool(const double *scores, long BH, long P, int pool, double *pooled)
+{
+    const int h = pool / 2;
+    for (long bh = 0; bh < BH; ++bh)
+        for (long t = 0; t < P; ++t) {
+            double m = -INFINITY;
+            for (long u = t - h; u <= t + h; ++u)
+                if (u >= 0 && u < P && scores[bh * P + u] > m)
+                    m = scores[bh * P + u];
+            pooled[bh * P + t] = m;
+        }
+}
+
+typedef struct {
+    double s;
+    long t;
+} tok_score;
+
+static int by_score_desc(const void *pa, const void *pb)
+{
+    const tok_score *a = (const tok_score *)pa, *b = (const tok_score *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->t > b->t) - (a->t < b->t);
+}
+
+static int by_index_asc(const void *pa, const void *pb)
+{
+    long a = *(const long *)pa, b = *(const long *)pb;
+    return (a > b) - (a < b);
+}
+
+/* Kept token indices [BH][keep] in original order (R13). */
+void oracle_snapkv_select(const double *pooled, long BH, long S, int W, int keep, long *idx)
+{
+    const long P = S - W;
+    const long kp = keep - W; /* prefix tokens kept */
+    tok_score *ord = (tok_score *)malloc(sizeof(tok_score) * (size_t)(P > 0 ? P : 1));
+    for (long bh = 0; bh < BH; ++bh) {
+        long *out = idx + bh * keep;
+        for (long t = 0; t < P; ++t) {
+            ord[t].s = pooled[bh * P + t];
+            ord[t].t = t;
+        }
+        qsort(ord, (size_t)P, sizeof(tok_score), by_score_desc);
+        for (long i = 0; i < kp; ++i)
+            out[i] = ord[i].t;
+        qsort(out, (size_t)kp, sizeof(long), by_index_asc);
+        for (int w = 0; w < W; ++w)
+            out[kp + w] = P + w;
+    }
+    free(ord);
+}
