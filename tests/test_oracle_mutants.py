@@ -12,7 +12,8 @@ import pytest
 import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_snapkv_pins.py")]
 
 MUTANTS = {
     "tie_rule_reversed": ("return (a->j > b->j) - (a->j < b->j);",
@@ -29,7 +30,17 @@ MUTANTS = {
     "mean_wrong_denominator": ("? sw / n : 0.0;", "? sw / (n + 1.0) : 0.0;"),
     "keeps_one_less": ("for (int r = 0; r < T; ++r)", "for (int r = 0; r < T - 1; ++r)"),
     "vals_reversed": ("vrow[pos++] = krow[j];", "vrow[T - 1 - pos++] = krow[j];"),
-    "score_scale_1_over_D": ("1.0 / sqrt((double)D);", "1.0 / (double)D;"),
+    "score_scale_1_over_D": ("const double scale = 1.0 / sqrt((double)D);\n    for (long bh = 0; bh < BH; ++bh) {\n        oracle_recover_keys",
+                             "const double scale = 1.0 / (double)D;\n    for (long bh = 0; bh < BH; ++bh) {\n        oracle_recover_keys"),
+    # SnapKV pre-pass (readings R11-R13)
+    "snapkv_normaliser_not_causal": ("for (long t = 0; t <= p; ++t)\n                    l += exp(logit[t] - m);",
+                                     "for (long t = 0; t < S; ++t)\n                    l += exp(logit[t] - m);"),
+    "snapkv_one_head": ("for (int g = 0; g < G; ++g)\n            for (int w = 0; w < W; ++w) {\n                const float *q = q_obs",
+                        "for (int g = 0; g < 1; ++g)\n            for (int w = 0; w < W; ++w) {\n                const float *q = q_obs"),
+    "snapkv_unnormalised": ("sc[t] += exp(logit[t] - m) / l;", "sc[t] += exp(logit[t] - m);"),
+    "snapkv_pool_narrow": ("for (long u = t - h; u <= t + h; ++u)", "for (long u = t - h + 1; u <= t + h; ++u)"),
+    "snapkv_ties_reversed": ("return (a->t > b->t) - (a->t < b->t);", "return (a->t < b->t) - (a->t > b->t);"),
+    "snapkv_drops_window": ("out[kp + w] = P + w;", "out[kp + w] = P + w - 1;"),
     "gqa_transposed": ("const float *qrow = q + (bh * G + g) * (long)D;",
                        "const float *qrow = q + ((long)g * BH + bh) * (long)D;"),
     "tail_keys_from_values": ("(double)k_tail[(bh * tail_cap + t) * D + j];",
@@ -48,6 +59,6 @@ def test_pins_catch_planted_mistake(tmp_path, name):
     mutant_c.write_text(src.replace(before, after))
     lib = oracle.build(force=True, src=str(mutant_c), out=str(tmp_path / "libmutant.so"))
     env = dict(os.environ, ORACLE_LIB=lib)
-    r = subprocess.run([sys.executable, "-m", "pytest", PINS, "-x", "-q", "-p", "no:cacheprovider"],
+    r = subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
