@@ -27,10 +27,11 @@ SPARK_F_GAUSSIAN = 1
 SPARK_F_EXPONENTIAL = 2
 SPARK_OP_PRUNE = 0
 SPARK_OP_DECODE = 1
+SPARK_OP_SNAPKV = 2
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
            "spark_prune", "spark_prune_noalloc", "spark_decode_attn", "spark_tail_append", "spark_device_status",
-           "spark_status_str")
+           "spark_status_str", "spark_snapkv_evict")
 
 
 class SparkError(RuntimeError):
@@ -72,6 +73,8 @@ def lib():
         L.spark_decode_attn.argtypes = [P, ctypes.POINTER(spark_kcache), P, P, P, I, I, I, I,
                                         ctypes.c_ulonglong, P, P, Z, P]
         L.spark_decode_attn.restype = I
+        L.spark_snapkv_evict.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P, Z, P]
+        L.spark_snapkv_evict.restype = I
         L.spark_tail_append.argtypes = [P, P, P, P, I, I, I, I, I, I, P]
         L.spark_tail_append.restype = I
         L.spark_device_status.argtypes = [P, ctypes.POINTER(I), I, P]
@@ -194,6 +197,18 @@ def spark_decode_attn(q: torch.Tensor, kc: KCache, v: torch.Tensor, k_tail, v_ta
                                  n_tail, G, recovery, seed, _ptr(out), _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_decode_attn")
+
+
+def spark_snapkv_evict(k: torch.Tensor, v: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, keep: int,
+                       pool: int, k_out: torch.Tensor, v_out: torch.Tensor, idx_out: torch.Tensor,
+                       ws: torch.Tensor, stream=None) -> None:
+    """SnapKV-style eviction: k, v [B, Hkv, S, D] -> k_out, v_out [B, Hkv, keep, D],
+    idx_out int32 [B, Hkv, keep]."""
+    B, H, S, D = k.shape
+    rc = lib().spark_snapkv_evict(_ptr(k), _ptr(v), _ptr(q_obs), B, H, S, D, G, W, keep, pool,
+                                  _dtype_code(k.dtype), _ptr(k_out), _ptr(v_out), _ptr(idx_out), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_snapkv_evict")
 
 
 def spark_tail_append(k_new, v_new, k_tail, v_tail, B, Hkv, D, tail_cap, slot, stream=None) -> None:

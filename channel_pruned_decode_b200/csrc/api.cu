@@ -11,6 +11,12 @@ cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const s
 cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const void *k_tail,
                           const void *v_tail, int tail_cap, int n_tail, int G, float *out, void *ws,
                           const DecodeGeom &geo, cudaStream_t st);
+cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
+                          int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st);
+
+static size_t snapkv_workspace(long BH, int S, int W) {
+    return kWsHeader + (size_t)BH * (size_t)(S - W) * 8;
+}
 
 static int elem_size(int dtype) {
     return dtype == SPARK_F32 ? 4 : (dtype == SPARK_BF16 ? 2 : 0);
@@ -93,6 +99,7 @@ size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D, int T,
     if (B < 0 || Hkv < 0 || S < 0 || D != kD || T < 0 || T > D || G < 1 || n_tail < 0) return 0;
     const long BH = (long)B * Hkv;
     if (op == SPARK_OP_PRUNE) return round256(prune_workspace(BH, S));
+    if (op == SPARK_OP_SNAPKV) return round256(snapkv_workspace(BH, S, 0));
     if (op == SPARK_OP_DECODE) {
         if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
         // the geometry depends on the element size only through the stage
@@ -145,6 +152,26 @@ int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, cons
     if (BH * (long)geo.units >= (1L << 31)) return SPARK_ERR_UNSUPPORTED;  // 32-bit item indices
     if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
     cudaError_t e = launch_decode(q, *kc, v, k_tail, v_tail, tail_cap, n_tail, G, out, workspace, geo,
+                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_snapkv_evict(const void *k, const void *v, const void *q_obs, int B, int Hkv, int S, int D, int G,
+                       int W, int keep, int pool, int dtype, void *k_out, void *v_out, int32_t *idx_out,
+                       void *workspace, size_t ws_bytes, void *stream) {
+    if (B < 0 || Hkv < 0 || S < 0 || G < 1 || W < 1 || elem_size(dtype) == 0) return SPARK_ERR_ARG;
+    if (D != kD || dtype != SPARK_BF16) return SPARK_ERR_UNSUPPORTED;
+    if ((G * W) % 16 != 0 || G * W > 128) return SPARK_ERR_UNSUPPORTED;
+    if (keep < W || keep > S || pool < 1 || (pool & 1) == 0) return SPARK_ERR_ARG;
+    const long BH = (long)B * Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!k || !v || !q_obs || !k_out || !v_out || !idx_out) return SPARK_ERR_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(q_obs) || !aligned16(k_out) || !aligned16(v_out) ||
+        !aligned16(idx_out))
+        return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < snapkv_workspace(BH, S, W)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_snapkv(k, v, q_obs, BH, S, G, W, keep, pool, k_out, v_out, idx_out, workspace,
                                   static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }

@@ -65,7 +65,7 @@ typedef enum {
     SPARK_F_EXPONENTIAL = 2   /* w~ ~ Exp(1/mu)        (not built: UNSUPPORTED) */
 } spark_recovery;
 
-typedef enum { SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1 } spark_op;
+typedef enum { SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1, SPARK_OP_SNAPKV = 2 } spark_op;
 
 /*
  * The packed key cache of [W] 3.3 step 1 / Fig. 3: per token the kept key
@@ -111,7 +111,8 @@ SPARK_API size_t spark_cache_bytes(int B, int Hkv, int S, int D, int T, int dtyp
 /* Workspace bytes that `op` needs for the given shape (device memory,
  * 256-byte aligned, caller-owned; its first 4 bytes hold the device status
  * word and must be zero before first use).  For SPARK_OP_DECODE pass the
- * tail capacity as n_tail.  Depends on the current device's SM count.
+ * tail capacity as n_tail; for SPARK_OP_SNAPKV, S is the prompt length and T
+ * and n_tail are ignored.  Depends on the current device's SM count.
  * Returns 0 on bad arguments. */
 SPARK_API size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D,
                              int T, int n_tail);
@@ -186,6 +187,31 @@ SPARK_API int spark_decode_attn(const void *q, const spark_kcache *kc, const voi
                       int n_tail, int G, int recovery, unsigned long long seed,
                       float *out, void *workspace, size_t ws_bytes,
                       void *stream);
+
+/*
+ * SnapKV-style token eviction, the pre-pass SparK is stacked on ([W] 2 and
+ * 4.1: SnapKV / PyramidKV bases; 3.2: the observation window).  The pages do
+ * not define SnapKV; this build reads it as follows:
+ *   - the W window queries are the last W prompt positions p = S-W+w; each of
+ *     the G*W (query head, window row) rows attends causally over keys 0..p
+ *     (scale 1/sqrt(D)); a prefix token's score (t < S-W) is the sum of its
+ *     softmax probabilities over the G*W rows;
+ *   - scores are max-pooled along t (kernel `pool`, odd, stride 1, window
+ *     clipped to the prefix);
+ *   - the keep-W prefix tokens with the largest pooled score (ties -> lower
+ *     t) and all W window tokens are kept, in original order.
+ *   k, v   [B][Hkv][S][D] bf16;  q_obs [B][Hkv*G][W][D] bf16
+ *   k_out, v_out [B][Hkv][keep][D] bf16 (caller-owned, not aliasing k, v)
+ *   idx_out int32 [B][Hkv][keep]: kept token indices, ascending.
+ * Requires bf16, D == 128, G*W a multiple of 16 and <= 128, 1 <= W <= keep
+ * <= S, odd pool >= 1, and spark_workspace_bytes(SPARK_OP_SNAPKV, ...).
+ * Logits are bf16 x bf16 products accumulated in fp32 on tensor cores;
+ * probabilities and scores are fp32.
+ */
+SPARK_API int spark_snapkv_evict(const void *k, const void *v, const void *q_obs, int B, int Hkv,
+                                 int S, int D, int G, int W, int keep, int pool, int dtype,
+                                 void *k_out, void *v_out, int32_t *idx_out, void *workspace,
+                                 size_t ws_bytes, void *stream);
 
 /*
  * Append one unpruned decode-time key/value per (row, kv head) into the
