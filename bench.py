@@ -56,9 +56,10 @@ def _workload_desc(wl, T):
 
 
 def _byte_model(wl, T, n_tail):
-    """Algorithmic HBM bytes per launch of the two heavy calls."""
+    """Algorithmic HBM bytes per launch of the two heavy calls (on the
+    prompt as it stands after any eviction)."""
     es = 2 if wl.dtype == "bf16" else 4
-    BH, S, D, G = wl.BH, wl.S, wl.D, wl.G
+    BH, S, D, G = wl.BH, wl.S_kept, wl.D, wl.G
     prune = BH * S * (D * es + 16 + T * es) + BH * G * wl.W * D * es + BH * (D * 4 + 32)
     decode = (BH * S * (16 + T * es + D * es) + BH * n_tail * 2 * D * es
               + BH * G * D * (es + 4) + BH * (D * 4 + 32))
@@ -144,20 +145,40 @@ class Job:
         self.out = torch.empty((R, wl.Hq, D), dtype=torch.float32, device=dev)
         self.n_tail = 0
         self.launches_per_step = 6  # qnorm, prune, stats, tail append, decode, combine
+        self.S_kept = S
+        if wl.keep:
+            # SnapKV-style eviction first: the cache then holds `keep` tokens
+            self.S_kept = wl.keep
+            self.k_ev = torch.empty((R, H, wl.keep, D), dtype=wl.torch_dtype, device=dev)
+            self.v_ev = torch.empty_like(self.k_ev)
+            self.idx = torch.empty((R, H, wl.keep), dtype=torch.int32, device=dev)
+            self.wse = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_SNAPKV, R, H, G, S, D, 0, 0), dev)
+            self.kc = sp.KCache.empty(R, H, wl.keep, D, self.T, wl.torch_dtype, device=dev)
+            self.wsp = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_PRUNE, R, H, G, wl.keep, D, self.T, 0), dev)
+            self.wsd = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_DECODE, R, H, G, wl.keep, D, self.T,
+                                                             self.cap), dev)
+            self.launches_per_step += 3  # scores, select, gather
 
     def step(self, stream, ev=None):
         sp, wl = self.sp, self.wl
         slot = 0  # one decode step per bench step: the tail holds this step's token
+        k, v = self.k, self.v
+        if ev is not None:
+            ev[4].record(stream)
+        if wl.keep:
+            sp.spark_snapkv_evict(self.k, self.v, self.q_obs, wl.G, wl.W, wl.keep, wl.pool, self.k_ev, self.v_ev,
+                                  self.idx, self.wse, stream)
+            k, v = self.k_ev, self.v_ev
         if ev is not None:
             ev[0].record(stream)
-        sp.spark_prune(self.k, self.q_obs, wl.G, wl.W, self.kc, self.wsp, stream)
+        sp.spark_prune(k, self.q_obs, wl.G, wl.W, self.kc, self.wsp, stream)
         if ev is not None:
             ev[1].record(stream)
         sp.spark_tail_append(self.k_new, self.v_new, self.kt, self.vt, wl.rows, wl.Hkv, wl.D, self.cap,
                              slot, stream)
         if ev is not None:
             ev[2].record(stream)
-        sp.spark_decode_attn(self.q, self.kc, self.v, self.kt, self.vt, self.cap, slot + 1, wl.G,
+        sp.spark_decode_attn(self.q, self.kc, v, self.kt, self.vt, self.cap, slot + 1, wl.G,
                              self.out, self.wsd, stream=stream)
         if ev is not None:
             ev[3].record(stream)
@@ -251,7 +272,7 @@ def run_gpu(args):
             job.step(stream)
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index) if rank == 0 else None
     _barrier(dist_on)
@@ -271,13 +292,14 @@ def run_gpu(args):
     prune_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     decode_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
     append_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    evict_ms = sum(e[4].elapsed_time(e[0]) for e in evs) / args.steps
     ms = _max_over_ranks(ms_local, dist_on)
     st = job.sp.spark_device_status(job.wsd)
     st |= job.sp.spark_device_status(job.wsp)
     if st != 0:
         raise RuntimeError(f"device status {st} after timed region")
 
-    token_heads = wl.BH * (wl.S + 1)
+    token_heads = wl.BH * (wl.S_kept + 1)
     ms_per_step = ms / args.steps
     value = world * token_heads / (ms_per_step / 1e3)
     bm = _byte_model(wl, job.T, 1)
@@ -307,7 +329,8 @@ def run_gpu(args):
             "config": {"workload": _workload_desc(wl, job.T), "B": wl.B, "layers": wl.L, "Hkv": wl.Hkv,
                        "G": wl.G, "S": wl.S, "D": wl.D, "W": wl.W, "lambda": wl.lam, "T": job.T,
                        "parallelism": f"replicas x{world} (independent (layer, head) work per GPU)",
-                       "l2": "inputs (K, V: 17.2 GB) exceed the 126 MB L2; no flush needed"},
+                       "l2": f"inputs (K, V: {2 * wl.BH * wl.S * wl.D * (2 if wl.dtype == 'bf16' else 4) / 1e9:.1f} GB) "
+                             "exceed the 126 MB L2; no flush needed"},
             "decode": {"us_per_step": decode_ms * 1e3, "gbs": decode_gbs,
                        "frac_8tbs": decode_gbs / NOMINAL_HBM_GBS, f"frac_{peak_kind}": decode_gbs / peak,
                        "token_heads_per_s": world * token_heads / (decode_ms / 1e3),
@@ -315,6 +338,7 @@ def run_gpu(args):
             "prune": {"us_per_step": prune_ms * 1e3, "gbs": prune_gbs, "frac_8tbs": prune_gbs / NOMINAL_HBM_GBS,
                       f"frac_{peak_kind}": prune_gbs / peak, "bytes_per_step": bm["prune"]},
             "tail_append_us": append_ms * 1e3,
+            "snapkv_evict_us": evict_ms * 1e3 if wl.keep else None,
             "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic,
@@ -367,7 +391,7 @@ def run_e2e(job, wl, steps, dist_on, world):
     ms = _max_over_ranks(start.elapsed_time(end), dist_on) / steps
     h2d = need
     d2h = hout.numel() * hout.element_size()
-    return {"value": world * wl.BH * (wl.S + 1) / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": world * wl.BH * (wl.S_kept + 1) / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
 
 

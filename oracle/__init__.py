@@ -60,6 +60,14 @@ def _bind(lib):
     lib.oracle_recover_keys.restype = None
     lib.oracle_decode.argtypes = [P, P, P, P, P, P, P, P, L, L, L, I, L, I, I, P]
     lib.oracle_decode.restype = None
+    lib.oracle_philox4x32_10.argtypes = [P, P, P]
+    lib.oracle_philox4x32_10.restype = None
+    lib.oracle_sample_score.argtypes = [I, P, ctypes.c_ulonglong, L, L, I]
+    lib.oracle_sample_score.restype = ctypes.c_double
+    lib.oracle_recover_keys_f.argtypes = [P, P, P, P, L, L, I, I, I, ctypes.c_ulonglong, P]
+    lib.oracle_recover_keys_f.restype = None
+    lib.oracle_decode_f.argtypes = [P, P, P, P, P, P, P, P, L, L, L, I, L, I, I, I, ctypes.c_ulonglong, P]
+    lib.oracle_decode_f.restype = None
     lib.oracle_snapkv_scores.argtypes = [P, P, L, I, I, L, I, P]
     lib.oracle_snapkv_scores.restype = None
     lib.oracle_snapkv_pool.argtypes = [P, L, L, I, P]
@@ -189,3 +197,62 @@ def snapkv_select(pooled, S: int, W: int, keep: int, lib=None) -> np.ndarray:
     idx = np.empty((BH, keep), np.int64)
     lib.oracle_snapkv_select(_ptr(pl), BH, S, W, keep, _ptr(idx))
     return idx
+
+
+DEGENERATE, GAUSSIAN, EXPONENTIAL = 0, 1, 2
+
+
+def philox4x32_10(ctr, key, lib=None):
+    """Philox4x32-10 of one counter block (reading R14)."""
+    lib = lib or load()
+    c = np.ascontiguousarray(ctr, np.uint32)
+    k = np.ascontiguousarray(key, np.uint32)
+    out = np.empty(4, np.uint32)
+    lib.oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def sample_score(mode: int, stats_row, seed: int, bh: int, t: int, j: int, lib=None) -> float:
+    lib = lib or load()
+    st = np.ascontiguousarray(stats_row, np.float64)
+    return float(lib.oracle_sample_score(mode, _ptr(st), seed, bh, t, j))
+
+
+def recover_keys_f(mask, vals, qn, stats, bh: int, mode: int, seed: int, lib=None) -> np.ndarray:
+    lib = lib or load()
+    mask = np.ascontiguousarray(mask, np.uint32)
+    vals = _f32(vals)
+    qn = _f32(qn)
+    stats = np.ascontiguousarray(stats, np.float64)
+    BH, S, _ = mask.shape
+    D = qn.shape[-1]
+    T = vals.shape[-1]
+    out = np.empty((S, D), np.float64)
+    lib.oracle_recover_keys_f(_ptr(mask), _ptr(vals), _ptr(qn), _ptr(stats), bh, S, D, T, mode, seed, _ptr(out))
+    return out
+
+
+def decode_f(q, mask, vals, qn, stats, v, k_tail=None, v_tail=None, n_tail: int = 0, G: int = 1,
+             mode: int = DEGENERATE, seed: int = 0, lib=None) -> np.ndarray:
+    """Decode with recovery F (Degenerate, Gaussian or Exponential)."""
+    lib = lib or load()
+    q = _f32(q)
+    mask = np.ascontiguousarray(mask, np.uint32)
+    vals = _f32(vals)
+    qn = _f32(qn)
+    stats = np.ascontiguousarray(stats, np.float64)
+    v = _f32(v)
+    BH, D = qn.shape
+    S = mask.shape[1]
+    T = vals.shape[-1]
+    if k_tail is None:
+        cap = max(n_tail, 1)
+        k_tail = np.zeros((BH, cap, D), np.float32)
+        v_tail = np.zeros((BH, cap, D), np.float32)
+    k_tail = _f32(k_tail)
+    v_tail = _f32(v_tail)
+    cap = k_tail.shape[1]
+    out = np.empty((BH * G, D), np.float32)
+    lib.oracle_decode_f(_ptr(q), _ptr(mask), _ptr(vals), _ptr(qn), _ptr(stats), _ptr(v), _ptr(k_tail),
+                        _ptr(v_tail), cap, n_tail, BH, G, S, D, T, mode, seed, _ptr(out))
+    return out

@@ -43,7 +43,11 @@
  *   q, out [BH*G][D]; k_tail, v_tail [BH][tail_cap][D]
  * Query head g of kv head h is row h*G + g (consecutive GQA grouping).
  */
+#define _USE_MATH_DEFINES
 #include <math.h>
+#ifndef M_PI
+#define M_PI 3.14159265358979323846
+#endif
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -329,4 +333,140 @@ void oracle_snapkv_select(const double *pooled, long BH, long S, int W, int keep
             out[kp + w] = P + w;
     }
     free(ord);
+}
+
+/*
+ * Sampling recoveries of the F table ([W] 3.3): Gaussian w~ ~ N(mu, sigma^2)
+ * and Exponential w~ ~ Exp(1/mu) (mean mu).  Reading R14 (the pages do not
+ * say when or how the score is drawn): one draw per pruned (token, channel)
+ * entry, fixed for a given seed, from the counter-based generator
+ * Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+ * easy as 1, 2, 3", SC'11) with counter (t, j, bh low word, bh high word) and
+ * key (seed low word, seed high word).  Uniforms from the top 24 bits:
+ * u1 = (x0 >> 8 + 1) / 2^24 in (0, 1], u2 = (x1 >> 8) / 2^24 in [0, 1).
+ * Gaussian: mu + sigma * sqrt(-2 ln u1) * cos(2 pi u2) (Box-Muller), with
+ * mu, sigma the mean and population standard deviation of the pruned
+ * saliencies of the head; Exponential: -mu ln u1.
+ */
+static void philox_round(uint32_t c[4], const uint32_t k[2])
+{
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c[0];
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c[2];
+    const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    const uint32_t n0 = hi1 ^ c[1] ^ k[0], n2 = hi0 ^ c[3] ^ k[1];
+    c[0] = n0;
+    c[1] = lo1;
+    c[2] = n2;
+    c[3] = lo0;
+}
+
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+    uint32_t k[2] = {key[0], key[1]};
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k[0] += 0x9E3779B9u;
+            k[1] += 0xBB67AE85u;
+        }
+        philox_round(c, k);
+    }
+    for (int i = 0; i < 4; ++i)
+        out[i] = c[i];
+}
+
+/* mode: 0 Degenerate, 1 Gaussian, 2 Exponential.  Returns the sampled score. */
+double oracle_sample_score(int mode, const double *st, unsigned long long seed, long bh, long t, int j)
+{
+    const double mu = st[3];
+    if (mode == 0)
+        return mu;
+    uint32_t ctr[4] = {(uint32_t)t, (uint32_t)j, (uint32_t)((unsigned long long)bh & 0xffffffffu),
+                       (uint32_t)((unsigned long long)bh >> 32)};
+    uint32_t key[2] = {(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
+    uint32_t x[4];
+    oracle_philox4x32_10(ctr, key, x);
+    const double u1 = (double)((x[0] >> 8) + 1u) / 16777216.0;
+    const double u2 = (double)(x[1] >> 8) / 16777216.0;
+    if (mode == 2)
+        return -mu * log(u1);
+    double var = (st[0] > 0.0) ? st[2] / st[0] - mu * mu : 0.0;
+    if (var < 0.0)
+        var = 0.0;
+    return mu + sqrt(var) * sqrt(-2.0 * log(u1)) * cos(2.0 * M_PI * u2);
+}
+
+/* Recovered keys with any F ([W] 3.3 steps 2-4): k~_j = w~ / qn_j. */
+void oracle_recover_keys_f(const uint32_t *mask, const float *vals, const float *qn, const double *stats,
+                           long bh, long S, int D, int T, int mode, unsigned long long seed, double *Kt)
+{
+    const int nw = (D + 31) / 32;
+    for (long t = 0; t < S; ++t) {
+        const uint32_t *mrow = mask + (bh * S + t) * nw;
+        const float *vrow = vals + (bh * S + t) * (long)T;
+        int pos = 0;
+        for (int j = 0; j < D; ++j) {
+            int kept = (mrow[j / 32] >> (j % 32)) & 1u;
+            if (kept) {
+                Kt[t * D + j] = (double)vrow[pos++];
+            } else {
+                double qj = (double)qn[bh * D + j];
+                double w = oracle_sample_score(mode, stats + bh * 4, seed, bh, t, j);
+                Kt[t * D + j] = (qj > 0.0) ? w / qj : 0.0;
+            }
+        }
+    }
+}
+
+/* Decode with any F: as oracle_decode, keys recovered by oracle_recover_keys_f. */
+void oracle_decode_f(const float *q, const uint32_t *mask, const float *vals, const float *qn,
+                     const double *stats, const float *v, const float *k_tail, const float *v_tail,
+                     long tail_cap, long n_tail, long BH, int G, long S, int D, int T, int mode,
+                     unsigned long long seed, float *out)
+{
+    const long L = S + n_tail;
+    double *Kt = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * (size_t)D);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *acc = (double *)malloc(sizeof(double) * (size_t)D);
+    const double scale = 1.0 / sqrt((double)D);
+    for (long bh = 0; bh < BH; ++bh) {
+        oracle_recover_keys_f(mask, vals, qn, stats, bh, S, D, T, mode, seed, Kt);
+        for (long t = 0; t < n_tail; ++t)
+            for (int j = 0; j < D; ++j)
+                Kt[(S + t) * D + j] = (double)k_tail[(bh * tail_cap + t) * D + j];
+        for (int g = 0; g < G; ++g) {
+            const float *qrow = q + (bh * G + g) * (long)D;
+            float *orow = out + (bh * G + g) * (long)D;
+            if (L == 0) {
+                for (int d = 0; d < D; ++d)
+                    orow[d] = 0.0f;
+                continue;
+            }
+            double m = -INFINITY;
+            for (long t = 0; t < L; ++t) {
+                double dot = 0.0;
+                for (int j = 0; j < D; ++j)
+                    dot += (double)qrow[j] * Kt[t * D + j];
+                s[t] = dot * scale;
+                if (s[t] > m)
+                    m = s[t];
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; ++d)
+                acc[d] = 0.0;
+            for (long t = 0; t < L; ++t) {
+                double p = exp(s[t] - m);
+                const float *vrow = (t < S) ? v + (bh * S + t) * D : v_tail + (bh * tail_cap + (t - S)) * D;
+                l += p;
+                for (int d = 0; d < D; ++d)
+                    acc[d] += p * (double)vrow[d];
+            }
+            for (int d = 0; d < D; ++d)
+                orow[d] = (float)(acc[d] / l);
+        }
+    }
+    free(Kt);
+    free(s);
+    free(acc);
 }

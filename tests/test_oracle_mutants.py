@@ -13,7 +13,8 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_snapkv_pins.py")]
+        os.path.join(ROOT, "tests", "test_oracle_snapkv_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_sampling_pins.py")]
 
 MUTANTS = {
     "tie_rule_reversed": ("return (a->j > b->j) - (a->j < b->j);",
@@ -41,6 +42,14 @@ MUTANTS = {
     "snapkv_pool_narrow": ("for (long u = t - h; u <= t + h; ++u)", "for (long u = t - h + 1; u <= t + h; ++u)"),
     "snapkv_ties_reversed": ("return (a->t > b->t) - (a->t < b->t);", "return (a->t < b->t) - (a->t > b->t);"),
     "snapkv_drops_window": ("out[kp + w] = P + w;", "out[kp + w] = P + w - 1;"),
+    # sampling recoveries (reading R14)
+    "philox_nine_rounds": ("for (int r = 0; r < 10; ++r) {", "for (int r = 0; r < 9; ++r) {"),
+    "philox_key_not_bumped": ("k[1] += 0xBB67AE85u;", "k[1] += 0u;"),
+    "gaussian_variance_as_sd": ("return mu + sqrt(var) * sqrt(-2.0 * log(u1)) * cos(2.0 * M_PI * u2);",
+                                "return mu + var * sqrt(-2.0 * log(u1)) * cos(2.0 * M_PI * u2);"),
+    "gaussian_angle_from_radius_draw": ("cos(2.0 * M_PI * u2)", "cos(2.0 * M_PI * u1)"),
+    "exponential_unit_mean": ("return -mu * log(u1);", "return -log(u1);"),
+    "sampled_key_not_back_solved": ("Kt[t * D + j] = (qj > 0.0) ? w / qj : 0.0;", "Kt[t * D + j] = w;"),
     "gqa_transposed": ("const float *qrow = q + (bh * G + g) * (long)D;",
                        "const float *qrow = q + ((long)g * BH + bh) * (long)D;"),
     "tail_keys_from_values": ("(double)k_tail[(bh * tail_cap + t) * D + j];",
