@@ -9,8 +9,8 @@ namespace spark {
 cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const spark_kcache &kc,
                          void *ws, cudaStream_t st);
 cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const void *k_tail,
-                          const void *v_tail, int tail_cap, int n_tail, int G, float *out, void *ws,
-                          const DecodeGeom &geo, cudaStream_t st);
+                          const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
+                          unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st);
 cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
                           int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st);
 
@@ -131,14 +131,11 @@ int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, cons
                       const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
                       unsigned long long seed, float *out, void *workspace, size_t ws_bytes,
                       void *stream) {
-    (void)seed;
     int rc = check_cache(kc);
     if (rc != SPARK_OK) return rc;
     if (G != 1 && G != 2 && G != 4 && G != 8) return G < 1 ? SPARK_ERR_ARG : SPARK_ERR_UNSUPPORTED;
-    if (recovery != SPARK_F_DEGENERATE) {
-        if (recovery == SPARK_F_GAUSSIAN || recovery == SPARK_F_EXPONENTIAL) return SPARK_ERR_UNSUPPORTED;
+    if (recovery != SPARK_F_DEGENERATE && recovery != SPARK_F_GAUSSIAN && recovery != SPARK_F_EXPONENTIAL)
         return SPARK_ERR_ARG;
-    }
     if (tail_cap < 0 || n_tail < 0 || n_tail > tail_cap) return SPARK_ERR_ARG;
     const long BH = (long)kc->B * kc->Hkv;
     if (BH == 0) return SPARK_OK;
@@ -151,8 +148,8 @@ int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, cons
     const DecodeGeom geo = decode_geometry(BH, kc->S, kc->T, es, G, num_sms());
     if (BH * (long)geo.units >= (1L << 31)) return SPARK_ERR_UNSUPPORTED;  // 32-bit item indices
     if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
-    cudaError_t e = launch_decode(q, *kc, v, k_tail, v_tail, tail_cap, n_tail, G, out, workspace, geo,
-                                  static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_decode(q, *kc, v, k_tail, v_tail, tail_cap, n_tail, G, recovery, seed, out, workspace,
+                                  geo, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 

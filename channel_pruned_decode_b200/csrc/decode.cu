@@ -62,11 +62,48 @@ struct DecArgs {
     int nstage;
     int nwarp;
     size_t warp_bytes;
+    unsigned long long seed;  // sampling recoveries only
 };
 
 // log2(e) / sqrt(128): folds the softmax scale and the exp -> exp2 change
 // into the query.
 constexpr float kQScale = 0.12751743074602467f;
+
+// ---- sampling recoveries (F table: Gaussian N(mu, sigma^2), Exponential
+// Exp(1/mu)).  One draw per pruned (token, channel) entry, fixed for a given
+// seed: Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) with counter
+// (t, j, bh low word, bh high word) and key (seed low word, seed high word);
+// uniforms from the top 24 bits of the first two output words.
+__device__ __forceinline__ void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c[0]), lo0 = 0xD2511F53u * c[0];
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c[2]), lo1 = 0xCD9E8D57u * c[2];
+        const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+        c[0] = n0;
+        c[1] = lo1;
+        c[2] = n2;
+        c[3] = lo0;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+}
+
+// sampled saliency score of pruned entry (bh, t, j); kF = 1 Gaussian, 2 Exponential
+template <int kF>
+__device__ __forceinline__ float sample_score(unsigned long long seed, long bh, long t, int j, float mu,
+                                              float sigma) {
+    uint32_t c[4] = {(uint32_t)t, (uint32_t)j, (uint32_t)((unsigned long long)bh & 0xffffffffu),
+                     (uint32_t)((unsigned long long)bh >> 32)};
+    philox4x32_10(c, (uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32));
+    const float u1 = (float)((c[0] >> 8) + 1u) * (1.0f / 16777216.0f);  // (0, 1], exact
+    if constexpr (kF == 2) {
+        return -mu * logf(u1);
+    } else {
+        const float u2 = (float)(c[1] >> 8) * (1.0f / 16777216.0f);    // [0, 1), exact
+        return mu + sigma * sqrtf(-2.0f * logf(u1)) * cospif(2.0f * u2);
+    }
+}
 
 // 4 consecutive channels of a key row (dense tail) as fp32
 template <typename E> struct Row4;
@@ -281,7 +318,7 @@ __device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, 
 // spilling warps on the G = 4 workloads
 __host__ __device__ constexpr int dec_max_warps(int G) { return G > 2 ? 12 : kMaxWarps; }
 
-template <typename E, int G>
+template <typename E, int G, int kF>
 __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -384,6 +421,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
     VRegs<E> vr;
     int tab_bh = -1;
     bool failed = false;
+    float f_mu = 0.f, f_sigma = 0.f;  // sampling recoveries: pruned-score mean, sd
 
     for (int item = gw; item < n_items && !failed; item += nwt) {
         const int bh = item_head(item);
@@ -398,6 +436,12 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         if (bh != tab_bh) {
             const E *q = static_cast<const E *>(a.q) + (size_t)bh * G * kD;
             const double mu = a.stats[bh * 4 + 3];
+            if constexpr (kF != SPARK_F_DEGENERATE) {
+                const double n = a.stats[bh * 4 + 0];
+                const double var = n > 0.0 ? a.stats[bh * 4 + 2] / n - mu * mu : 0.0;
+                f_mu = (float)mu;
+                f_sigma = (float)sqrt(var > 0.0 ? var : 0.0);
+            }
             float part[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) part[g] = 0.f;
@@ -405,13 +449,16 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             for (int i = 0; i < kD / 32; ++i) {
                 const int j = lane + 32 * i;
                 const float qnj = a.qn[bh * kD + j];
-                const float c = qnj > 0.f ? (float)(mu / (double)qnj) : 0.f;
+                // Degenerate: c_j = mu / qn_j (folded into Qc); sampling: 1 / qn_j
+                const float c = qnj > 0.f ? (kF == SPARK_F_DEGENERATE ? (float)(mu / (double)qnj)
+                                                                       : (float)(1.0 / (double)qnj))
+                                          : 0.f;
                 ws.tabc[j] = c;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     const float qq = Elem<E>::to_f(q[(size_t)g * kD + j]) * kQScale;
                     ws.tabq[j * G + g] = qq;
-                    part[g] = fmaf(qq, c, part[g]);
+                    if constexpr (kF == SPARK_F_DEGENERATE) part[g] = fmaf(qq, c, part[g]);
                 }
             }
 #pragma unroll
@@ -488,7 +535,28 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             float s[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) s[g] = 0.f;
-            if (a.T > 0) {
+            if constexpr (kF != SPARK_F_DEGENERATE) {
+                // every channel: kept -> stored value, pruned -> sampled score / qn_j
+                const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
+                const uint32_t wds[4] = {mw.x, mw.y, mw.z, mw.w};
+                const E *vp = ws.svals(st) + lane;
+                const long t_tok = t0 + lane;
+                int pos = 0;
+#pragma unroll 1
+                for (int j = 0; j < kD; ++j) {
+                    float x;
+                    if ((wds[j >> 5] >> (j & 31)) & 1u) {
+                        x = Elem<E>::to_f(vp[min(pos, a.T - 1) * kWT]);
+                        ++pos;
+                    } else {
+                        x = sample_score<kF>(a.seed, bh, t_tok, j, f_mu, f_sigma) * ws.tabc[j];
+                    }
+                    QVec<G> qv;
+                    qv.load(ws.tabq + j * G);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
+                }
+            } else if (a.T > 0) {
                 const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
                 uint32_t w1 = mw.y, w2 = mw.z, w3 = mw.w;
                 uint32_t cur = mw.x;
@@ -617,7 +685,7 @@ DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms) {
     return g;
 }
 
-template <typename E, int G>
+template <typename E, int G, int kF>
 static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, float *out, cudaStream_t st) {
     DecArgs a = a0;
     a.chunk = geo.chunk;
@@ -626,7 +694,7 @@ static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, flo
     a.nstage = geo.nstage;
     a.nwarp = geo.nwarp;
     a.warp_bytes = geo.warp_bytes;
-    auto kern = decode_kernel<E, G>;
+    auto kern = decode_kernel<E, G, kF>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)geo.smem);
     if (e != cudaSuccess) return e;
     kern<<<geo.ctas, geo.nwarp * 32, geo.smem, st>>>(a);
@@ -634,20 +702,31 @@ static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, flo
     return cudaGetLastError();
 }
 
-template <typename E>
+template <typename E, int kF>
 static cudaError_t dispatch_g(const DecArgs &a, const DecodeGeom &geo, int G, float *out, cudaStream_t st) {
     switch (G) {
-    case 1: return launch_decode_t<E, 1>(a, geo, out, st);
-    case 2: return launch_decode_t<E, 2>(a, geo, out, st);
-    case 4: return launch_decode_t<E, 4>(a, geo, out, st);
-    case 8: return launch_decode_t<E, 8>(a, geo, out, st);
+    case 1: return launch_decode_t<E, 1, kF>(a, geo, out, st);
+    case 2: return launch_decode_t<E, 2, kF>(a, geo, out, st);
+    case 4: return launch_decode_t<E, 4, kF>(a, geo, out, st);
+    case 8: return launch_decode_t<E, 8, kF>(a, geo, out, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename E>
+static cudaError_t dispatch_f(const DecArgs &a, const DecodeGeom &geo, int G, int recovery, float *out,
+                              cudaStream_t st) {
+    switch (recovery) {
+    case SPARK_F_DEGENERATE: return dispatch_g<E, SPARK_F_DEGENERATE>(a, geo, G, out, st);
+    case SPARK_F_GAUSSIAN: return dispatch_g<E, SPARK_F_GAUSSIAN>(a, geo, G, out, st);
+    case SPARK_F_EXPONENTIAL: return dispatch_g<E, SPARK_F_EXPONENTIAL>(a, geo, G, out, st);
     default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const void *k_tail,
-                          const void *v_tail, int tail_cap, int n_tail, int G, float *out, void *ws,
-                          const DecodeGeom &geo, cudaStream_t st) {
+                          const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
+                          unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st) {
     const long BH = (long)kc.B * kc.Hkv;
     if (BH == 0) return cudaSuccess;
     DecArgs a{};
@@ -668,8 +747,9 @@ cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, 
     a.T = kc.T;
     a.tail_cap = tail_cap;
     a.n_tail = n_tail;
-    if (kc.dtype == SPARK_BF16) return dispatch_g<__nv_bfloat16>(a, geo, G, out, st);
-    return dispatch_g<float>(a, geo, G, out, st);
+    a.seed = seed;
+    if (kc.dtype == SPARK_BF16) return dispatch_f<__nv_bfloat16>(a, geo, G, recovery, out, st);
+    return dispatch_f<float>(a, geo, G, recovery, out, st);
 }
 
 }  // namespace spark

@@ -61,8 +61,8 @@ typedef enum { SPARK_F32 = 0, SPARK_BF16 = 1 } spark_dtype;
 /* Recovery function F of [W] 3.3 (F table). */
 typedef enum {
     SPARK_F_DEGENERATE = 0,   /* w~ = mu_pruned                              */
-    SPARK_F_GAUSSIAN = 1,     /* w~ ~ N(mu, sigma^2)   (not built: UNSUPPORTED) */
-    SPARK_F_EXPONENTIAL = 2   /* w~ ~ Exp(1/mu)        (not built: UNSUPPORTED) */
+    SPARK_F_GAUSSIAN = 1,     /* w~ ~ N(mu, sigma^2), sigma over the pruned set */
+    SPARK_F_EXPONENTIAL = 2   /* w~ ~ Exp(1/mu) (mean mu)                     */
 } spark_recovery;
 
 typedef enum { SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1, SPARK_OP_SNAPKV = 2 } spark_op;
@@ -179,8 +179,15 @@ SPARK_API int spark_prune_noalloc(const void *k, const void *q_obs, int G, int W
  * rebuilt by F (Degenerate: k~_j = mu_pruned / qn_j, 0 when qn_j == 0),
  * then out = softmax(q . K~^T / sqrt(D)) V over prefix + tail, a split-K
  * (flash-decoding) pass followed by a log-sum-exp combine.  An empty
- * context (S + n_tail == 0) gives zeros.  `seed` is reserved for the
- * sampling recoveries.  Requires the decode workspace size for tail_cap.
+ * context (S + n_tail == 0) gives zeros.  Gaussian / Exponential F draw one
+ * score per pruned (token, channel) entry from Philox4x32-10 (Salmon et al.,
+ * SC'11) with counter (t, j, bh low, bh high) and key (seed low, seed high),
+ * where bh = b*Hkv + h; uniforms u1 = ((x0 >> 8) + 1) / 2^24,
+ * u2 = (x1 >> 8) / 2^24; Gaussian = mu + sigma sqrt(-2 ln u1) cos(2 pi u2)
+ * (mu, sigma: mean and population sd of the head's pruned saliencies),
+ * Exponential = -mu ln u1; the key is then w~ / qn_j.  The same seed gives
+ * the same draws at every step.  Degenerate ignores `seed`.  Requires the
+ * decode workspace size for tail_cap.
  */
 SPARK_API int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v,
                       const void *k_tail, const void *v_tail, int tail_cap,

@@ -119,7 +119,9 @@ def test_decode_rejects_bad_args(L):
         k.get("ws", 256), 1 << 20, None)
     assert call(G=3) == B.SPARK_ERR_UNSUPPORTED
     assert call(G=0) == B.SPARK_ERR_ARG
-    assert call(rec=B.SPARK_F_GAUSSIAN) == B.SPARK_ERR_UNSUPPORTED
+    # (every call here must fail validation: the pointers are not real)
+    assert call(rec=B.SPARK_F_GAUSSIAN, ws=None) == B.SPARK_ERR_WORKSPACE
+    assert call(rec=B.SPARK_F_EXPONENTIAL, G=3) == B.SPARK_ERR_UNSUPPORTED
     assert call(rec=9) == B.SPARK_ERR_ARG
     assert call(n=9) == B.SPARK_ERR_ARG          # n_tail > tail_cap
     assert call(cap=-1) == B.SPARK_ERR_ARG
@@ -147,3 +149,17 @@ def test_status_strings(L):
 def test_empty_batch_is_a_no_op(L):
     kc = _kc(B=0)
     assert L.spark_prune(None, None, 4, 32, ctypes.byref(kc), None, 0, None) == B.SPARK_OK
+
+
+def test_snapkv_rejects_bad_args(L):
+    f = lambda **k: L.spark_snapkv_evict(16, 16, 16, 1, 2, k.get("S", 256), k.get("D", 128), k.get("G", 4),
+                                         k.get("W", 32), k.get("keep", 64), k.get("pool", 7),
+                                         k.get("dt", B.SPARK_BF16), 16, 16, 16, k.get("ws", None), 1 << 20, None)
+    assert f(D=64) == B.SPARK_ERR_UNSUPPORTED
+    assert f(dt=B.SPARK_F32) == B.SPARK_ERR_UNSUPPORTED
+    assert f(G=3, W=5) == B.SPARK_ERR_UNSUPPORTED     # G*W not a multiple of 16
+    assert f(G=8, W=32) == B.SPARK_ERR_UNSUPPORTED    # G*W > 128
+    assert f(keep=16) == B.SPARK_ERR_ARG              # keep < W
+    assert f(keep=300) == B.SPARK_ERR_ARG             # keep > S
+    assert f(pool=6) == B.SPARK_ERR_ARG               # even pool
+    assert f() == B.SPARK_ERR_WORKSPACE               # no workspace

@@ -226,3 +226,59 @@ def test_long_context_32_layers():
     # popcount == T
     wl = WORKLOADS["long"]
     _multi_step(wl, check_steps={0}, sample_bh=[0, 37, 130, 255])
+
+
+# ------------------------------------------ sampling recoveries (F table)
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("dtype,S,T,G,n_tail", [(torch.bfloat16, 1000, 26, 4, 3), (torch.float32, 257, 64, 2, 0),
+                                                (torch.bfloat16, 64, 0, 4, 1), (torch.bfloat16, 300, 127, 8, 0)])
+def test_sampling_recovery_parity(mode, dtype, S, T, G, n_tail):
+    wl = scaled(WORKLOADS["tiny"], S=S, G=G, dtype="f32" if dtype == torch.float32 else "bf16", Hkv=3,
+                seed=101 + S + T + mode)
+    pre = make_prefill(wl, DEV)
+    kc = run_prune(pre["k"], pre["q_obs"], G, wl.W, T)
+    torch.cuda.synchronize()
+    BH = wl.rows * wl.Hkv
+    qn, m, vals, st = _check_prune(kc, to_np(pre["k"]), to_np(pre["q_obs"]), G, T, "sampling")
+    cap = max(n_tail, 4)
+    kt = torch.zeros((wl.rows, wl.Hkv, cap, D), dtype=dtype, device=DEV)
+    vt = torch.zeros_like(kt)
+    for i in range(n_tail):
+        stp = make_decode_step(wl, i, DEV)
+        spark_tail_append(stp["k_new"], stp["v_new"], kt, vt, wl.rows, wl.Hkv, D, cap, i)
+    q = make_decode_step(wl, 7, DEV)["q"]
+    seed = 0x1234_5678_9ABC
+    out = torch.empty((wl.rows, wl.Hq, D), dtype=torch.float32, device=DEV)
+    ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, G, S, D, T, cap))
+    spark_decode_attn(q, kc, pre["v"], kt, vt, cap, n_tail, G, out, ws, recovery=mode, seed=seed)
+    torch.cuda.synchronize()
+    assert spark_device_status(ws) == 0
+    o_ref = oracle.decode_f(to_np(q).reshape(BH * G, D), m, vals, qn, st, to_np(pre["v"]).reshape(BH, S, D),
+                            to_np(kt).reshape(BH, cap, D), to_np(vt).reshape(BH, cap, D), n_tail, G,
+                            mode=mode, seed=seed)
+    assert_out_close(out.cpu().numpy().reshape(BH * G, D), o_ref, f"F={mode} S={S} T={T}")
+    # the draw depends on the seed: another seed changes the output
+    out2 = torch.empty_like(out)
+    spark_decode_attn(q, kc, pre["v"], kt, vt, cap, n_tail, G, out2, ws, recovery=mode, seed=seed + 1)
+    torch.cuda.synchronize()
+    if T < D:
+        assert not torch.equal(out, out2)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_sampling_recovery_llama_layer(mode):
+    wl = scaled(WORKLOADS["llama1l"], S=8192)
+    T = spark_lambda_to_T(wl.lam)
+    pre = make_prefill(wl, DEV)
+    kc = run_prune(pre["k"], pre["q_obs"], wl.G, wl.W, T)
+    BH, S, G = wl.BH, wl.S, wl.G
+    q = make_decode_step(wl, 0, DEV)["q"]
+    out = torch.empty((wl.rows, wl.Hq, D), dtype=torch.float32, device=DEV)
+    ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, G, S, D, T, 0))
+    spark_decode_attn(q, kc, pre["v"], None, None, 0, 0, G, out, ws, recovery=mode, seed=42)
+    torch.cuda.synchronize()
+    qn = oracle.qnorm(to_np(pre["q_obs"]).reshape(BH * G, -1, D), G)
+    m, vals, st = oracle.prune(to_np(pre["k"]).reshape(BH, S, D), qn, T)
+    o_ref = oracle.decode_f(to_np(q).reshape(BH * G, D), m, vals, qn, st, to_np(pre["v"]).reshape(BH, S, D),
+                            G=G, mode=mode, seed=42)
+    assert_out_close(out.cpu().numpy().reshape(BH * G, D), o_ref, f"llama layer F={mode}")
