@@ -557,24 +557,36 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }
             } else if (a.T > 0) {
+                // Walk the T set bits from the top channel down (one find-leading-
+                // one per bit); the packed values are in ascending channel order,
+                // so they are read from the last one backwards.  Empty words are
+                // skipped by a short branch taken at most 3 times per token.
                 const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
-                uint32_t w1 = mw.y, w2 = mw.z, w3 = mw.w;
-                uint32_t cur = mw.x;
-                int wi = 0;
-                const E *vp = ws.svals(st) + lane;
+                const uint32_t w0 = mw.x, w1 = mw.y, w2 = mw.z;
+                uint32_t cur = mw.w;
+                int wi = 3;
+                const float *qrow = ws.tabq + 3 * 32 * G;  // q' rows of the current word
+                const float *crow = ws.tabc + 3 * 32;      // c of the current word
+                const E *vp = ws.svals(st) + lane + (a.T - 1) * kWT;
 #pragma unroll 2
-                for (int i = 0; i < a.T; ++i) {
-                    while (cur == 0u && wi < 3) {
-                        ++wi;
-                        cur = (wi == 1) ? w1 : ((wi == 2) ? w2 : w3);
+                for (int i = a.T; i > 0; --i) {
+                    if (cur == 0u && wi > 0) {
+                        // a mask with fewer than T bits (a cache never written by
+                        // spark_prune, or a lane past n) stops at word 0 and keeps
+                        // indexing in bounds
+                        do {
+                            --wi;
+                            cur = (wi == 2) ? w2 : ((wi == 1) ? w1 : w0);
+                        } while (cur == 0u && wi > 0);
+                        qrow = ws.tabq + wi * 32 * G;
+                        crow = ws.tabc + wi * 32;
                     }
-                    // a mask with fewer than T bits (a cache never written by
-                    // spark_prune, or a lane past n) still indexes in bounds
-                    const int j = (32 * wi + __ffs(cur) - 1) & (kD - 1);
-                    cur &= cur - 1u;
-                    const float x = Elem<E>::to_f(vp[i * kWT]) - ws.tabc[j];
+                    const int b = (31 - __clz(cur)) & 31;
+                    cur ^= 1u << b;
+                    const float x = Elem<E>::to_f(*vp) - crow[b];
+                    vp -= kWT;
                     QVec<G> qv;
-                    qv.load(ws.tabq + j * G);
+                    qv.load(qrow + b * G);
 #pragma unroll
                     for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }

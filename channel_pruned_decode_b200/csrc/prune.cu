@@ -117,7 +117,7 @@ __device__ __forceinline__ int quad_sum(int v) {
 // packed compare + add (one instruction each per two channels) count them.
 // `mid` is 0 or >= 0x400 (a normal fp16 pattern); keys below 0x400 sit below
 // every probe.  Counts <= 32 per lane are exact in fp16.
-__device__ __forceinline__ int quad_count16(const uint32_t (&kp)[16], uint32_t mid) {
+__device__ __forceinline__ __half quad_count16(const uint32_t (&kp)[16], uint32_t mid) {
     const uint32_t mm = mid * 0x10001u;
     const __half2 m2 = *reinterpret_cast<const __half2 *>(&mm);
     const __half2 z = __float2half2_rn(0.f);
@@ -130,8 +130,11 @@ __device__ __forceinline__ int quad_count16(const uint32_t (&kp)[16], uint32_t m
         a3 = __hadd2(a3, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 3]), m2));
     }
     a0 = __hadd2(__hadd2(a0, a1), __hadd2(a2, a3));
-    const int c = (int)(__low2float(a0) + __high2float(a0));
-    return quad_sum(c);
+    // both halves -> one count (<= 32, exact), then the quad's sum (<= 128, exact)
+    __half c = __hadd(__low2half(a0), __high2half(a0));
+    c = __hadd(c, __shfl_xor_sync(0xffffffffu, c, 1));
+    c = __hadd(c, __shfl_xor_sync(0xffffffffu, c, 2));
+    return c;
 }
 
 __device__ __forceinline__ int quad_count32(const uint32_t (&key)[32], uint32_t mid) {
@@ -156,39 +159,38 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     if (T <= 0) return 0u;
     if (T >= kD) return 0xffffffffu;
 
-    // ---- phase 1: 16-bit keys.  count(>= lo) >= T > count(>= hi)
+    // ---- phase 1: 16-bit keys.  count(>= lo) >= T > count(>= hi).
+    // Probes: the previous token's threshold, then galloping away from an
+    // open side of the bracket (step doubling), then bisection.  The bracket
+    // update is written with selects so that quads in different states of
+    // the search do not diverge.
     constexpr uint32_t kTop = 0x7c00u;  // above the clamp: nothing reaches it
+    const __half hT = __int2half_rn(T);
     uint32_t lo = 0u, hi = kTop;
-    int c_hi = 0;
+    __half c_hi_h = __int2half_rn(0);
     bool exact = false;
     bool done = false;
     uint32_t step = 64u;
     uint32_t mid = min(max(tau16, 1u), kTop - 1u);
     while (__any_sync(0xffffffffu, !done)) {
         const uint32_t probe = (mid > 0u && mid < 0x400u) ? 0x400u : mid;
-        const int c = quad_count16(kp, probe);
-        if (!done) {
-            if (c >= T) {
-                lo = mid;
-                if (c == T) { exact = true; done = true; }
-            } else {
-                hi = mid;
-                c_hi = c;
-            }
-            if (hi - lo <= 1u) done = true;
-            // next probe: gallop away from an unknown side, else bisect
-            if (hi == kTop) {
-                mid = min(lo + step, kTop - 1u);
-                step <<= 1;
-            } else if (lo == 0u) {
-                mid = hi > step ? hi - step : hi >> 1;
-                mid = max(mid, 1u);
-                step <<= 1;
-            } else {
-                mid = lo + ((hi - lo) >> 1);
-            }
-        }
+        const __half c = quad_count16(kp, probe);
+        const bool ge = __hge(c, hT);
+        const bool eq = __heq(c, hT);
+        const bool act = !done;
+        lo = (act && ge) ? mid : lo;
+        hi = (act && !ge) ? mid : hi;
+        c_hi_h = (act && !ge) ? c : c_hi_h;
+        exact = exact || (act && eq);
+        done = done || eq || (hi - lo <= 1u);
+        const bool up = (hi == kTop), down = (lo == 0u);
+        const uint32_t gal_up = min(lo + step, kTop - 1u);
+        const uint32_t gal_dn = max(hi > step ? hi - step : hi >> 1, 1u);
+        const uint32_t bis = lo + ((hi - lo) >> 1);
+        mid = up ? gal_up : (down ? gal_dn : bis);
+        step = (up || down) ? step << 1 : step;
     }
+    int c_hi = __half2int_rn(c_hi_h);
     tau16 = lo;
 
     // ---- phase 2: exact keys inside the band of 16-bit key == lo.  Quads
