@@ -184,14 +184,17 @@ template <int G> struct QVec {
     }
 };
 
-// Per-warp shared memory: tables, p buffer, mbarriers, then the stage ring.
+// Per-warp shared memory: tables, p buffers, mbarriers, then the stage ring.
 template <typename E, int G>
 struct WarpSmem {
+    unsigned char *vt;  // bf16 values: swizzled V tile [kWT][kD]
+    float *pT;     // [G][kWT] p of the tile, head-major (tensor-core P.V)
     float *tabq;   // [kD][G]   q' per channel
-    float *tabc;   // [kD]      c_j = mu / qn_j
-    float *pdup;   // [kWT][G][2] p duplicated into fp32 pairs
+    float *tabc;   // [kD]      c_j = mu / qn_j (1 / qn_j for sampling F)
+    float *pdup;   // [kWT][G][2] p duplicated into fp32 pairs (CUDA-core P.V)
     float *qc;     // [G] Qc = sum_j q'_j c_j of the current head
     uint64_t *bars;
+    uint8_t *lst;  // [T][kWT] kept channel indices of the tile's tokens
     unsigned char *stages;
     uint32_t stage_bytes;
     __device__ __forceinline__ const uint32_t *smask(int st) const {
@@ -202,30 +205,29 @@ struct WarpSmem {
     }
 };
 
-// flash-decoding state of one warp for the item in progress
+// online-softmax state of one warp for the item in progress
 template <int G>
 struct Flash {
-    float m[G];       // running max (log2 domain), warp-uniform
-    float l[G];       // this lane's share of the running sum
-    float2 acc[G][2]; // this lane's 4 value channels, as fp32 pairs
+    float m[G];  // running max (log2 domain), warp-uniform
+    float l[G];  // this lane's share of the running sum
     __device__ __forceinline__ void reset() {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             m[g] = -INFINITY;
             l[g] = 0.f;
-            acc[g][0] = make_float2(0.f, 0.f);
-            acc[g][1] = make_float2(0.f, 0.f);
         }
     }
 };
 
 // Online-softmax update for one tile: s[] is this lane's token score (-inf
-// for lanes past the tile end).  Leaves p (duplicated pairs) in shared
-// memory and rescales the accumulators when the running max moved.
+// for lanes past the tile end).  Leaves p in shared memory in the layout the
+// P.V engine reads and returns the factor each head's accumulator is scaled
+// by (all 1 when no running max moved).
 template <typename E, int G>
-__device__ __forceinline__ void tile_softmax(const WarpSmem<E, G> &ws, Flash<G> &f, const float (&s)[G]) {
+__device__ __forceinline__ bool tile_softmax(const WarpSmem<E, G> &ws, Flash<G> &f, const float (&s)[G],
+                                             float (&alpha)[G]) {
     const int lane = threadIdx.x & 31;
-    float alpha[G], p[G];
+    float p[G];
     bool rescale = false;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -237,72 +239,211 @@ __device__ __forceinline__ void tile_softmax(const WarpSmem<E, G> &ws, Flash<G> 
         p[g] = (m_new == -INFINITY) ? 0.f : exp2f(s[g] - m_new);
         f.l[g] = fmaf(f.l[g], alpha[g], p[g]);
     }
-    float *pd = ws.pdup + lane * G * 2;
-    if constexpr (G == 1) {
-        *reinterpret_cast<float2 *>(pd) = make_float2(p[0], p[0]);
+    if constexpr (sizeof(E) == 2) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) ws.pT[g * kWT + lane] = p[g];
     } else {
+        float *pd = ws.pdup + lane * G * 2;
+        if constexpr (G == 1) {
+            *reinterpret_cast<float2 *>(pd) = make_float2(p[0], p[0]);
+        } else {
 #pragma unroll
-        for (int g = 0; g < G; g += 2)
-            *reinterpret_cast<float4 *>(pd + 2 * g) = make_float4(p[g], p[g], p[g + 1], p[g + 1]);
-    }
-    if (rescale) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float2 a2 = make_float2(alpha[g], alpha[g]);
-            f.acc[g][0] = __fmul2_rn(f.acc[g][0], a2);
-            f.acc[g][1] = __fmul2_rn(f.acc[g][1], a2);
+            for (int g = 0; g < G; g += 2)
+                *reinterpret_cast<float4 *>(pd + 2 * g) = make_float4(p[g], p[g], p[g + 1], p[g + 1]);
         }
     }
     __syncwarp();
+    return rescale;
 }
 
-// P.V over tokens [t_lo, t_lo + VRegs::kTok) of the tile (those < n), V rows
-// from registers, p from shared memory.
-template <typename E, int G, bool kFull>
-__device__ __forceinline__ void tile_pv_impl(const WarpSmem<E, G> &ws, Flash<G> &f, const VRegs<E> &vr,
-                                             int t_lo, int n) {
+// P.V accumulator of one warp.  fp32 values: CUDA cores, V rows streamed into
+// registers; bf16 values: tensor cores (below).
+template <typename E, int G> struct PV;
+
+template <int G> struct PV<float, G> {
+    float2 acc[G][2];  // this lane's 4 value channels, as fp32 pairs
+    VRegs<float> vr;
+    __device__ __forceinline__ void reset() {
 #pragma unroll
-    for (int t = 0; t < VRegs<E>::kTok; ++t) {
-        if (kFull || t_lo + t < n) {
-            float2 x01, x23;
-            vr.get(t, x01, x23);
-            const float *pd = ws.pdup + (t_lo + t) * G * 2;
-            if constexpr (G == 1) {
-                const float2 pp = *reinterpret_cast<const float2 *>(pd);
-                f.acc[0][0] = __ffma2_rn(pp, x01, f.acc[0][0]);
-                f.acc[0][1] = __ffma2_rn(pp, x23, f.acc[0][1]);
-            } else {
+        for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = make_float2(0.f, 0.f);
+    }
+    // row0: channel 0 of the tile's first value row (global memory)
+    __device__ __forceinline__ void begin(const WarpSmem<float, G> &, const float *row0, int n) {
+        vr.load(row0 + 4 * (threadIdx.x & 31), n);
+    }
+    __device__ __forceinline__ void rescale(const float (&alpha)[G]) {
 #pragma unroll
-                for (int g = 0; g < G; g += 2) {
-                    const float4 pp = *reinterpret_cast<const float4 *>(pd + 2 * g);
-                    const float2 pa = make_float2(pp.x, pp.y), pb = make_float2(pp.z, pp.w);
-                    f.acc[g][0] = __ffma2_rn(pa, x01, f.acc[g][0]);
-                    f.acc[g][1] = __ffma2_rn(pa, x23, f.acc[g][1]);
-                    f.acc[g + 1][0] = __ffma2_rn(pb, x01, f.acc[g + 1][0]);
-                    f.acc[g + 1][1] = __ffma2_rn(pb, x23, f.acc[g + 1][1]);
+        for (int g = 0; g < G; ++g) {
+            const float2 a2 = make_float2(alpha[g], alpha[g]);
+            acc[g][0] = __fmul2_rn(acc[g][0], a2);
+            acc[g][1] = __fmul2_rn(acc[g][1], a2);
+        }
+    }
+    __device__ __forceinline__ void accumulate(const WarpSmem<float, G> &ws, const float *row0, int n) {
+        const int lane = threadIdx.x & 31;
+        for (int tb = 0; tb < n; tb += VRegs<float>::kTok) {
+            if (tb > 0) vr.load(row0 + (size_t)tb * kD + 4 * lane, n - tb);
+#pragma unroll
+            for (int t = 0; t < VRegs<float>::kTok; ++t) {
+                if (tb + t < n) {
+                    float2 x01, x23;
+                    vr.get(t, x01, x23);
+                    const float *pd = ws.pdup + (tb + t) * G * 2;
+                    if constexpr (G == 1) {
+                        const float2 pp = *reinterpret_cast<const float2 *>(pd);
+                        acc[0][0] = __ffma2_rn(pp, x01, acc[0][0]);
+                        acc[0][1] = __ffma2_rn(pp, x23, acc[0][1]);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < G; g += 2) {
+                            const float4 pp = *reinterpret_cast<const float4 *>(pd + 2 * g);
+                            const float2 pa = make_float2(pp.x, pp.y), pb = make_float2(pp.z, pp.w);
+                            acc[g][0] = __ffma2_rn(pa, x01, acc[g][0]);
+                            acc[g][1] = __ffma2_rn(pa, x23, acc[g][1]);
+                            acc[g + 1][0] = __ffma2_rn(pb, x01, acc[g + 1][0]);
+                            acc[g + 1][1] = __ffma2_rn(pb, x23, acc[g + 1][1]);
+                        }
+                    }
                 }
             }
         }
+        __syncwarp();  // p buffer free
     }
+    __device__ __forceinline__ void store(float *acc_out) const {  // acc_out: [G][kD] of this item
+        const int lane = threadIdx.x & 31;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            *reinterpret_cast<float4 *>(acc_out + g * kD + 4 * lane) =
+                make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+    }
+};
+
+// byte offset of 16-byte chunk c of row t in the swizzled V tile: chunks are
+// XOR-ed with the row's low 3 bits so that ldmatrix over 8 rows is free of
+// bank conflicts
+__device__ __forceinline__ uint32_t vswz(int t, int c) { return (uint32_t)(t * 256 + ((c ^ (t & 7)) << 4)); }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    const int n = valid ? 16 : 0;  // zero-fill rows past the tile end
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
 
-template <typename E, int G>
-__device__ __forceinline__ void tile_pv(const WarpSmem<E, G> &ws, Flash<G> &f, const VRegs<E> &vr, int t_lo,
-                                        int n) {
-    if (t_lo + VRegs<E>::kTok <= n) tile_pv_impl<E, G, true>(ws, f, vr, t_lo, n);
-    else tile_pv_impl<E, G, false>(ws, f, vr, t_lo, n);
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+
+// bf16 values: out^T[d][g] += V^T[d][t] P^T[t][g] on tensor cores
+// (mma.sync m16n8k16, fp32 accumulate): A = V^T read by ldmatrix.trans from
+// the swizzled V tile, B = P^T from the head-major p buffer, split into a bf16
+// high part and a bf16 remainder (two MMAs) so that p keeps ~16 bits.  The
+// accumulator fragment holds channel d = 16*mt + lane/4 (+8) and heads
+// 2*(lane%4) (+1); heads >= G are padding.
+template <int G> struct PV<__nv_bfloat16, G> {
+    static_assert(G <= 8, "the MMA n-dimension holds up to 8 heads");
+    float c[8][4];
+    __device__ __forceinline__ void reset() {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[mt][e] = 0.f;
+    }
+    // copy the tile's V rows (channel 0 of row 0 at row0) into the V tile
+    __device__ __forceinline__ void begin(const WarpSmem<__nv_bfloat16, G> &ws, const __nv_bfloat16 *row0,
+                                          int n) {
+        const int lane = threadIdx.x & 31;
+        const int ch = lane & 15, half = lane >> 4;
+        const uint32_t base = smem_u32(ws.vt);
+#pragma unroll
+        for (int i = 0; i < kWT / 2; ++i) {
+            const int t = half + 2 * i;
+            cp_async16(base + vswz(t, ch), row0 + (size_t)min(t, max(n - 1, 0)) * kD + 8 * ch, t < n);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    __device__ __forceinline__ void rescale(const float (&alpha)[G]) {
+        const int lane = threadIdx.x & 31;
+        const int h0 = 2 * (lane & 3), h1 = h0 + 1;
+        float a0 = 1.f, a1 = 1.f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            a0 = (h0 == g) ? alpha[g] : a0;
+            a1 = (h1 == g) ? alpha[g] : a1;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            c[mt][0] *= a0;
+            c[mt][1] *= a1;
+            c[mt][2] *= a0;
+            c[mt][3] *= a1;
+        }
+    }
+    __device__ __forceinline__ void accumulate(const WarpSmem<__nv_bfloat16, G> &ws, const __nv_bfloat16 *,
+                                               int) {
+        const int lane = threadIdx.x & 31;
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncwarp();
+        const int head = lane >> 2, tq = 2 * (lane & 3);
+        const uint32_t vbase = smem_u32(ws.vt);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            // B fragments: p of head `head` at tokens 16ks + tq (+1) and +8 (+9)
+            uint32_t bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;
+            if (head < G) {
+                const float2 p01 = *reinterpret_cast<const float2 *>(ws.pT + head * kWT + 16 * ks + tq);
+                const float2 p89 = *reinterpret_cast<const float2 *>(ws.pT + head * kWT + 16 * ks + tq + 8);
+                const __nv_bfloat162 h01 = __floats2bfloat162_rn(p01.x, p01.y);
+                const __nv_bfloat162 h89 = __floats2bfloat162_rn(p89.x, p89.y);
+                const __nv_bfloat162 r01 = __floats2bfloat162_rn(p01.x - __low2float(h01), p01.y - __high2float(h01));
+                const __nv_bfloat162 r89 = __floats2bfloat162_rn(p89.x - __low2float(h89), p89.y - __high2float(h89));
+                bh0 = *reinterpret_cast<const uint32_t *>(&h01);
+                bh1 = *reinterpret_cast<const uint32_t *>(&h89);
+                bl0 = *reinterpret_cast<const uint32_t *>(&r01);
+                bl1 = *reinterpret_cast<const uint32_t *>(&r89);
+            }
+            const int t = 16 * ks + (lane & 7) + ((lane >> 4) & 1) * 8;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                uint32_t a[4];
+                const int ch = 2 * mt + ((lane >> 3) & 1);
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                             : "r"(vbase + vswz(t, ch)));
+                mma_bf16_16816(c[mt], a, bh0, bh1);
+                mma_bf16_16816(c[mt], a, bl0, bl1);
+            }
+        }
+        __syncwarp();  // V tile and p buffer free
+    }
+    __device__ __forceinline__ void store(float *acc_out) const {  // acc_out: [G][kD] of this item
+        const int lane = threadIdx.x & 31;
+        const int d0 = lane >> 2, h0 = 2 * (lane & 3), h1 = h0 + 1;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            if (h0 < G) {
+                acc_out[h0 * kD + 16 * mt + d0] = c[mt][0];
+                acc_out[h0 * kD + 16 * mt + d0 + 8] = c[mt][2];
+            }
+            if (h1 < G) {
+                acc_out[h1 * kD + 16 * mt + d0] = c[mt][1];
+                acc_out[h1 * kD + 16 * mt + d0 + 8] = c[mt][3];
+            }
+        }
+    }
+};
 
 // Write one item's partial state (acc[G][D], m, l) to the workspace.
-template <int G>
-__device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, Flash<G> &f) {
+template <typename E, int G>
+__device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, const Flash<G> &f,
+                                              const PV<E, G> &pv) {
     const int lane = threadIdx.x & 31;
     const size_t row = (size_t)bh * a.units + u;
-    float *acc = a.acc + row * G * kD;
+    pv.store(a.acc + row * G * kD);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        *reinterpret_cast<float4 *>(acc + g * kD + 4 * lane) =
-            make_float4(f.acc[g][0].x, f.acc[g][0].y, f.acc[g][1].x, f.acc[g][1].y);
         float l = f.l[g];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -324,17 +465,19 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= a.nwarp) return;
     const int es = (int)sizeof(E);
-    constexpr int kVB = VRegs<E>::kTok;
 
     WarpSmem<E, G> ws;
     {
         unsigned char *base = smem_raw + (size_t)warp * a.warp_bytes;
-        ws.tabq = reinterpret_cast<float *>(base);
+        ws.vt = base;  // 8 KB for bf16 values, empty for fp32
+        ws.pT = reinterpret_cast<float *>(base + dec_vtile_bytes(es));
+        ws.tabq = ws.pT + G * kWT;
         ws.tabc = ws.tabq + kD * G;
         ws.pdup = ws.tabc + kD;
         ws.qc = ws.pdup + kWT * G * 2;
         ws.bars = reinterpret_cast<uint64_t *>(ws.qc + 16);
-        ws.stages = base + dec_table_bytes(G);
+        ws.lst = reinterpret_cast<uint8_t *>(ws.bars + kMaxStagesW);
+        ws.stages = base + dec_table_bytes(G, a.T, es);
         ws.stage_bytes = (uint32_t)dec_stage_bytes(a.T, es);
     }
     if (lane == 0) {
@@ -418,7 +561,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
     }
 
     Flash<G> f;
-    VRegs<E> vr;
+    PV<E, G> pv;
     int tab_bh = -1;
     bool failed = false;
     float f_mu = 0.f, f_sigma = 0.f;  // sampling recoveries: pruned-score mean, sd
@@ -429,7 +572,8 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         const bool tail = (u == a.n_pre);
         if (tail && a.n_tail == 0) {
             f.reset();
-            write_partial<G>(a, bh, u, f);
+            pv.reset();
+            write_partial<E, G>(a, bh, u, f, pv);
             continue;
         }
         // ---- tables of this head: q' (scaled query), c_j = mu / qn_j, Qc
@@ -471,6 +615,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             __syncwarp();
         }
         f.reset();
+        pv.reset();
 
         if (tail) {
             // ---- dense tail: keys and values read from global memory
@@ -478,7 +623,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             const E *vt = static_cast<const E *>(a.v_tail) + (size_t)bh * a.tail_cap * kD;
             for (int t0 = 0; t0 < a.n_tail; t0 += kWT) {
                 const int n = min(kWT, a.n_tail - t0);
-                vr.load(vt + (size_t)t0 * kD + 4 * lane, n);
+                pv.begin(ws, vt + (size_t)t0 * kD, n);
                 float s[G];
 #pragma unroll
                 for (int g = 0; g < G; ++g) s[g] = 0.f;
@@ -499,14 +644,11 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 }
 #pragma unroll
                 for (int g = 0; g < G; ++g) s[g] = (lane < n) ? s[g] : -INFINITY;
-                tile_softmax<E, G>(ws, f, s);
-                for (int tb = 0; tb < n; tb += kVB) {
-                    if (tb > 0) vr.load(vt + (size_t)(t0 + tb) * kD + 4 * lane, n - tb);
-                    tile_pv<E, G>(ws, f, vr, tb, n);
-                }
-                __syncwarp();
+                float alpha[G];
+                if (tile_softmax<E, G>(ws, f, s, alpha)) pv.rescale(alpha);
+                pv.accumulate(ws, vt + (size_t)t0 * kD, n);
             }
-            write_partial<G>(a, bh, u, f);
+            write_partial<E, G>(a, bh, u, f, pv);
             continue;
         }
 
@@ -514,12 +656,13 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         const int ntiles = item_tiles(u);
         const long t_item = (long)u * a.chunk;
         const long t_end = min((long)a.S, t_item + a.chunk);
-        const E *vbase = gv + (size_t)bh * a.S * kD + 4 * lane;
+        const E *vbase = gv + (size_t)bh * a.S * kD;
         for (int tile = 0; tile < ntiles; ++tile) {
             const long t0 = t_item + (long)tile * kWT;
             const int n = (int)min((long)kWT, t_end - t0);
-            // this tile's first V rows go to registers under the q.k~ below
-            vr.load(vbase + (size_t)t0 * kD, n);
+            // this tile's V rows start moving (registers or shared memory) under
+            // the q.k~ below
+            pv.begin(ws, vbase + (size_t)t0 * kD, n);
 
             const int st = (int)(consumed % a.nstage);
             const uint32_t par = (uint32_t)((consumed / a.nstage) & 1);
@@ -557,36 +700,28 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }
             } else if (a.T > 0) {
-                // Walk the T set bits from the top channel down (one find-leading-
-                // one per bit); the packed values are in ascending channel order,
-                // so they are read from the last one backwards.  Empty words are
-                // skipped by a short branch taken at most 3 times per token.
+                // Walk the T set bits of the 128-bit mask in ascending order with
+                // no branch: the mask is two 64-bit halves, a select picks the
+                // lower non-empty one, and clearing its lowest bit is 64-bit
+                // arithmetic.  All lanes run exactly T iterations; the i-th set
+                // bit pairs with the i-th packed value.  A mask with fewer than T
+                // bits (a cache never written by spark_prune, or a lane past n)
+                // keeps every index in range.
                 const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
-                const uint32_t w0 = mw.x, w1 = mw.y, w2 = mw.z;
-                uint32_t cur = mw.w;
-                int wi = 3;
-                const float *qrow = ws.tabq + 3 * 32 * G;  // q' rows of the current word
-                const float *crow = ws.tabc + 3 * 32;      // c of the current word
-                const E *vp = ws.svals(st) + lane + (a.T - 1) * kWT;
-#pragma unroll 2
-                for (int i = a.T; i > 0; --i) {
-                    if (cur == 0u && wi > 0) {
-                        // a mask with fewer than T bits (a cache never written by
-                        // spark_prune, or a lane past n) stops at word 0 and keeps
-                        // indexing in bounds
-                        do {
-                            --wi;
-                            cur = (wi == 2) ? w2 : ((wi == 1) ? w1 : w0);
-                        } while (cur == 0u && wi > 0);
-                        qrow = ws.tabq + wi * 32 * G;
-                        crow = ws.tabc + wi * 32;
-                    }
-                    const int b = (31 - __clz(cur)) & 31;
-                    cur ^= 1u << b;
-                    const float x = Elem<E>::to_f(*vp) - crow[b];
-                    vp -= kWT;
+                unsigned long long mlo = ((unsigned long long)mw.y << 32) | mw.x;
+                unsigned long long mhi = ((unsigned long long)mw.w << 32) | mw.z;
+                const E *vp = ws.svals(st) + lane;
+#pragma unroll 4
+                for (int i = 0; i < a.T; ++i) {
+                    const bool use_lo = mlo != 0ull;
+                    const unsigned long long cur = use_lo ? mlo : mhi;
+                    const unsigned long long nxt = cur & (cur - 1ull);
+                    mlo = use_lo ? nxt : mlo;
+                    mhi = use_lo ? mhi : nxt;
+                    const int j = ((__ffsll((long long)cur) - 1) + (use_lo ? 0 : 64)) & (kD - 1);
+                    const float x = Elem<E>::to_f(vp[i * kWT]) - ws.tabc[j];
                     QVec<G> qv;
-                    qv.load(qrow + b * G);
+                    qv.load(ws.tabq + j * G);
 #pragma unroll
                     for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }
@@ -605,14 +740,11 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             }
 #pragma unroll
             for (int g = 0; g < G; ++g) s[g] = valid ? s[g] + ws.qc[g] : -INFINITY;
-            tile_softmax<E, G>(ws, f, s);
-            for (int tb = 0; tb < n; tb += kVB) {
-                if (tb > 0) vr.load(vbase + (size_t)(t0 + tb) * kD, n - tb);
-                tile_pv<E, G>(ws, f, vr, tb, n);
-            }
-            __syncwarp();  // p buffer free
+            float alpha[G];
+            if (tile_softmax<E, G>(ws, f, s, alpha)) pv.rescale(alpha);
+            pv.accumulate(ws, vbase + (size_t)t0 * kD, n);
         }
-        if (!failed) write_partial<G>(a, bh, u, f);
+        if (!failed) write_partial<E, G>(a, bh, u, f, pv);
     }
 
     if (failed) {
@@ -655,7 +787,7 @@ __global__ void __launch_bounds__(kD) combine_kernel(const float *__restrict__ a
 DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms) {
     DecodeGeom g{};
     const size_t stage = dec_stage_bytes(T, es);
-    const size_t table = dec_table_bytes(G);
+    const size_t table = dec_table_bytes(G, T, es);
     const size_t budget = 227 * 1024;
     const int max_w = dec_max_warps(G);
     auto warps_for = [&](int ns) {

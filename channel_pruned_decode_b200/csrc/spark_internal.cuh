@@ -53,10 +53,14 @@ __host__ __device__ inline size_t dec_stage_bytes(int T, int es) {
     return (size_t)kWT * 16 + (size_t)kWT * T * es;
 }
 
-// q' table [kD][G], c table [kD], duplicated p buffer [kWT][G][2], Qc [16],
-// mbarriers, rounded to 128 bytes so that the stages start aligned
-__host__ __device__ inline size_t dec_table_bytes(int G) {
-    const size_t b = (size_t)kD * G * 4 + kD * 4 + (size_t)kWT * G * 8 + 64 + kMaxStagesW * 8;
+// Per-warp tables: bf16 values add a swizzled V tile [kWT][kD] (8 KB) and
+// p as [G][kWT] fp32; then q' [kD][G], c [kD], p as duplicated pairs
+// [kWT][G][2] (fp32 values), Qc [16], mbarriers and the tile's kept-channel
+// lists [T][kWT] bytes; rounded to 128 bytes so that the stages start aligned.
+__host__ __device__ inline size_t dec_vtile_bytes(int es) { return es == 2 ? (size_t)kWT * kD * 2 : 0; }
+__host__ __device__ inline size_t dec_table_bytes(int G, int T, int es) {
+    const size_t b = dec_vtile_bytes(es) + (size_t)G * kWT * 4 + (size_t)kD * G * 4 + kD * 4 +
+                     (size_t)kWT * G * 8 + 64 + kMaxStagesW * 8 + (size_t)kWT * (T > 0 ? T : 1);
     return (b + 127) / 128 * 128;
 }
 
