@@ -184,6 +184,41 @@ template <int G> struct QVec {
     }
 };
 
+// Position of the highest set bit, 0xffffffff for zero.
+__device__ __forceinline__ uint32_t bit_top(uint32_t x) {
+    uint32_t p;
+    asm("bfind.u32 %0, %1;" : "=r"(p) : "r"(x));
+    return p;
+}
+
+// x << n with shift counts of 32 and above giving 0 (PTX shl clamps).
+__device__ __forceinline__ uint32_t shl_clamped(uint32_t x, uint32_t n) {
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
+    return r;
+}
+
+// Stable compaction of the queue (q0, q1, q2, q3) so that its non-empty words
+// come first; byte k of bq is the channel base of word k and moves with it.
+// Works from the back: after the step for slot k, slots k..3 are compacted.
+__device__ __forceinline__ void queue_nonempty(uint32_t &q0, uint32_t &q1, uint32_t &q2, uint32_t &q3,
+                                               uint32_t &bq) {
+    bool e = q2 == 0u;  // drop slot 2
+    q2 = e ? q3 : q2;
+    q3 = e ? 0u : q3;
+    bq = e ? __byte_perm(bq, 0u, 0x4310) : bq;
+    e = q1 == 0u;       // drop slot 1
+    q1 = e ? q2 : q1;
+    q2 = e ? q3 : q2;
+    q3 = e ? 0u : q3;
+    bq = e ? __byte_perm(bq, 0u, 0x4320) : bq;
+    e = q0 == 0u;       // drop slot 0
+    q0 = e ? q1 : q0;
+    q1 = e ? q2 : q1;
+    q2 = e ? q3 : q2;
+    bq = e ? (bq >> 8) : bq;
+}
+
 // Per-warp shared memory: tables, p buffers, mbarriers, then the stage ring.
 template <typename E, int G>
 struct WarpSmem {
@@ -700,26 +735,31 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }
             } else if (a.T > 0) {
-                // Walk the T set bits of the 128-bit mask in ascending order with
-                // no branch: the mask is two 64-bit halves, a select picks the
-                // lower non-empty one, and clearing its lowest bit is 64-bit
-                // arithmetic.  All lanes run exactly T iterations; the i-th set
-                // bit pairs with the i-th packed value.  A mask with fewer than T
-                // bits (a cache never written by spark_prune, or a lane past n)
-                // keeps every index in range.
+                // Walk the T set bits of the 128-bit mask from the top channel
+                // down, pairing the i-th bit from the top with the i-th packed
+                // value from the end.  The non-empty mask words are queued in
+                // descending order first (cur, n1, n2, n3, with their channel
+                // bases as the bytes of bq), so every step is branch-free:
+                // find the top bit, clear it, and move to the next queued word
+                // once the current one is used up.  All lanes run exactly T
+                // steps.  A mask with fewer than T bits (a cache never written
+                // by spark_prune, or a lane past n) keeps every index in range.
                 const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
-                unsigned long long mlo = ((unsigned long long)mw.y << 32) | mw.x;
-                unsigned long long mhi = ((unsigned long long)mw.w << 32) | mw.z;
-                const E *vp = ws.svals(st) + lane;
+                uint32_t cur = mw.w, n1 = mw.z, n2 = mw.y, n3 = mw.x;
+                uint32_t bq = 0x00204060u;  // bases 96, 64, 32, 0 from the low byte up
+                queue_nonempty(cur, n1, n2, n3, bq);
+                const E *vp = ws.svals(st) + lane + (a.T - 1) * kWT;
 #pragma unroll 4
                 for (int i = 0; i < a.T; ++i) {
-                    const bool use_lo = mlo != 0ull;
-                    const unsigned long long cur = use_lo ? mlo : mhi;
-                    const unsigned long long nxt = cur & (cur - 1ull);
-                    mlo = use_lo ? nxt : mlo;
-                    mhi = use_lo ? mhi : nxt;
-                    const int j = ((__ffsll((long long)cur) - 1) + (use_lo ? 0 : 64)) & (kD - 1);
-                    const float x = Elem<E>::to_f(vp[i * kWT]) - ws.tabc[j];
+                    const uint32_t pos = bit_top(cur);        // 0xffffffff when cur == 0
+                    const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
+                    cur ^= shl_clamped(1u, pos);
+                    const bool e = cur == 0u;
+                    cur = e ? n1 : cur;
+                    n1 = e ? n2 : n1;
+                    n2 = e ? n3 : n2;
+                    bq = e ? (bq >> 8) : bq;
+                    const float x = Elem<E>::to_f(vp[-i * kWT]) - ws.tabc[j];
                     QVec<G> qv;
                     qv.load(ws.tabq + j * G);
 #pragma unroll
