@@ -62,10 +62,10 @@ template <> struct KSlice<__nv_bfloat16> {
 #pragma unroll
         for (int i = 0; i < kWords; ++i) w[i] = 0u;
     }
-    // |k| as fp32 bits
-    __device__ __forceinline__ uint32_t abs_bits(int i) const {
-        const uint32_t x = w[i >> 1];
-        return (i & 1) ? (x & 0x7fff0000u) : ((x << 16) & 0x7fffffffu);
+    // (|k_2i|, |k_2i+1|) as fp32
+    __device__ __forceinline__ float2 abs_pair(int i) const {
+        const uint32_t a = w[i] & 0x7fff7fffu;
+        return make_float2(__uint_as_float(a << 16), __uint_as_float(a & 0xffff0000u));
     }
     __device__ __forceinline__ uint16_t raw(int i) const {
         const uint32_t x = w[i >> 1];
@@ -88,7 +88,9 @@ template <> struct KSlice<float> {
 #pragma unroll
         for (int i = 0; i < kWords; ++i) w[i] = 0u;
     }
-    __device__ __forceinline__ uint32_t abs_bits(int i) const { return w[i] & 0x7fffffffu; }
+    __device__ __forceinline__ float2 abs_pair(int i) const {
+        return make_float2(__uint_as_float(w[2 * i] & 0x7fffffffu), __uint_as_float(w[2 * i + 1] & 0x7fffffffu));
+    }
     __device__ __forceinline__ uint32_t raw(int i) const { return w[i]; }
 };
 
@@ -111,30 +113,45 @@ __device__ __forceinline__ int quad_sum(int v) {
     return v;
 }
 
-// Count of the quad's keys >= mid over the packed 16-bit keys.  A key16 is
-// the upper half of the fp32 saliency (a positive bf16 pattern), clamped to
-// 0x7bff: read as fp16 bit patterns these stay in the same order, and fp16
-// packed compare + add (one instruction each per two channels) count them.
-// `mid` is 0 or >= 0x400 (a normal fp16 pattern); keys below 0x400 sit below
-// every probe.  Counts <= 32 per lane are exact in fp16.
-__device__ __forceinline__ __half quad_count16(const uint32_t (&kp)[16], uint32_t mid) {
-    const uint32_t mm = mid * 0x10001u;
-    const __half2 m2 = *reinterpret_cast<const __half2 *>(&mm);
-    const __half2 z = __float2half2_rn(0.f);
-    __half2 a0 = z, a1 = z, a2 = z, a3 = z;
+// fp16x2 a >= b per half: 1.0 / 0.0.  Subnormal halves compare exactly (no
+// flush to zero).
+__device__ __forceinline__ uint32_t hge2_one(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("set.ge.f16x2.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// fp16x2 a >= b per half: 0xffff / 0x0000.
+__device__ __forceinline__ uint32_t hge2_mask(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("set.ge.u32.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// D += A * B for one m16n8k16 fp16 tile with fp16 accumulators.
+__device__ __forceinline__ void mma_f16(uint32_t &d0, uint32_t &d1, uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f16.f16.f16.f16 {%0,%1}, {%2,%3,%4,%5}, {%6,%7}, {%0,%1};"
+        : "+r"(d0), "+r"(d1)
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Number of the quad's 128 16-bit keys >= the probe p2 (the probe in both
+// halves), as an exact fp16 integer.  The 0/1 compare results are the A
+// operand of tensor-core tiles whose B operand is all ones: row r of A takes
+// its 16 entries from the quad r mod 8 of the warp, so each row sum counts
+// keys of one token, and rows r and r + 8 (the two accumulator registers)
+// together cover all 128 channels.  Which channel sits in which column is
+// irrelevant to a sum.  Every lane of the quad receives the count.
+__device__ __forceinline__ __half count_ge16(const uint32_t (&kp)[16], uint32_t p2) {
+    constexpr uint32_t kOne2 = 0x3c003c00u;  // fp16 (1, 1)
+    uint32_t d0 = 0u, d1 = 0u;
 #pragma unroll
-    for (int i = 0; i < 16; i += 4) {
-        a0 = __hadd2(a0, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 0]), m2));
-        a1 = __hadd2(a1, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 1]), m2));
-        a2 = __hadd2(a2, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 2]), m2));
-        a3 = __hadd2(a3, __hge2(*reinterpret_cast<const __half2 *>(&kp[i + 3]), m2));
-    }
-    a0 = __hadd2(__hadd2(a0, a1), __hadd2(a2, a3));
-    // both halves -> one count (<= 32, exact), then the quad's sum (<= 128, exact)
-    __half c = __hadd(__low2half(a0), __high2half(a0));
-    c = __hadd(c, __shfl_xor_sync(0xffffffffu, c, 1));
-    c = __hadd(c, __shfl_xor_sync(0xffffffffu, c, 2));
-    return c;
+    for (int m = 0; m < 4; ++m)
+        mma_f16(d0, d1, hge2_one(kp[4 * m + 0], p2), hge2_one(kp[4 * m + 1], p2), hge2_one(kp[4 * m + 2], p2),
+                hge2_one(kp[4 * m + 3], p2), kOne2, kOne2);
+    const __half2 c = __hadd2(*reinterpret_cast<const __half2 *>(&d0), *reinterpret_cast<const __half2 *>(&d1));
+    return __low2half(c);
 }
 
 __device__ __forceinline__ int quad_count32(const uint32_t (&key)[32], uint32_t mid) {
@@ -144,63 +161,66 @@ __device__ __forceinline__ int quad_count32(const uint32_t (&key)[32], uint32_t 
     return quad_sum(c);
 }
 
-// Mask word (32 channels) of this lane's quarter of the token: the T largest
-// exact fp32 keys over the quad, ties to the lower channel index.
-//
-// Phase 1 searches the T-th largest 16-bit key with packed counts, starting
-// at the previous token's threshold `tau16` and galloping outward until the
-// bracket closes, then bisecting; it ends either with a probe that leaves
-// exactly T keys above it (the usual case) or with the 16-bit tie band
-// [tau16, tau16+1) holding the boundary.  Phase 2 bisects the exact 32-bit
-// keys inside that band.  Both loops have warp-uniform trip counts (quads
-// that are done idle), so the quad shuffles always see the full warp.
-__device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
-                                                 int s, uint32_t &tau16) {
-    if (T <= 0) return 0u;
-    if (T >= kD) return 0xffffffffu;
+__device__ __forceinline__ float half_bits_to_float(uint32_t p) {
+    return __half2float(__ushort_as_half((unsigned short)p));
+}
 
-    // ---- phase 1: 16-bit keys.  count(>= lo) >= T > count(>= hi).
-    // Probes: the previous token's threshold, then galloping away from an
-    // open side of the bracket (step doubling), then bisection.  The bracket
-    // update is written with selects so that quads in different states of
-    // the search do not diverge.
-    constexpr uint32_t kTop = 0x7c00u;  // above the clamp: nothing reaches it
+constexpr uint32_t kTop16 = 0x7c01u;  // above +inf: no key reaches it, never probed
+constexpr uint32_t kGallop16 = 256u;  // first gallop step, fp16 units (1/4 octave)
+
+// Mask word (32 channels) of this lane's quarter of the token: the T largest
+// exact fp32 keys over the quad, ties to the lower channel index.  0 < T < 128.
+//
+// kp[i] holds the 16-bit keys of channels i (low half) and i + 16 (high
+// half): the fp32 keys scaled by a power of two and rounded to fp16, which is
+// monotone in the key.  Phase 1 finds the fp16 threshold: starting at `tau`,
+// it gallops away from the open side of the bracket (step doubling), then
+// bisects, and ends either with a probe that leaves exactly T keys at or
+// above it (the usual case) or with a one-unit bracket [lo, lo + 1) whose
+// band of equal fp16 keys holds the boundary.  Phase 2 bisects the exact
+// fp32 keys inside that band, and a scan over the quad settles exact ties.
+// Every loop has a warp-uniform trip count (finished quads idle), so the
+// quad shuffles and the warp-wide tensor-core counts see the full warp.
+__device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
+                                                 int s, float inv_scale, uint32_t &tau) {
     const __half hT = __int2half_rn(T);
-    uint32_t lo = 0u, hi = kTop;
-    __half c_hi_h = __int2half_rn(0);
-    bool exact = false;
-    bool done = false;
-    uint32_t step = 64u;
-    uint32_t mid = min(max(tau16, 1u), kTop - 1u);
+    uint32_t lo = 0u, hi = kTop16;  // count(>= lo) >= T > count(>= hi)
+    bool exact = false, done = false;
+    uint32_t step = kGallop16;
+    uint32_t mid = min(max(tau, 1u), kTop16 - 1u);
     while (__any_sync(0xffffffffu, !done)) {
-        const uint32_t probe = (mid > 0u && mid < 0x400u) ? 0x400u : mid;
-        const __half c = quad_count16(kp, probe);
+        const __half c = count_ge16(kp, mid * 0x10001u);
         const bool ge = __hge(c, hT);
-        const bool eq = __heq(c, hT);
         const bool act = !done;
         lo = (act && ge) ? mid : lo;
         hi = (act && !ge) ? mid : hi;
-        c_hi_h = (act && !ge) ? c : c_hi_h;
+        const bool eq = __heq(c, hT);
         exact = exact || (act && eq);
         done = done || eq || (hi - lo <= 1u);
-        const bool up = (hi == kTop), down = (lo == 0u);
-        const uint32_t gal_up = min(lo + step, kTop - 1u);
+        const bool up = hi == kTop16, down = lo == 0u;
+        const uint32_t gal_up = min(lo + step, kTop16 - 1u);
         const uint32_t gal_dn = max(hi > step ? hi - step : hi >> 1, 1u);
         const uint32_t bis = lo + ((hi - lo) >> 1);
         mid = up ? gal_up : (down ? gal_dn : bis);
         step = (up || down) ? step << 1 : step;
     }
-    int c_hi = __half2int_rn(c_hi_h);
-    tau16 = lo;
+    tau = lo;
 
-    // ---- phase 2: exact keys inside the band of 16-bit key == lo.  Quads
-    // whose phase 1 was exact skip it (done2) but stay in the uniform loop.
-    // Bands in fp32 key space: [0, 0x400 << 16) for lo == 0 (every probe
-    // below 0x400 acts as 0x400), [0x7bff << 16, 2^31) for the clamp value,
-    // [lo << 16, (lo + 1) << 16) otherwise.  When exact, exactly T keys have a
-    // 16-bit key >= lo, i.e. an fp32 key >= max(lo, 0x400) << 16.
-    uint32_t lo32 = exact ? (max(lo, 0x400u) << 16) : ((lo == 0u) ? 0u : (lo << 16));
-    uint32_t hi32 = (lo == 0u) ? (0x400u << 16) : ((lo >= 0x7bffu) ? 0x80000000u : ((lo + 1u) << 16));
+    // fp16 decision: keys >= lo (exactly T of them when `exact`)
+    uint32_t m = 0u;
+    {
+        const uint32_t p2 = lo * 0x10001u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m |= hge2_mask(kp[i], p2) & (0x00010001u << i);
+    }
+    if (!__any_sync(0xffffffffu, !exact)) return m;
+
+    // ---- phase 2 on the exact keys.  With v = the fp16 value of lo - 1 and
+    // u that of hi, every key whose fp16 key is >= lo is > v / scale, and
+    // every key >= u / scale has an fp16 key >= hi, so [v / scale, u / scale)
+    // in fp32 bit patterns brackets the T-th largest key.
+    uint32_t lo32 = lo == 0u ? 0u : __float_as_uint(half_bits_to_float(lo - 1u) * inv_scale);
+    uint32_t hi32 = hi >= kTop16 ? 0x7f800001u : __float_as_uint(half_bits_to_float(hi) * inv_scale);
     bool exact32 = exact;
     bool done2 = exact || (hi32 - lo32 <= 1u);
     while (__any_sync(0xffffffffu, !done2)) {
@@ -212,36 +232,37 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
                 if (c == T) { exact32 = true; done2 = true; }
             } else {
                 hi32 = mid32;
-                c_hi = c;
             }
             if (hi32 - lo32 <= 1u) done2 = true;
         }
     }
-    // exact32: exactly T keys are >= lo32.  Otherwise lo32 is the T-th largest
-    // key, c_hi keys are above it, and the first T - c_hi keys equal to it (in
-    // channel order over the quad) are kept.
+    // exact32: exactly T keys are >= lo32.  Otherwise lo32 is the T-th
+    // largest key: the keys above it are kept, and of the keys equal to it the
+    // first T - (number above) in channel order over the quad.
     const uint32_t thr = exact32 ? lo32 : lo32 + 1u;
-    uint32_t m = 0u;
+    uint32_t m32 = 0u;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) m |= (key[i] >= thr ? 1u : 0u) << i;
-    if (__any_sync(0xffffffffu, !exact32)) {  // warp-uniform: the scan below shuffles
+    for (int i = 0; i < 32; ++i) m32 |= (key[i] >= thr ? 1u : 0u) << i;
+    if (__any_sync(0xffffffffu, !exact32)) {  // warp-uniform: the scans below shuffle
+        const int above = quad_sum(__popc(m32));
         int e = 0;
 #pragma unroll
         for (int i = 0; i < 32; ++i) e += (key[i] == lo32) ? 1 : 0;
         int r = quad_excl_scan(e, s);
         if (!exact32) {
-            const int need = T - c_hi;
+            const int need = T - above;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 if (key[i] == lo32) {
-                    if (r < need) m |= 1u << i;
+                    if (r < need) m32 |= 1u << i;
                     ++r;
                 }
             }
         }
     }
-    return m;
+    return exact ? m : m32;
 }
+
 template <typename E>
 __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
@@ -249,6 +270,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     using Raw = typename RawT<E>::type;
     __shared__ __align__(16) Raw vtile[2][kD * 32];  // [kept index][token in group]
     __shared__ double red[2][kPruneThreads / 32];
+    __shared__ uint32_t qmax[kPruneThreads / 32];
     // window-query norms of this head, one padded row per quarter (stride 36
     // floats): the 4 quarters' 16-byte reads fall in distinct banks
     __shared__ __align__(16) float qs[4 * 36];
@@ -260,10 +282,31 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     const int tl = warp * 8 + (lane >> 2);  // token within the 32-token group
     const long S32 = ((long)S + 31) / 32 * 32;
 
-    if (tid < kD) qs[(tid >> 5) * 36 + (tid & 31)] = __ldg(qn + bh * kD + tid);
+    // the 16-bit keys are fp16(key * scale), scale = 2^-floor(log2 max_j qn_j),
+    // so the largest window-query norm maps into [1, 2) and the keys of
+    // ordinary keys sit in fp16's normal range
+    {
+        const float q = __ldg(qn + bh * kD + tid);  // kPruneThreads == kD
+        qs[(tid >> 5) * 36 + (tid & 31)] = q;
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(q) & 0x7fffffffu);
+        if (lane == 0) qmax[warp] = mx;
+    }
     __syncthreads();
+    float scale = 1.f, inv_scale = 1.f;
+    {
+        uint32_t mx = qmax[0];
+#pragma unroll
+        for (int w = 1; w < kPruneThreads / 32; ++w) mx = max(mx, qmax[w]);
+        const int e = (int)(mx >> 23);
+        if (e > 0 && e < 255) {
+            const int x = min(max(127 - e, -64), 64);
+            scale = __uint_as_float((uint32_t)(127 + x) << 23);
+            inv_scale = __uint_as_float((uint32_t)(127 - x) << 23);
+        }
+    }
+    const float2 scale2 = make_float2(scale, scale);
 
-    uint32_t tau16 = 0x3f80u;  // reset from the first token's keys below
+    uint32_t tau = 1u;
     double acc_w = 0.0, acc_w2 = 0.0;
     const long g_first = (long)chunk * kPruneGroups;
     KSlice<E> ks, ks_next;
@@ -285,54 +328,62 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
             else ks_next.zero();
         }
 
-        // exact fp32 saliency keys and their packed 16-bit truncations
+        // exact fp32 saliency keys w_j = qn_j * |k_j| (packed fp32 multiplies,
+        // each rounded like a scalar one)
         uint32_t key[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float4 q4 = *reinterpret_cast<const float4 *>(qs + s * 36 + 4 * c);
-            const float qq[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                key[4 * c + e] = __float_as_uint(__fmul_rn(qq[e], __uint_as_float(ks.abs_bits(4 * c + e))));
+            const float2 w01 = __fmul2_rn(make_float2(q4.x, q4.y), ks.abs_pair(2 * c));
+            const float2 w23 = __fmul2_rn(make_float2(q4.z, q4.w), ks.abs_pair(2 * c + 1));
+            key[4 * c + 0] = __float_as_uint(w01.x);
+            key[4 * c + 1] = __float_as_uint(w01.y);
+            key[4 * c + 2] = __float_as_uint(w23.x);
+            key[4 * c + 3] = __float_as_uint(w23.y);
         }
-        uint32_t kp[16];
-        {
-            const uint32_t cap = 0x7bff7bffu;
-            const __half2 cap2 = *reinterpret_cast<const __half2 *>(&cap);
+        uint32_t m;
+        if (T <= 0) {
+            m = 0u;
+        } else if (T >= kD) {
+            m = 0xffffffffu;
+        } else {
+            // 16-bit keys of channels (i, i + 16)
+            uint32_t kp[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const uint32_t pr = __byte_perm(key[2 * i], key[2 * i + 1], 0x7632);
-                const __half2 c = __hmin2(*reinterpret_cast<const __half2 *>(&pr), cap2);
-                kp[i] = *reinterpret_cast<const uint32_t *>(&c);
+                const float2 v = __fmul2_rn(make_float2(__uint_as_float(key[i]), __uint_as_float(key[i + 16])),
+                                            scale2);
+                const __half2 h = __floats2half2_rn(v.x, v.y);
+                kp[i] = *reinterpret_cast<const uint32_t *>(&h);
             }
-        }
-
-        if (gi == 0) {
-            // first token of this quad: start 1.5 octaves (192 key16 units)
-            // below its largest key instead of at a fixed guess
-            __half2 mx = *reinterpret_cast<const __half2 *>(&kp[0]);
+            if (gi == 0) {
+                // first token of this quad: start 1.5 octaves below its largest key
+                __half2 mx = *reinterpret_cast<const __half2 *>(&kp[0]);
 #pragma unroll
-            for (int i = 1; i < 16; ++i) mx = __hmax2(mx, *reinterpret_cast<const __half2 *>(&kp[i]));
-            const uint32_t mb = *reinterpret_cast<const uint32_t *>(&mx);
-            uint32_t m16 = max(mb & 0xffffu, mb >> 16);
-            m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
-            m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
-            tau16 = m16 > 192u ? m16 - 192u : 1u;
+                for (int i = 1; i < 16; ++i) mx = __hmax2(mx, *reinterpret_cast<const __half2 *>(&kp[i]));
+                const uint32_t mb = *reinterpret_cast<const uint32_t *>(&mx);
+                uint32_t m16 = max(mb & 0xffffu, mb >> 16);
+                m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
+                m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
+                tau = m16 > 1536u ? m16 - 1536u : 1u;
+            }
+            uint32_t lo = tau;
+            m = select_top_t(key, kp, T, s, inv_scale, lo);
+            // next start: running mean of this quad's thresholds
+            tau = gi == 0 ? lo : (uint32_t)((int)tau + (((int)lo - (int)tau) >> 1));
         }
-        const uint32_t m = select_top_t(key, kp, T, s, tau16);
         if (valid) mask[((size_t)bh * S + t) * kMaskWords + s] = m;
 
         // pruned-saliency sums (fp32 over this lane's 32 channels, fp64 across
         // tokens) and the kept values, in ascending channel order, into the
         // staging tile
-        Raw *vt = vtile[gi & 1];
-        int pos = quad_excl_scan(__popc(m), s);
+        Raw *dst = vtile[gi & 1] + quad_excl_scan(__popc(m), s) * 32 + tl;
         float sw = 0.f, sw2 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             if ((m >> i) & 1u) {
-                vt[pos * 32 + tl] = (Raw)ks.raw(i);
-                ++pos;
+                *dst = (Raw)ks.raw(i);
+                dst += 32;
             } else {
                 const float w = __uint_as_float(key[i]);
                 sw = __fadd_rn(sw, w);
@@ -346,9 +397,9 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
         __syncthreads();
         // 32 tokens x T values, contiguous in the interleaved layout
         const int nvec = (int)((size_t)32 * T * sizeof(E) / 16);
-        uint4 *dst = reinterpret_cast<uint4 *>(vals + (size_t)bh * S32 * T + (size_t)t0 * T);
-        const uint4 *src = reinterpret_cast<const uint4 *>(vt);
-        for (int vi = tid; vi < nvec; vi += kPruneThreads) __stcs(dst + vi, src[vi]);
+        uint4 *dstg = reinterpret_cast<uint4 *>(vals + (size_t)bh * S32 * T + (size_t)t0 * T);
+        const uint4 *src = reinterpret_cast<const uint4 *>(vtile[gi & 1]);
+        for (int vi = tid; vi < nvec; vi += kPruneThreads) __stcs(dstg + vi, src[vi]);
         ks = ks_next;
     }
 

@@ -128,6 +128,25 @@ def test_ties_and_zero_norm_channels():
         assert_out_close(out.cpu().numpy().reshape(-1, D), o_ref, f"ties T={T}")
 
 
+@pytest.mark.parametrize("k_exp,q_exp,spread", [(-30, 0, 0), (-12, 0, 0), (20, 0, 0), (40, 0, 0),
+                                                 (0, -40, 0), (0, 30, 0), (0, 0, 30), (-20, 10, 12)])
+def test_key_magnitude_extremes(k_exp, q_exp, spread):
+    # keys and window queries scaled by powers of two (and, with `spread`, a
+    # random per-channel exponent in [-spread, spread]): saliencies far below,
+    # inside and far above the 16-bit search keys' normal range, which pushes
+    # the selection into its underflow, overflow and exact-tie paths
+    g = torch.Generator(device=DEV).manual_seed(100 + k_exp + 3 * q_exp + spread)
+    R, Hkv, G, W, S = 1, 2, 4, 16, 520
+    ch = torch.randint(-spread, spread + 1, (D,), generator=g, device=DEV).float() if spread else \
+        torch.zeros(D, device=DEV)
+    k = (torch.randn((R, Hkv, S, D), generator=g, device=DEV) * torch.exp2(ch + k_exp)).to(torch.bfloat16)
+    q_obs = (torch.randn((R, Hkv * G, W, D), generator=g, device=DEV) * 2.0 ** q_exp).to(torch.bfloat16)
+    for T in (1, 26, 64, 127):
+        kc = run_prune(k, q_obs, G, W, T)
+        torch.cuda.synchronize()
+        _check_prune(kc, to_np(k), to_np(q_obs), G, T, f"extremes k2^{k_exp} q2^{q_exp} spread {spread} T={T}")
+
+
 def test_lambda0_matches_dense_sdpa():
     # T = D keeps every channel: the GPU decode must equal plain attention
     wl = scaled(WORKLOADS["llama1l"], S=3000, Hkv=2, seed=9)
