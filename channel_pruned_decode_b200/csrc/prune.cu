@@ -166,43 +166,67 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t p) {
 }
 
 constexpr uint32_t kTop16 = 0x7c01u;  // above +inf: no key reaches it, never probed
-constexpr uint32_t kGallop16 = 256u;  // first gallop step, fp16 units (1/4 octave)
+constexpr uint32_t kGallop16 = 256u;  // first gallop step of the fallback search, fp16 units
+constexpr int kLift = 11;             // search window 2^11 fp16 units (2 octaves) around the estimate
+constexpr int kLiftCold = 12;         // first token of a quad: 2^12 units (4 octaves) below its top key
 
 // Mask word (32 channels) of this lane's quarter of the token: the T largest
 // exact fp32 keys over the quad, ties to the lower channel index.  0 < T < 128.
 //
 // kp[i] holds the 16-bit keys of channels i (low half) and i + 16 (high
 // half): the fp32 keys scaled by a power of two and rounded to fp16, which is
-// monotone in the key.  Phase 1 finds the fp16 threshold: starting at `tau`,
-// it gallops away from the open side of the bracket (step doubling), then
-// bisects, and ends either with a probe that leaves exactly T keys at or
-// above it (the usual case) or with a one-unit bracket [lo, lo + 1) whose
-// band of equal fp16 keys holds the boundary.  Phase 2 bisects the exact
-// fp32 keys inside that band, and a scan over the quad settles exact ties.
-// Every loop has a warp-uniform trip count (finished quads idle), so the
-// quad shuffles and the warp-wide tensor-core counts see the full warp.
+// monotone in the key.  Phase 1 finds the fp16 threshold by binary lifting
+// over the window [base, base + 2^K): assuming count(>= base) >= T, after the
+// probe for bit b, lo is the largest point base + j * 2^b with
+// count(>= lo) >= T.  A probe that counts exactly T keys fixes the mask
+// (keys >= lo), and later probes keep that true, so the loop ends as soon as
+// every quad of the warp has seen one.  Otherwise the band of fp16 keys equal
+// to lo holds the boundary; if the window may not have bracketed it (lo never
+// moved, or reached the window's top) a gallop + bisection over the whole key
+// range redoes the search.  Phase 2 bisects the exact fp32 keys inside the
+// band, and a scan over the quad settles exact ties.  Every loop has a
+// warp-uniform trip count (finished quads idle), so the quad shuffles and the
+// warp-wide tensor-core counts see the full warp.
 __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
-                                                 int s, float inv_scale, uint32_t &tau) {
+                                                 int s, float inv_scale, uint32_t base, int K, bool skip,
+                                                 uint32_t &tau) {
     const __half hT = __int2half_rn(T);
-    uint32_t lo = 0u, hi = kTop16;  // count(>= lo) >= T > count(>= hi)
-    bool exact = false, done = false;
-    uint32_t step = kGallop16;
-    uint32_t mid = min(max(tau, 1u), kTop16 - 1u);
-    while (__any_sync(0xffffffffu, !done)) {
-        const __half c = count_ge16(kp, mid * 0x10001u);
-        const bool ge = __hge(c, hT);
-        const bool act = !done;
-        lo = (act && ge) ? mid : lo;
-        hi = (act && !ge) ? mid : hi;
-        const bool eq = __heq(c, hT);
-        exact = exact || (act && eq);
-        done = done || eq || (hi - lo <= 1u);
-        const bool up = hi == kTop16, down = lo == 0u;
-        const uint32_t gal_up = min(lo + step, kTop16 - 1u);
-        const uint32_t gal_dn = max(hi > step ? hi - step : hi >> 1, 1u);
-        const uint32_t bis = lo + ((hi - lo) >> 1);
-        mid = up ? gal_up : (down ? gal_dn : bis);
-        step = (up || down) ? step << 1 : step;
+    uint32_t lo = base;
+    bool exact = skip;  // lanes past the end of the keys take no part
+    for (int b = K - 1; b >= 0; --b) {
+        const uint32_t p = lo + (1u << b);
+        const __half c = count_ge16(kp, p * 0x10001u);
+        lo = __hge(c, hT) ? p : lo;
+        exact = exact || __heq(c, hT);
+        if (__all_sync(0xffffffffu, exact)) break;
+    }
+    uint32_t hi = lo + 1u;
+    const bool suspect = !exact && (lo == base || lo == base + (1u << K) - 1u);
+    if (__any_sync(0xffffffffu, suspect)) {
+        // count(>= glo) >= T > count(>= ghi); gallop from lo away from the
+        // open side of the bracket (step doubling), then bisect
+        uint32_t glo = 0u, ghi = kTop16;
+        bool done = !suspect;
+        uint32_t step = kGallop16;
+        uint32_t mid = min(max(lo, 1u), kTop16 - 1u);
+        while (__any_sync(0xffffffffu, !done)) {
+            const __half c = count_ge16(kp, mid * 0x10001u);
+            const bool ge = __hge(c, hT);
+            const bool act = !done;
+            glo = (act && ge) ? mid : glo;
+            ghi = (act && !ge) ? mid : ghi;
+            const bool eq = __heq(c, hT);
+            exact = exact || (act && eq);
+            done = done || eq || (ghi - glo <= 1u);
+            const bool up = ghi == kTop16, down = glo == 0u;
+            const uint32_t gal_up = min(glo + step, kTop16 - 1u);
+            const uint32_t gal_dn = (uint32_t)max((int)ghi - (int)step, 1);
+            const uint32_t bis = glo + ((ghi - glo) >> 1);
+            mid = up ? gal_up : (down ? gal_dn : bis);
+            step <<= 1;
+        }
+        lo = suspect ? glo : lo;
+        hi = suspect ? ghi : hi;
     }
     tau = lo;
 
@@ -216,9 +240,9 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     if (!__any_sync(0xffffffffu, !exact)) return m;
 
     // ---- phase 2 on the exact keys.  With v = the fp16 value of lo - 1 and
-    // u that of hi, every key whose fp16 key is >= lo is > v / scale, and
-    // every key >= u / scale has an fp16 key >= hi, so [v / scale, u / scale)
-    // in fp32 bit patterns brackets the T-th largest key.
+    // u that of hi = lo + 1, every key whose fp16 key is >= lo is > v / scale,
+    // and every key >= u / scale has an fp16 key >= hi, so [v / scale,
+    // u / scale) in fp32 bit patterns brackets the T-th largest key.
     uint32_t lo32 = lo == 0u ? 0u : __float_as_uint(half_bits_to_float(lo - 1u) * inv_scale);
     uint32_t hi32 = hi >= kTop16 ? 0x7f800001u : __float_as_uint(half_bits_to_float(hi) * inv_scale);
     bool exact32 = exact;
@@ -268,7 +292,8 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
                  E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks) {
     using Raw = typename RawT<E>::type;
-    __shared__ __align__(16) Raw vtile[2][kD * 32];  // [kept index][token in group]
+    // per-warp staging of the kept values: [kept index][8 tokens of the warp]
+    __shared__ __align__(16) Raw vtile[kPruneThreads / 32][kD * 8];
     __shared__ double red[2][kPruneThreads / 32];
     __shared__ uint32_t qmax[kPruneThreads / 32];
     // window-query norms of this head, one padded row per quarter (stride 36
@@ -279,7 +304,8 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     const int chunk = blockIdx.x % n_chunks;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int s = lane & 3;                 // quarter: channels [32s, 32s+32)
-    const int tl = warp * 8 + (lane >> 2);  // token within the 32-token group
+    const int tq = lane >> 2;               // token within the warp's 8
+    const int tl = warp * 8 + tq;           // token within the 32-token group
     const long S32 = ((long)S + 31) / 32 * 32;
 
     // the 16-bit keys are fp16(key * scale), scale = 2^-floor(log2 max_j qn_j),
@@ -306,40 +332,37 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     }
     const float2 scale2 = make_float2(scale, scale);
 
+    Raw *vt = vtile[warp];
     uint32_t tau = 1u;
     double acc_w = 0.0, acc_w2 = 0.0;
     const long g_first = (long)chunk * kPruneGroups;
-    KSlice<E> ks, ks_next;
-    {
-        const long t = g_first * 32 + tl;
-        if (t < S) ks.load(k + ((size_t)bh * S + t) * kD + 32 * s);
-        else ks.zero();
-    }
-    for (int gi = 0; gi < kPruneGroups; ++gi) {
-        const long grp = g_first + gi;
-        const long t0 = grp * 32;
-        if (t0 >= S) break;  // uniform across the CTA
-        const long t = t0 + tl;
+    const E *krow = k + ((size_t)bh * S + g_first * 32 + tl) * kD + 32 * s;  // this lane's slice, group 0
+    E *gvals = vals + (size_t)bh * S32 * T + (size_t)g_first * 32 * T;      // group 0's values
+
+    // one 32-token group: select, write the mask, stage and store the kept
+    // values, accumulate the pruned-saliency sums.  `cur` holds this group's
+    // slice; the next group's slice is loaded into `nxt` first.
+    auto group = [&](int gi, KSlice<E> &cur, KSlice<E> &nxt) {
+        const long t = (g_first + gi) * 32 + tl;
         const bool valid = t < S;
-        // prefetch the next group's slice while this one is selected
-        {
-            const long tn = t + 32;
-            if (gi + 1 < kPruneGroups && tn < S) ks_next.load(k + ((size_t)bh * S + tn) * kD + 32 * s);
-            else ks_next.zero();
-        }
+        if (gi + 1 < kPruneGroups && t + 32 < S) nxt.load(krow + (size_t)(gi + 1) * 32 * kD);
+        else nxt.zero();
 
         // exact fp32 saliency keys w_j = qn_j * |k_j| (packed fp32 multiplies,
-        // each rounded like a scalar one)
+        // each rounded like a scalar one), and their scaled copies
         uint32_t key[32];
+        float2 wsc[16];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             const float4 q4 = *reinterpret_cast<const float4 *>(qs + s * 36 + 4 * c);
-            const float2 w01 = __fmul2_rn(make_float2(q4.x, q4.y), ks.abs_pair(2 * c));
-            const float2 w23 = __fmul2_rn(make_float2(q4.z, q4.w), ks.abs_pair(2 * c + 1));
+            const float2 w01 = __fmul2_rn(make_float2(q4.x, q4.y), cur.abs_pair(2 * c));
+            const float2 w23 = __fmul2_rn(make_float2(q4.z, q4.w), cur.abs_pair(2 * c + 1));
             key[4 * c + 0] = __float_as_uint(w01.x);
             key[4 * c + 1] = __float_as_uint(w01.y);
             key[4 * c + 2] = __float_as_uint(w23.x);
             key[4 * c + 3] = __float_as_uint(w23.y);
+            wsc[2 * c] = __fmul2_rn(w01, scale2);
+            wsc[2 * c + 1] = __fmul2_rn(w23, scale2);
         }
         uint32_t m;
         if (T <= 0) {
@@ -351,13 +374,15 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
             uint32_t kp[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float2 v = __fmul2_rn(make_float2(__uint_as_float(key[i]), __uint_as_float(key[i + 16])),
-                                            scale2);
-                const __half2 h = __floats2half2_rn(v.x, v.y);
+                const float a = (i & 1) ? wsc[i >> 1].y : wsc[i >> 1].x;
+                const float b = (i & 1) ? wsc[8 + (i >> 1)].y : wsc[8 + (i >> 1)].x;
+                const __half2 h = __floats2half2_rn(a, b);
                 kp[i] = *reinterpret_cast<const uint32_t *>(&h);
             }
+            uint32_t base;
+            int K;
             if (gi == 0) {
-                // first token of this quad: start 1.5 octaves below its largest key
+                // first token of this quad: the window ends at its largest key
                 __half2 mx = *reinterpret_cast<const __half2 *>(&kp[0]);
 #pragma unroll
                 for (int i = 1; i < 16; ++i) mx = __hmax2(mx, *reinterpret_cast<const __half2 *>(&kp[i]));
@@ -365,25 +390,33 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
                 uint32_t m16 = max(mb & 0xffffu, mb >> 16);
                 m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
                 m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
-                tau = m16 > 1536u ? m16 - 1536u : 1u;
+                K = kLiftCold;
+                base = m16 > (1u << K) - 1u ? m16 - ((1u << K) - 1u) : 0u;
+            } else {
+                // later tokens: centred on the running threshold estimate
+                K = kLift;
+                base = tau > (1u << (K - 1)) ? tau - (1u << (K - 1)) : 0u;
             }
-            uint32_t lo = tau;
-            m = select_top_t(key, kp, T, s, inv_scale, lo);
-            // next start: running mean of this quad's thresholds
+            base = min(base, kTop16 - (1u << K));
+            uint32_t lo;
+            m = select_top_t(key, kp, T, s, inv_scale, base, K, !valid, lo);
+            m = valid ? m : 0u;
+            // next estimate: running mean of this quad's thresholds
             tau = gi == 0 ? lo : (uint32_t)((int)tau + (((int)lo - (int)tau) >> 1));
+            tau = valid ? tau : 1u;
         }
         if (valid) mask[((size_t)bh * S + t) * kMaskWords + s] = m;
 
         // pruned-saliency sums (fp32 over this lane's 32 channels, fp64 across
         // tokens) and the kept values, in ascending channel order, into the
-        // staging tile
-        Raw *dst = vtile[gi & 1] + quad_excl_scan(__popc(m), s) * 32 + tl;
+        // warp's staging tile
+        Raw *dst = vt + quad_excl_scan(__popc(m), s) * 8 + tq;
         float sw = 0.f, sw2 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             if ((m >> i) & 1u) {
-                *dst = (Raw)ks.raw(i);
-                dst += 32;
+                *dst = (Raw)cur.raw(i);
+                dst += 8;
             } else {
                 const float w = __uint_as_float(key[i]);
                 sw = __fadd_rn(sw, w);
@@ -394,13 +427,28 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
             acc_w = __dadd_rn(acc_w, (double)sw);
             acc_w2 = __dadd_rn(acc_w2, (double)sw2);
         }
-        __syncthreads();
-        // 32 tokens x T values, contiguous in the interleaved layout
-        const int nvec = (int)((size_t)32 * T * sizeof(E) / 16);
-        uint4 *dstg = reinterpret_cast<uint4 *>(vals + (size_t)bh * S32 * T + (size_t)t0 * T);
-        const uint4 *src = reinterpret_cast<const uint4 *>(vtile[gi & 1]);
-        for (int vi = tid; vi < nvec; vi += kPruneThreads) __stcs(dstg + vi, src[vi]);
-        ks = ks_next;
+        __syncwarp();
+        // kept index i of the warp's 8 tokens: 8 * sizeof(E) contiguous bytes
+        // of the interleaved layout, in 16-byte pieces
+        constexpr int kParts = (int)sizeof(E) / 2;  // 16-byte pieces per row
+        unsigned char *g = reinterpret_cast<unsigned char *>(gvals + (size_t)gi * 32 * T + warp * 8);
+        const unsigned char *src = reinterpret_cast<const unsigned char *>(vt);
+        for (int c = lane; c < T * kParts; c += 32) {
+            const int row = c / kParts, part = c % kParts;
+            __stcs(reinterpret_cast<uint4 *>(g + (size_t)row * 32 * sizeof(E) + part * 16),
+                   *reinterpret_cast<const uint4 *>(src + row * 8 * sizeof(E) + part * 16));
+        }
+        __syncwarp();
+    };
+
+    KSlice<E> ka, kb;
+    if (g_first * 32 + tl < S) ka.load(krow);
+    else ka.zero();
+    for (int gi = 0; gi < kPruneGroups; gi += 2) {
+        if ((g_first + gi) * 32 >= S) break;  // uniform across the CTA
+        group(gi, ka, kb);
+        if ((g_first + gi + 1) * 32 >= S) break;
+        group(gi + 1, kb, ka);
     }
 
     // fixed-order reduction: xor tree inside each warp, then warps in order
