@@ -17,19 +17,27 @@
 // decode_kernel: a persistent grid, one CTA per SM, whose warps are
 // independent flash-decoding workers.  Work items are (row, kv head, chunk of
 // prompt tokens) plus one dense-tail item per head; warp w of the grid takes
-// items w, w + #warps, ...  Each warp streams its items' 32-token tiles: the
-// mask (16 B/token) and one 32-token group of interleaved kept values
-// (T*es B/token) by cp.async.bulk copies, issued by its lane 0 into its own
-// ring of shared-memory stages and completed on per-stage mbarriers (bounded
-// waits); the dense V rows (256 B/token) by coalesced 8-byte loads straight
-// into registers, issued before the tile's q.k~ so that they land under it.
-// No CTA-wide barrier is on the path.  Per tile:
+// items w, w + #warps, ... (prompt items first, warps numbered CTA-fastest).
+// Each warp streams its items' 32-token tiles: the mask (16 B/token) and one
+// 32-token group of interleaved kept values (T*es B/token) by cp.async.bulk
+// copies, issued by its lane 0 into its own ring of shared-memory stages and
+// completed on per-stage mbarriers (bounded waits).  The dense V rows
+// (256 B/token) are issued before the tile's q.k~ so that they land under it:
+// for bf16 by cp.async into an XOR-swizzled per-warp tile, for fp32 by
+// coalesced 8-byte loads into registers.  No CTA-wide barrier is on the path.
+// Per tile:
 //   q.k~     lane = token; the lane walks exactly T set bits of its 128-bit
-//            mask and accumulates q'_g (k_j - c_j) for the G heads of the
-//            group from the q' / c tables (q' = q * log2(e)/sqrt(D));
+//            mask from the top channel down (a queue of the non-empty mask
+//            words, one bfind and one bit clear per step, no branch) and
+//            accumulates q'_g (k_j - c_j) for the G heads of the group from
+//            the q' / c tables (q' = q * log2(e)/sqrt(D));
 //   softmax  warp max (integer REDUX on an order-preserving map) updates the
-//            running max; p = 2^(s - m) goes to shared memory as fp32 pairs;
-//   P.V      lane = 4 value channels; packed fp32x2 FMAs over the tokens.
+//            running max; p = 2^(s - m) goes to shared memory;
+//   P.V      bf16: tensor cores -- the V tile is the B operand
+//            (ldmatrix.trans), p is the A operand split into bf16 hi + lo
+//            parts (two mma.sync m16n8k16 per tile, fp32 accumulators), so
+//            the products keep ~16 bits of p; fp32: lane = 4 value channels,
+//            packed fp32x2 FMAs over the tokens.
 // At the end of an item the warp writes (acc[G][D], m, l) for it;
 // combine_kernel merges a head's items in a fixed order.
 #include "spark_internal.cuh"

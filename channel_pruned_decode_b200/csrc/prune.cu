@@ -11,15 +11,20 @@
 //                  fp64 sum of squares over the G*W window rows of the group,
 //                  rounded once to fp32.
 //   prune_kernel   one CTA per 256-token chunk of one (row, kv head).  Four
-//                  lanes own one token (32 channels each, saliency keys kept in
-//                  registers); the T-th largest key is found by a quad-level
-//                  bisection on the fp32 bit pattern (w >= 0, so the bit
-//                  pattern is monotone in w), ties broken toward the lower
-//                  channel by an exclusive scan across the quad.  Kept values
-//                  are staged in shared memory in the 32-token interleaved
-//                  layout and written back with 16-byte stores; fp32 partial
-//                  sums of the pruned saliencies go to fp64 per-lane
-//                  accumulators and one fp64 partial per CTA.
+//                  lanes own one token (32 channels each): exact fp32 keys
+//                  w = qn_j * |k_j| in registers, plus 16-bit search keys
+//                  fp16(w * 2^-floor(log2 max qn)), two channels per word.
+//                  The fp16 threshold is found by binary lifting over a window
+//                  around a running estimate; each probe compares the keys
+//                  with packed fp16 compares and counts the results on the
+//                  tensor cores (mma.sync against an all-ones operand).  A
+//                  probe that leaves exactly T keys fixes the mask; otherwise
+//                  the exact fp32 keys are bisected inside the fp16 tie band
+//                  and remaining exact ties go to the lower channel by a scan
+//                  across the quad.  Kept values are staged per warp in the
+//                  32-token interleaved layout and written back with 16-byte
+//                  stores; fp32 partial sums of the pruned saliencies go to
+//                  fp64 per-lane accumulators and one fp64 partial per CTA.
 //   stats_kernel   fixed-order fp64 sum of the CTA partials per head, then
 //                  N = S*(D-T) and mu_pruned = sum w / N.
 // All reductions have a fixed order, so reruns are bit-identical.

@@ -434,9 +434,9 @@ void oracle_decode_f(const float *q, const uint32_t *mask, const float *vals, co
         oracle_recover_keys_f(mask, vals, qn, stats, bh, S, D, T, mode, seed, Kt);
         for (long t = 0; t < n_tail; ++t)
             for (int j = 0; j < D; ++j)
-                Kt[(S + t) * D + j] = (double)k_tail[(bh * tail_cap + t) * D + j];
+                Kt[(S + t) * D + j] = (double)k_tail[bh * tail_cap * (long)D + t * D + j];
         for (int g = 0; g < G; ++g) {
-            const float *qrow = q + (bh * G + g) * (long)D;
+            const float *qrow = &q[(bh * G + g) * (long)D];  /* query head g of kv head bh */
             float *orow = out + (bh * G + g) * (long)D;
             if (L == 0) {
                 for (int d = 0; d < D; ++d)

@@ -31,8 +31,8 @@ MUTANTS = {
     "mean_wrong_denominator": ("? sw / n : 0.0;", "? sw / (n + 1.0) : 0.0;"),
     "keeps_one_less": ("for (int r = 0; r < T; ++r)", "for (int r = 0; r < T - 1; ++r)"),
     "vals_reversed": ("vrow[pos++] = krow[j];", "vrow[T - 1 - pos++] = krow[j];"),
-    "score_scale_1_over_D": ("const double scale = 1.0 / sqrt((double)D);\n    for (long bh = 0; bh < BH; ++bh) {\n        oracle_recover_keys",
-                             "const double scale = 1.0 / (double)D;\n    for (long bh = 0; bh < BH; ++bh) {\n        oracle_recover_keys"),
+    "score_scale_1_over_D": ("const double scale = 1.0 / sqrt((double)D);\n    for (long bh = 0; bh < BH; ++bh) {\n        oracle_recover_keys(mask",
+                             "const double scale = 1.0 / (double)D;\n    for (long bh = 0; bh < BH; ++bh) {\n        oracle_recover_keys(mask"),
     # SnapKV pre-pass (readings R11-R13)
     "snapkv_normaliser_not_causal": ("for (long t = 0; t <= p; ++t)\n                    l += exp(logit[t] - m);",
                                      "for (long t = 0; t < S; ++t)\n                    l += exp(logit[t] - m);"),
