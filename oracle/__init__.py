@@ -74,6 +74,12 @@ def _bind(lib):
     lib.oracle_snapkv_pool.restype = None
     lib.oracle_snapkv_select.argtypes = [P, L, L, I, I, P]
     lib.oracle_snapkv_select.restype = None
+    lib.oracle_group_of_channel.argtypes = [P, L, I, I, P]
+    lib.oracle_group_of_channel.restype = None
+    lib.oracle_group_budget.argtypes = [I, I, P, P]
+    lib.oracle_group_budget.restype = None
+    lib.oracle_prune_grouped.argtypes = [P, P, L, L, I, I, P, P, P, P]
+    lib.oracle_prune_grouped.restype = None
     return lib
 
 
@@ -120,6 +126,48 @@ def prune(k, qn, T: int, lib=None):
     vals = np.zeros((BH, S, T), np.float32)
     stats = np.zeros((BH, 4), np.float64)
     lib.oracle_prune(_ptr(k), _ptr(qn), BH, S, D, T, _ptr(mask), _ptr(vals), _ptr(stats))
+    return mask, vals, stats
+
+
+def group_of_channel(qn, g: int, lib=None) -> np.ndarray:
+    """SparK-g channel groups by window-query norm rank (reading R15).
+    qn: [BH, D] -> gid [BH, D] int32."""
+    lib = lib or load()
+    qn = _f32(qn)
+    D = qn.shape[-1]
+    BH = qn.size // D
+    gid = np.zeros((BH, D), np.int32)
+    lib.oracle_group_of_channel(_ptr(qn), BH, D, g, _ptr(gid))
+    return gid
+
+
+def group_budget(D: int, rates, lib=None) -> list:
+    """Per-group kept-channel budgets from pruning rates (reading R15)."""
+    lib = lib or load()
+    r = _f32(rates)
+    Tg = np.zeros(len(r), np.int32)
+    lib.oracle_group_budget(D, len(r), _ptr(r), _ptr(Tg))
+    return [int(x) for x in Tg]
+
+
+def prune_grouped(k, qn, Tg, lib=None):
+    """SparK-g pruning (reading R15).  k: [BH, S, D]; qn: [BH, D]; Tg: one
+    kept-channel budget per group.  Returns (mask, vals [BH, S, sum Tg],
+    stats) in the layouts of prune()."""
+    lib = lib or load()
+    k = _f32(k)
+    qn = _f32(qn)
+    D = k.shape[-1]
+    S = k.shape[-2]
+    BH = k.size // (S * D) if S > 0 else qn.size // D
+    tg = np.ascontiguousarray(Tg, np.int32)
+    T = int(tg.sum())
+    nw = (D + 31) // 32
+    mask = np.zeros((BH, S, nw), np.uint32)
+    vals = np.zeros((BH, S, T), np.float32)
+    stats = np.zeros((BH, 4), np.float64)
+    lib.oracle_prune_grouped(_ptr(k), _ptr(qn), BH, S, D, len(tg), _ptr(tg), _ptr(mask), _ptr(vals),
+                             _ptr(stats))
     return mask, vals, stats
 
 

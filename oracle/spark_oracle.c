@@ -151,6 +151,126 @@ void oracle_prune(const float *k, const float *qn, long BH, long S, int D,
     free(w);
 }
 
+/*
+ * SparK-g ([W] 5.2): channels are split into g groups by importance and each
+ * group has its own pruning rate, low-importance groups pruned harder
+ * (g = 4 with rates (0.25, 0.5, 0.75, 1.0) in [W]).  Reading R15 (the pages
+ * do not say what "importance" is or how large the groups are):
+ *   - the importance of channel j of a head is its window-query norm qn_j,
+ *     the query factor of the saliency, fixed for the head; channels ordered
+ *     by (qn desc, j asc) are cut into g consecutive groups, group k holding
+ *     the ranks [k*D/g, (k+1)*D/g) (integer division);
+ *   - group k keeps Tg[k] = round((1 - rate_k) * |group k|) channels per
+ *     token (half away from zero, as R7): its Tg[k] channels of largest
+ *     saliency, ties to the lower channel, i.e. the greedy solution of the
+ *     relaxed objective of [W] 3.1 with one budget per group;
+ *   - the cache is the plain one with T = sum_k Tg[k] (mask, kept values in
+ *     ascending channel order, statistics over the pruned entries).
+ * With equal-size groups the mean pruning rate is the mean of the rates
+ * (0.625 for [W]'s g = 4 rates); [W] reports 0.44, which equal groups cannot
+ * give, so the group sizes of the original are not those of this reading.
+ */
+typedef struct {
+    float q;
+    int j;
+} chan_norm;
+
+static int by_norm_desc(const void *pa, const void *pb)
+{
+    const chan_norm *a = (const chan_norm *)pa, *b = (const chan_norm *)pb;
+    if (a->q > b->q) return -1;
+    if (a->q < b->q) return 1;
+    return a->j < b->j ? -1 : (a->j > b->j);  /* equal norms: lower channel first */
+}
+
+/* gid [BH][D]: group of every channel (R15). */
+void oracle_group_of_channel(const float *qn, long BH, int D, int g, int *gid)
+{
+    chan_norm *ord = (chan_norm *)malloc(sizeof(chan_norm) * (size_t)D);
+    for (long bh = 0; bh < BH; ++bh) {
+        for (int j = 0; j < D; ++j) {
+            ord[j].q = qn[bh * D + j];
+            ord[j].j = j;
+        }
+        qsort(ord, (size_t)D, sizeof(chan_norm), by_norm_desc);
+        for (int k = 0; k < g; ++k)
+            for (int r = k * D / g; r < (k + 1) * D / g; ++r)
+                gid[bh * D + ord[r].j] = k;
+    }
+    free(ord);
+}
+
+/* Per-group budgets Tg[k] from pruning rates (R15). */
+void oracle_group_budget(int D, int g, const float *rates, int *Tg)
+{
+    for (int k = 0; k < g; ++k) {
+        const int size = (k + 1) * D / g - k * D / g;
+        Tg[k] = (int)llround((1.0 - (double)rates[k]) * (double)size);
+    }
+}
+
+/* SparK-g pruning (R15): per token and group, the group's Tg[k] largest
+ * saliencies; packing and statistics as in oracle_prune with T = sum Tg. */
+void oracle_prune_grouped(const float *k, const float *qn, long BH, long S, int D, int g, const int *Tg,
+                          uint32_t *mask, float *vals, double *stats)
+{
+    const int nw = (D + 31) / 32;
+    int T = 0;
+    for (int q = 0; q < g; ++q)
+        T += Tg[q];
+    int *gid = (int *)malloc(sizeof(int) * (size_t)(BH > 0 ? BH : 1) * (size_t)D);
+    oracle_group_of_channel(qn, BH, D, g, gid);
+    chan_score *order = (chan_score *)malloc(sizeof(chan_score) * (size_t)D);
+    unsigned char *keep = (unsigned char *)malloc((size_t)D);
+    float *w = (float *)malloc(sizeof(float) * (size_t)D);
+    for (long bh = 0; bh < BH; ++bh) {
+        double n = 0.0, sw = 0.0, sw2 = 0.0;
+        for (long t = 0; t < S; ++t) {
+            const float *krow = k + (bh * S + t) * D;
+            for (int j = 0; j < D; ++j)
+                w[j] = saliency(qn[bh * D + j], krow[j]);
+            memset(keep, 0, (size_t)D);
+            for (int grp = 0; grp < g; ++grp) {
+                int m = 0;
+                for (int j = 0; j < D; ++j)
+                    if (gid[bh * D + j] == grp) {
+                        order[m].w = w[j];
+                        order[m].j = j;
+                        ++m;
+                    }
+                qsort(order, (size_t)m, sizeof(chan_score), by_saliency_desc);
+                for (int r = 0; r < Tg[grp] && r < m; ++r)
+                    keep[order[r].j] = 1;
+            }
+            uint32_t *mrow = mask + (bh * S + t) * nw;
+            for (int q = 0; q < nw; ++q)
+                mrow[q] = 0u;
+            float *vrow = vals + (bh * S + t) * (long)T;
+            int pos = 0;
+            for (int j = 0; j < D; ++j) {
+                if (keep[j]) {
+                    mrow[j / 32] |= 1u << (j % 32);
+                    vrow[pos] = krow[j];
+                    ++pos;
+                } else {
+                    const double x = (double)w[j];
+                    n += 1.0;
+                    sw += x;
+                    sw2 += x * x;
+                }
+            }
+        }
+        stats[bh * 4 + 0] = n;
+        stats[bh * 4 + 1] = sw;
+        stats[bh * 4 + 2] = sw2;
+        stats[bh * 4 + 3] = n > 0.0 ? (sw / n) : 0.0;
+    }
+    free(gid);
+    free(order);
+    free(keep);
+    free(w);
+}
+
 /* Recovery F = Degenerate, [W] 3.3 steps 2-4 and the F table: the sampled
  * score is mu_pruned, and the key is back-solved from it as
  * k~ = w~ / ||q^j||_2 (R5).  Kept channels are the stored key values.

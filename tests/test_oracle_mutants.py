@@ -14,7 +14,8 @@ import oracle
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_snapkv_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_sampling_pins.py")]
+        os.path.join(ROOT, "tests", "test_oracle_sampling_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_group_pins.py")]
 
 MUTANTS = {
     "tie_rule_reversed": ("return (a->j > b->j) - (a->j < b->j);",
@@ -54,6 +55,17 @@ MUTANTS = {
                        "const float *qrow = q + ((long)g * BH + bh) * (long)D;"),
     "tail_keys_from_values": ("(double)k_tail[(bh * tail_cap + t) * D + j];",
                               "(double)v_tail[(bh * tail_cap + t) * D + j];"),
+    # SparK-g (reading R15)
+    "group_order_ascending": ("if (a->q > b->q) return -1;\n    if (a->q < b->q) return 1;",
+                              "if (a->q < b->q) return -1;\n    if (a->q > b->q) return 1;"),
+    "group_norm_ties_reversed": ("return a->j < b->j ? -1 : (a->j > b->j);",
+                                 "return a->j > b->j ? -1 : (a->j < b->j);"),
+    "group_budget_truncates": ("Tg[k] = (int)llround((1.0 - (double)rates[k]) * (double)size);",
+                               "Tg[k] = (int)((1.0 - (double)rates[k]) * (double)size);"),
+    "group_budget_of_whole_head": ("Tg[k] = (int)llround((1.0 - (double)rates[k]) * (double)size);",
+                                   "Tg[k] = (int)llround((1.0 - (double)rates[k]) * (double)D / 4);"),
+    "group_keeps_one_less": ("for (int r = 0; r < Tg[grp] && r < m; ++r)",
+                             "for (int r = 0; r < Tg[grp] - 1 && r < m; ++r)"),
     "lambda_truncates": ("return (int)llround((1.0 - (double)lambda) * (double)D);",
                          "return (int)((1.0 - (double)lambda) * (double)D);"),
 }
