@@ -10,6 +10,7 @@ import ctypes
 import os
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspark.so")
@@ -30,7 +31,7 @@ SPARK_OP_DECODE = 1
 SPARK_OP_SNAPKV = 2
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
-           "spark_prune", "spark_prune_noalloc", "spark_decode_attn", "spark_tail_append", "spark_device_status",
+           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_decode_attn", "spark_tail_append", "spark_device_status",
            "spark_status_str", "spark_snapkv_evict")
 
 
@@ -70,6 +71,8 @@ def lib():
         L.spark_prune.restype = I
         L.spark_prune_noalloc.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P]
         L.spark_prune_noalloc.restype = I
+        L.spark_prune_grouped.argtypes = [P, P, I, I, I, ctypes.POINTER(I), ctypes.POINTER(spark_kcache), P, Z, P]
+        L.spark_prune_grouped.restype = I
         L.spark_decode_attn.argtypes = [P, ctypes.POINTER(spark_kcache), P, P, P, I, I, I, I,
                                         ctypes.c_ulonglong, P, P, Z, P]
         L.spark_decode_attn.restype = I
@@ -187,6 +190,29 @@ def spark_prune_noalloc(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, kc
     s = kc.struct()
     rc = lib().spark_prune_noalloc(_ptr(k), _ptr(q_obs), G, W, ctypes.byref(s), _stream(stream))
     _check(rc, "spark_prune_noalloc")
+
+
+def spark_prune_grouped(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, group_T, kc: KCache,
+                        ws: torch.Tensor, stream=None) -> None:
+    """SparK-g: per-group kept-channel budgets group_T (host list, one entry
+    per group, sum == kc.T); groups by window-query norm rank (see spark.h)."""
+    tg = (ctypes.c_int * len(group_T))(*[int(x) for x in group_T])
+    s = kc.struct()
+    rc = lib().spark_prune_grouped(_ptr(k), _ptr(q_obs), G, W, len(group_T), tg, ctypes.byref(s), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_prune_grouped")
+
+
+def spark_group_budget(D: int, rates) -> list:
+    """Per-group kept-channel budgets round((1 - rate) * group size), half
+    away from zero, for len(rates) equal-rank groups of D channels."""
+    g = len(rates)
+    out = []
+    for q, r in enumerate(rates):
+        size = (q + 1) * D // g - q * D // g
+        x = (1.0 - float(np.float32(r))) * size
+        out.append(int(np.floor(x + 0.5)) if x >= 0 else -int(np.floor(-x + 0.5)))
+    return out
 
 
 def spark_decode_attn(q: torch.Tensor, kc: KCache, v: torch.Tensor, k_tail, v_tail, tail_cap: int,

@@ -8,6 +8,8 @@
 namespace spark {
 cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const spark_kcache &kc,
                          void *ws, cudaStream_t st);
+cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups,
+                                 const int *group_T, const spark_kcache &kc, void *ws, cudaStream_t st);
 cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const void *k_tail,
                           const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
                           unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st);
@@ -124,6 +126,30 @@ int spark_prune(const void *k, const void *q_obs, int G, int W, const spark_kcac
     if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
     if (ws_bytes < prune_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
     cudaError_t e = launch_prune(k, q_obs, G, W, *out, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups, const int *group_T,
+                        const spark_kcache *out, void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_cache(out);
+    if (rc != SPARK_OK) return rc;
+    if (G < 1 || W < 1) return SPARK_ERR_ARG;
+    if (n_groups < 1 || n_groups > kMaxGroups || !group_T) return SPARK_ERR_ARG;
+    int sum = 0;
+    for (int q = 0; q < n_groups; ++q) {
+        const int size = (q + 1) * out->D / n_groups - q * out->D / n_groups;
+        if (group_T[q] < 0 || group_T[q] > size) return SPARK_ERR_ARG;
+        sum += group_T[q];
+    }
+    if (sum != out->T) return SPARK_ERR_ARG;
+    const long BH = (long)out->B * out->Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
+    if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < prune_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_prune_grouped(k, q_obs, G, W, n_groups, group_T, *out, workspace,
+                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 

@@ -159,10 +159,12 @@ __device__ __forceinline__ __half count_ge16(const uint32_t (&kp)[16], uint32_t 
     return __low2half(c);
 }
 
-__device__ __forceinline__ int quad_count32(const uint32_t (&key)[32], uint32_t mid) {
+// Number of the quad's keys >= mid among the channels of `gm` (bit i =
+// channel i of this lane's quarter takes part).
+__device__ __forceinline__ int quad_count32(const uint32_t (&key)[32], uint32_t mid, uint32_t gm) {
     int c = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) c += (key[i] >= mid) ? 1 : 0;
+    for (int i = 0; i < 32; ++i) c += (key[i] >= mid && ((gm >> i) & 1u)) ? 1 : 0;
     return quad_sum(c);
 }
 
@@ -191,10 +193,12 @@ constexpr int kLiftCold = 12;         // first token of a quad: 2^12 units (4 oc
 // range redoes the search.  Phase 2 bisects the exact fp32 keys inside the
 // band, and a scan over the quad settles exact ties.  Every loop has a
 // warp-uniform trip count (finished quads idle), so the quad shuffles and the
-// warp-wide tensor-core counts see the full warp.
+// warp-wide tensor-core counts see the full warp.  Only the channels of gm
+// take part (a SparK-g group; all ones otherwise): the caller sets the fp16
+// keys of the others negative, below every probe.
 __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
                                                  int s, float inv_scale, uint32_t base, int K, bool skip,
-                                                 uint32_t &tau) {
+                                                 uint32_t gm, uint32_t &tau) {
     const __half hT = __int2half_rn(T);
     uint32_t lo = base;
     bool exact = skip;  // lanes past the end of the keys take no part
@@ -254,7 +258,7 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     bool done2 = exact || (hi32 - lo32 <= 1u);
     while (__any_sync(0xffffffffu, !done2)) {
         const uint32_t mid32 = lo32 + ((hi32 - lo32) >> 1);
-        const int c = quad_count32(key, mid32);
+        const int c = quad_count32(key, mid32, gm);
         if (!done2) {
             if (c >= T) {
                 lo32 = mid32;
@@ -272,17 +276,18 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     uint32_t m32 = 0u;
 #pragma unroll
     for (int i = 0; i < 32; ++i) m32 |= (key[i] >= thr ? 1u : 0u) << i;
+    m32 &= gm;
     if (__any_sync(0xffffffffu, !exact32)) {  // warp-uniform: the scans below shuffle
         const int above = quad_sum(__popc(m32));
         int e = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) e += (key[i] == lo32) ? 1 : 0;
+        for (int i = 0; i < 32; ++i) e += (key[i] == lo32 && ((gm >> i) & 1u)) ? 1 : 0;
         int r = quad_excl_scan(e, s);
         if (!exact32) {
             const int need = T - above;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                if (key[i] == lo32) {
+                if (key[i] == lo32 && ((gm >> i) & 1u)) {
                     if (r < need) m32 |= 1u << i;
                     ++r;
                 }
@@ -292,10 +297,17 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     return exact ? m : m32;
 }
 
-template <typename E>
+// SparK-g groups: number of groups and each group's kept-channel budget.
+struct GroupArgs {
+    int n;
+    int T[kMaxGroups];
+};
+
+template <typename E, bool kGrouped>
 __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
-                 E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks) {
+                 E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks,
+                 GroupArgs ga) {
     using Raw = typename RawT<E>::type;
     // per-warp staging of the kept values: [kept index][8 tokens of the warp]
     __shared__ __align__(16) Raw vtile[kPruneThreads / 32][kD * 8];
@@ -336,6 +348,41 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
         }
     }
     const float2 scale2 = make_float2(scale, scale);
+
+    // SparK-g: channel groups by window-query norm rank (equal norms: lower
+    // channel first; group q holds ranks [q*D/n, (q+1)*D/n)).  Per group and
+    // quarter: the channel bit mask and the 16 select words that keep the
+    // group's halves of the packed 16-bit keys.
+    __shared__ uint8_t sgid[kGrouped ? kD : 1];
+    __shared__ uint32_t gmask[kGrouped ? kMaxGroups : 1][4];
+    __shared__ __align__(16) uint32_t gsel[kGrouped ? kMaxGroups : 1][4][16];
+    __shared__ int gT[kGrouped ? kMaxGroups : 1];
+    __shared__ uint32_t staus[kGrouped ? kMaxGroups : 1][kPruneThreads];  // per-lane estimates
+    if constexpr (kGrouped) {
+        const float qj = qs[(tid >> 5) * 36 + (tid & 31)];
+        int rank = 0;
+        for (int i = 0; i < kD; ++i) {
+            const float qi = qs[(i >> 5) * 36 + (i & 31)];
+            rank += (qi > qj || (qi == qj && i < tid)) ? 1 : 0;
+        }
+        int gq = 0;
+        for (int q = 1; q < ga.n; ++q) gq += rank >= q * kD / ga.n ? 1 : 0;
+        sgid[tid] = (uint8_t)gq;
+        if (tid < kMaxGroups) gT[tid] = tid < ga.n ? ga.T[tid] : 0;
+        __syncthreads();
+        for (int e = tid; e < ga.n * 64; e += kPruneThreads) {
+            const int q = e >> 6, qs4 = (e >> 4) & 3, i = e & 15;
+            gsel[q][qs4][i] = (sgid[32 * qs4 + i] == q ? 0x0000ffffu : 0u) |
+                              (sgid[32 * qs4 + i + 16] == q ? 0xffff0000u : 0u);
+        }
+        if (tid < ga.n * 4) {
+            const int q = tid >> 2, qs4 = tid & 3;
+            uint32_t b = 0u;
+            for (int c = 0; c < 32; ++c) b |= (sgid[32 * qs4 + c] == q ? 1u : 0u) << c;
+            gmask[q][qs4] = b;
+        }
+        __syncthreads();
+    }
 
     Raw *vt = vtile[warp];
     uint32_t tau = 1u;
@@ -384,31 +431,67 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
                 const __half2 h = __floats2half2_rn(a, b);
                 kp[i] = *reinterpret_cast<const uint32_t *>(&h);
             }
-            uint32_t base;
-            int K;
-            if (gi == 0) {
-                // first token of this quad: the window ends at its largest key
-                __half2 mx = *reinterpret_cast<const __half2 *>(&kp[0]);
+            // one top-Tq selection over the channels of gm, with its own
+            // running threshold estimate tq
+            auto select_with = [&](const uint32_t(&kq)[16], int Tq, uint32_t gm, uint32_t &tq) -> uint32_t {
+                uint32_t base;
+                int K;
+                if (gi == 0) {
+                    // first token of this quad: the window ends at its largest
+                    // key (negative keys of channels outside gm count as 0)
+                    __half2 mx = *reinterpret_cast<const __half2 *>(&kq[0]);
 #pragma unroll
-                for (int i = 1; i < 16; ++i) mx = __hmax2(mx, *reinterpret_cast<const __half2 *>(&kp[i]));
-                const uint32_t mb = *reinterpret_cast<const uint32_t *>(&mx);
-                uint32_t m16 = max(mb & 0xffffu, mb >> 16);
-                m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
-                m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
-                K = kLiftCold;
-                base = m16 > (1u << K) - 1u ? m16 - ((1u << K) - 1u) : 0u;
+                    for (int i = 1; i < 16; ++i) mx = __hmax2(mx, *reinterpret_cast<const __half2 *>(&kq[i]));
+                    const uint32_t mb = *reinterpret_cast<const uint32_t *>(&mx);
+                    const uint32_t l16 = mb & 0xffffu, h16 = mb >> 16;
+                    uint32_t m16 = max((l16 & 0x8000u) ? 0u : l16, (h16 & 0x8000u) ? 0u : h16);
+                    m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
+                    m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
+                    K = kLiftCold;
+                    base = m16 > (1u << K) - 1u ? m16 - ((1u << K) - 1u) : 0u;
+                } else {
+                    // later tokens: centred on the running threshold estimate
+                    K = kLift;
+                    base = tq > (1u << (K - 1)) ? tq - (1u << (K - 1)) : 0u;
+                }
+                base = min(base, kTop16 - (1u << K));
+                uint32_t lo;
+                uint32_t mm = select_top_t(key, kq, Tq, s, inv_scale, base, K, !valid, gm, lo);
+                mm = valid ? mm : 0u;
+                // next estimate: running mean of this quad's thresholds
+                tq = gi == 0 ? lo : (uint32_t)((int)tq + (((int)lo - (int)tq) >> 1));
+                tq = valid ? tq : 1u;
+                return mm;
+            };
+            if constexpr (!kGrouped) {
+                m = select_with(kp, T, 0xffffffffu, tau);
             } else {
-                // later tokens: centred on the running threshold estimate
-                K = kLift;
-                base = tau > (1u << (K - 1)) ? tau - (1u << (K - 1)) : 0u;
+                m = 0u;
+#pragma unroll 1
+                for (int q = 0; q < ga.n; ++q) {
+                    const int Tq = gT[q];
+                    const int sz = (q + 1) * kD / ga.n - q * kD / ga.n;
+                    const uint32_t gm = gmask[q][s];
+                    if (Tq <= 0) continue;  // uniform: kernel arguments
+                    if (Tq >= sz) {
+                        m |= gm;
+                        continue;
+                    }
+                    uint32_t kq[16];
+                    const uint4 *sel4 = reinterpret_cast<const uint4 *>(&gsel[q][s][0]);
+#pragma unroll
+                    for (int i4 = 0; i4 < 4; ++i4) {
+                        const uint4 v = sel4[i4];
+                        const uint32_t sv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)  // members keep their key, others -1.0
+                            kq[4 * i4 + e] = (kp[4 * i4 + e] & sv[e]) | (0xbc00bc00u & ~sv[e]);
+                    }
+                    uint32_t tq = staus[q][tid];
+                    m |= select_with(kq, Tq, gm, tq);
+                    staus[q][tid] = tq;
+                }
             }
-            base = min(base, kTop16 - (1u << K));
-            uint32_t lo;
-            m = select_top_t(key, kp, T, s, inv_scale, base, K, !valid, lo);
-            m = valid ? m : 0u;
-            // next estimate: running mean of this quad's thresholds
-            tau = gi == 0 ? lo : (uint32_t)((int)tau + (((int)lo - (int)tau) >> 1));
-            tau = valid ? tau : 1u;
         }
         if (valid) mask[((size_t)bh * S + t) * kMaskWords + s] = m;
 
@@ -506,16 +589,21 @@ __global__ void stats_kernel(const double *__restrict__ partial, int n_chunks, l
 
 template <typename E>
 static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W,
-                                  const spark_kcache &kc, void *ws, cudaStream_t st) {
+                                  const spark_kcache &kc, void *ws, cudaStream_t st, const GroupArgs *ga) {
     const long BH = (long)kc.B * kc.Hkv;
     if (BH == 0) return cudaSuccess;
     double *partial = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
     qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn);
     const int nch = prune_chunks(kc.S);
     if (nch > 0) {
-        prune_kernel<E><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
-            static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-            nch);
+        if (ga)
+            prune_kernel<E, true><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+                static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
+                nch, *ga);
+        else
+            prune_kernel<E, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+                static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
+                nch, GroupArgs{});
     }
     stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.S, kc.T, kc.stats);
     return cudaGetLastError();
@@ -523,8 +611,17 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
 
 cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const spark_kcache &kc,
                          void *ws, cudaStream_t st) {
-    if (kc.dtype == SPARK_BF16) return launch_prune_t<__nv_bfloat16>(k, q_obs, G, W, kc, ws, st);
-    return launch_prune_t<float>(k, q_obs, G, W, kc, ws, st);
+    if (kc.dtype == SPARK_BF16) return launch_prune_t<__nv_bfloat16>(k, q_obs, G, W, kc, ws, st, nullptr);
+    return launch_prune_t<float>(k, q_obs, G, W, kc, ws, st, nullptr);
+}
+
+cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups,
+                                 const int *group_T, const spark_kcache &kc, void *ws, cudaStream_t st) {
+    GroupArgs ga{};
+    ga.n = n_groups;
+    for (int q = 0; q < n_groups; ++q) ga.T[q] = group_T[q];
+    if (kc.dtype == SPARK_BF16) return launch_prune_t<__nv_bfloat16>(k, q_obs, G, W, kc, ws, st, &ga);
+    return launch_prune_t<float>(k, q_obs, G, W, kc, ws, st, &ga);
 }
 
 // ---------------------------------------------------------------------------

@@ -19,6 +19,7 @@ constexpr uint32_t kDevTimeout = 1u;  // status bit: a bounded wait ran out
 // ----------------------------------------------------------------- prune
 constexpr int kPruneThreads = 128;    // 4 lanes per token, 32 tokens per group
 constexpr int kPruneGroups = 8;       // 32-token groups per CTA (256 tokens)
+constexpr int kMaxGroups = 8;         // SparK-g channel groups
 
 inline int prune_chunks(int S) {
     const int per = 32 * kPruneGroups;

@@ -140,6 +140,28 @@ SPARK_API int spark_prune(const void *k, const void *q_obs, int G, int W,
                 void *stream);
 
 /*
+ * SparK-g grouped pruning ([W] 5.2: channels split into groups by
+ * importance, each group with its own pruning rate).  Same arguments, cache
+ * layout, statistics and workspace as spark_prune, plus
+ *   n_groups  g, 1 <= g <= 8
+ *   group_T   host array of g budgets: group q keeps group_T[q] channels per
+ *             token, 0 <= group_T[q] <= |group q|; the caller passes
+ *             out->T == sum_q group_T[q]
+ * Groups (the library's reading; the pages do not define importance or group
+ * sizes): the channels of a (b, h) ordered by (qn desc, channel asc) are cut
+ * into g consecutive runs, group q holding the ranks [q*D/g, (q+1)*D/g)
+ * (integer division).  Per token and group the group_T[q] channels of
+ * largest w are kept (ties -> lower channel).  The mask, the kept values
+ * (ascending channel order over all groups) and the statistics are those of
+ * spark_prune with T = sum group_T, so spark_decode_attn reads the cache
+ * unchanged.  With pruning rates r_q, group_T[q] = round((1 - r_q) * |group q|)
+ * (half away from zero).  Returns SPARK_ERR_ARG on bad budgets.
+ */
+SPARK_API int spark_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups,
+                                  const int *group_T, const spark_kcache *out, void *workspace,
+                                  size_t ws_bytes, void *stream);
+
+/*
  * spark_prune without a workspace.  Not part of the SparK method: the paper
  * has no counterpart; this is a calling convention for this library.
  *

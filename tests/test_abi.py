@@ -163,3 +163,26 @@ def test_snapkv_rejects_bad_args(L):
     assert f(keep=300) == B.SPARK_ERR_ARG             # keep > S
     assert f(pool=6) == B.SPARK_ERR_ARG               # even pool
     assert f() == B.SPARK_ERR_WORKSPACE               # no workspace
+
+
+def test_prune_grouped_rejects_bad_budgets(L):
+    # every call here must fail validation: the pointers are not real
+    kc = _kc()  # T = 32
+    I = ctypes.c_int
+    f = lambda tg, n=None, **k: L.spark_prune_grouped(
+        16, 16, k.get("G", 4), 32, len(tg) if n is None else n, (I * max(len(tg), 1))(*tg),
+        ctypes.byref(kc), k.get("ws", 256), 1 << 20, None)
+    assert f([10, 10, 5]) == B.SPARK_ERR_ARG             # sum 25 != T
+    assert f([33, 0, -1]) == B.SPARK_ERR_ARG             # negative budget
+    assert f([26, 0]) == B.SPARK_ERR_ARG                 # sum 26 != T
+    assert f([32], n=0) == B.SPARK_ERR_ARG               # no groups
+    assert f([4] * 8 + [0]) == B.SPARK_ERR_ARG           # more than 8 groups
+    assert f([16, 16], G=0) == B.SPARK_ERR_ARG
+    assert f([0] * 7 + [32]) == B.SPARK_ERR_ARG          # 32 > group size 16
+    assert L.spark_prune_grouped(16, 16, 4, 32, 2, None, ctypes.byref(kc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert f([16, 16], ws=None) == B.SPARK_ERR_WORKSPACE
+
+
+def test_group_budget_matches_oracle():
+    for rates in ([0.25, 0.5, 0.75, 1.0], [0.5] * 5, [0.1, 0.3, 0.5, 0.7, 0.9], [0.0] * 8, [1.0] * 3, [0.33] * 7):
+        assert B.spark_group_budget(128, rates) == oracle.group_budget(128, rates)
