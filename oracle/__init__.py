@@ -80,6 +80,8 @@ def _bind(lib):
     lib.oracle_group_budget.restype = None
     lib.oracle_prune_grouped.argtypes = [P, P, L, L, I, I, P, P, P, P]
     lib.oracle_prune_grouped.restype = None
+    lib.oracle_recover_values.argtypes = [P, P, L, L, I, I, P]
+    lib.oracle_recover_values.restype = None
     return lib
 
 
@@ -169,6 +171,43 @@ def prune_grouped(k, qn, Tg, lib=None):
     lib.oracle_prune_grouped(_ptr(k), _ptr(qn), BH, S, D, len(tg), _ptr(tg), _ptr(mask), _ptr(vals),
                              _ptr(stats))
     return mask, vals, stats
+
+
+def prune_values(v, Tv: int, lib=None):
+    """V-channel pruning (reading R16): top-T_v channels of |v| per token,
+    i.e. prune() with unit query norms.  v: [BH, S, D].  Returns
+    (vmask, vvals, stats) in the layouts of prune()."""
+    v = _f32(v)
+    D = v.shape[-1]
+    BH = v.size // (v.shape[-2] * D) if v.shape[-2] > 0 else 0
+    return prune(v, np.ones((BH, D), np.float32), Tv, lib=lib)
+
+
+def recover_values(vmask, vvals, bh: int, lib=None) -> np.ndarray:
+    """Dense recovered value block V^ [S, D] (fp64) of one (b, h): kept
+    values, 0 on pruned channels (reading R16)."""
+    lib = lib or load()
+    vmask = np.ascontiguousarray(vmask, np.uint32)
+    vvals = _f32(vvals)
+    S = vmask.shape[-2]
+    D = vmask.shape[-1] * 32
+    Tv = vvals.shape[-1]
+    out = np.zeros((S, D), np.float64)
+    lib.oracle_recover_values(_ptr(vmask), _ptr(vvals), bh, S, D, Tv, _ptr(out))
+    return out
+
+
+def decode_kv(q, mask, vals, qn, stats, vmask, vvals, k_tail=None, v_tail=None, n_tail: int = 0, G: int = 1,
+              lib=None) -> np.ndarray:
+    """Decode over a pruned key cache and a pruned value cache: the value
+    rows are the recovered V^ of recover_values (R16), then decode()."""
+    vmask = np.ascontiguousarray(vmask, np.uint32)
+    BH, S = vmask.shape[0], vmask.shape[1]
+    D = vmask.shape[-1] * 32
+    vhat = np.zeros((BH, S, D), np.float32)
+    for bh in range(BH):
+        vhat[bh] = recover_values(vmask, vvals, bh, lib=lib).astype(np.float32)  # exact: kept values are fp32
+    return decode(q, mask, vals, qn, stats, vhat, k_tail, v_tail, n_tail, G, lib=lib)
 
 
 def recover_keys(mask, vals, qn, stats, bh: int, lib=None) -> np.ndarray:

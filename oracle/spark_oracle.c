@@ -271,6 +271,30 @@ void oracle_prune_grouped(const float *k, const float *qn, long BH, long S, int 
     free(w);
 }
 
+/*
+ * V-channel pruning ([W] 4.4: the value cache is pruned too, with a
+ * norm-based heuristic; SparK(0.5+0.5) prunes half of the key and half of
+ * the value channels).  Reading R16 (the pages name only "norm-based"): the
+ * saliency of value channel j of token t is its magnitude |v_t^j| -- the
+ * key rule of [W] 3.1 with the query factor set to 1, since a value channel
+ * meets no query -- so pruning is oracle_prune(v, qn = 1, T_v): top-T_v per
+ * token, ties to the lower channel, the same mask and packing.  A pruned
+ * value entry is recovered as 0 (dropped); the statistics over the pruned
+ * entries are computed but unused.  This writes the dense recovered value
+ * block Vt [S][D] (fp64) of one (b, h).
+ */
+void oracle_recover_values(const uint32_t *vmask, const float *vvals, long bh, long S, int D, int Tv, double *Vt)
+{
+    const int nw = (D + 31) / 32;
+    for (long t = 0; t < S; ++t) {
+        const uint32_t *mrow = vmask + (bh * S + t) * nw;
+        const float *vrow = vvals + (bh * S + t) * (long)Tv;
+        int pos = 0;
+        for (int j = 0; j < D; ++j)
+            Vt[t * D + j] = ((mrow[j / 32] >> (j % 32)) & 1u) ? (double)vrow[pos++] : 0.0;
+    }
+}
+
 /* Recovery F = Degenerate, [W] 3.3 steps 2-4 and the F table: the sampled
  * score is mu_pruned, and the key is back-solved from it as
  * k~ = w~ / ||q^j||_2 (R5).  Kept channels are the stored key values.

@@ -15,7 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_snapkv_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_sampling_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_group_pins.py")]
+        os.path.join(ROOT, "tests", "test_oracle_group_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_vprune_pins.py")]
 
 MUTANTS = {
     "tie_rule_reversed": ("return (a->j > b->j) - (a->j < b->j);",
@@ -66,6 +67,9 @@ MUTANTS = {
                                    "Tg[k] = (int)llround((1.0 - (double)rates[k]) * (double)D / 4);"),
     "group_keeps_one_less": ("for (int r = 0; r < Tg[grp] && r < m; ++r)",
                              "for (int r = 0; r < Tg[grp] - 1 && r < m; ++r)"),
+    # V-channel pruning (reading R16)
+    "values_pruned_not_dropped": ("? (double)vrow[pos++] : 0.0;", "? (double)vrow[pos++] : 1e-3;"),
+    "values_index_not_advanced": ("? (double)vrow[pos++] : 0.0;", "? (double)vrow[pos] : 0.0;"),
     "lambda_truncates": ("return (int)llround((1.0 - (double)lambda) * (double)D);",
                          "return (int)((1.0 - (double)lambda) * (double)D);"),
 }
