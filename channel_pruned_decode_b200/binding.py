@@ -31,7 +31,8 @@ SPARK_OP_DECODE = 1
 SPARK_OP_SNAPKV = 2
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
-           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_decode_attn", "spark_tail_append", "spark_device_status",
+           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_prune_values", "spark_decode_attn",
+           "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_tail_append", "spark_device_status",
            "spark_status_str", "spark_snapkv_evict")
 
 
@@ -73,6 +74,13 @@ def lib():
         L.spark_prune_noalloc.restype = I
         L.spark_prune_grouped.argtypes = [P, P, I, I, I, ctypes.POINTER(I), ctypes.POINTER(spark_kcache), P, Z, P]
         L.spark_prune_grouped.restype = I
+        L.spark_prune_values.argtypes = [P, ctypes.POINTER(spark_kcache), P, Z, P]
+        L.spark_prune_values.restype = I
+        L.spark_decode_attn_kv.argtypes = [P, ctypes.POINTER(spark_kcache), ctypes.POINTER(spark_kcache), P, P, I,
+                                           I, I, P, P, Z, P]
+        L.spark_decode_attn_kv.restype = I
+        L.spark_workspace_bytes_kv.argtypes = [I, I, I, I, I, I, I, I]
+        L.spark_workspace_bytes_kv.restype = Z
         L.spark_decode_attn.argtypes = [P, ctypes.POINTER(spark_kcache), P, P, P, I, I, I, I,
                                         ctypes.c_ulonglong, P, P, Z, P]
         L.spark_decode_attn.restype = I
@@ -201,6 +209,27 @@ def spark_prune_grouped(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, gr
     rc = lib().spark_prune_grouped(_ptr(k), _ptr(q_obs), G, W, len(group_T), tg, ctypes.byref(s), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_prune_grouped")
+
+
+def spark_prune_values(v: torch.Tensor, vc: KCache, ws: torch.Tensor, stream=None) -> None:
+    """Value-channel pruning: top-vc.T channels of |v| per token (see spark.h)."""
+    s = vc.struct()
+    rc = lib().spark_prune_values(_ptr(v), ctypes.byref(s), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream))
+    _check(rc, "spark_prune_values")
+
+
+def spark_decode_attn_kv(q: torch.Tensor, kc: KCache, vc: KCache, k_tail, v_tail, tail_cap: int, n_tail: int,
+                         G: int, out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    sk, sv = kc.struct(), vc.struct()
+    rc = lib().spark_decode_attn_kv(_ptr(q), ctypes.byref(sk), ctypes.byref(sv), _ptr(k_tail), _ptr(v_tail),
+                                    tail_cap, n_tail, G, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                    _stream(stream))
+    _check(rc, "spark_decode_attn_kv")
+
+
+def spark_workspace_bytes_kv(B: int, Hkv: int, G: int, S: int, D: int, T: int, Tv: int, n_tail: int) -> int:
+    return int(lib().spark_workspace_bytes_kv(B, Hkv, G, S, D, T, Tv, n_tail))
 
 
 def spark_group_budget(D: int, rates) -> list:

@@ -10,9 +10,10 @@ cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const s
                          void *ws, cudaStream_t st);
 cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups,
                                  const int *group_T, const spark_kcache &kc, void *ws, cudaStream_t st);
-cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const void *k_tail,
-                          const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
+cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const spark_kcache *vc,
+                          const void *k_tail, const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
                           unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st);
+cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws, cudaStream_t st);
 cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
                           int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st);
 
@@ -106,8 +107,8 @@ size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D, int T,
         if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
         // the geometry depends on the element size only through the stage
         // size; take the larger of the two so one workspace serves both
-        const DecodeGeom g2 = decode_geometry(BH, S, T, 2, G, num_sms());
-        const DecodeGeom g4 = decode_geometry(BH, S, T, 4, G, num_sms());
+        const DecodeGeom g2 = decode_geometry(BH, S, T, -1, 2, G, num_sms());
+        const DecodeGeom g4 = decode_geometry(BH, S, T, -1, 4, G, num_sms());
         const size_t a = decode_workspace(BH, g2, G), b = decode_workspace(BH, g4, G);
         return round256(a > b ? a : b);
     }
@@ -171,11 +172,55 @@ int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, cons
         return SPARK_ERR_ARG;
     if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
     const int es = elem_size(kc->dtype);
-    const DecodeGeom geo = decode_geometry(BH, kc->S, kc->T, es, G, num_sms());
+    const DecodeGeom geo = decode_geometry(BH, kc->S, kc->T, -1, es, G, num_sms());
     if (BH * (long)geo.units >= (1L << 31)) return SPARK_ERR_UNSUPPORTED;  // 32-bit item indices
     if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
-    cudaError_t e = launch_decode(q, *kc, v, k_tail, v_tail, tail_cap, n_tail, G, recovery, seed, out, workspace,
-                                  geo, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_decode(q, *kc, v, nullptr, k_tail, v_tail, tail_cap, n_tail, G, recovery, seed, out,
+                                  workspace, geo, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+size_t spark_workspace_bytes_kv(int B, int Hkv, int G, int S, int D, int T, int Tv, int n_tail) {
+    if (B < 0 || Hkv < 0 || S < 0 || D != kD || T < 0 || T > D || Tv < 0 || Tv > D || n_tail < 0) return 0;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
+    const DecodeGeom g = decode_geometry((long)B * Hkv, S, T, Tv, 2, G, num_sms());
+    return round256(decode_workspace((long)B * Hkv, g, G));
+}
+
+int spark_prune_values(const void *v, const spark_kcache *out, void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_cache(out);
+    if (rc != SPARK_OK) return rc;
+    const long BH = (long)out->B * out->Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (out->S > 0 && (!v || !aligned16(v))) return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < prune_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_prune_values(v, *out, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_decode_attn_kv(const void *q, const spark_kcache *kc, const spark_kcache *vc, const void *k_tail,
+                         const void *v_tail, int tail_cap, int n_tail, int G, float *out, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    int rc = check_cache(kc);
+    if (rc != SPARK_OK) return rc;
+    rc = check_cache(vc);
+    if (rc != SPARK_OK) return rc;
+    if (kc->B != vc->B || kc->Hkv != vc->Hkv || kc->S != vc->S || kc->dtype != vc->dtype) return SPARK_ERR_ARG;
+    if (kc->dtype != SPARK_BF16) return SPARK_ERR_UNSUPPORTED;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return G < 1 ? SPARK_ERR_ARG : SPARK_ERR_UNSUPPORTED;
+    if (tail_cap < 0 || n_tail < 0 || n_tail > tail_cap) return SPARK_ERR_ARG;
+    const long BH = (long)kc->B * kc->Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!q || !aligned16(q) || !out || !aligned16(out)) return SPARK_ERR_ARG;
+    if (tail_cap > 0 && (!k_tail || !v_tail || !aligned16(k_tail) || !aligned16(v_tail)))
+        return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    const DecodeGeom geo = decode_geometry(BH, kc->S, kc->T, vc->T, 2, G, num_sms());
+    if (BH * (long)geo.units >= (1L << 31)) return SPARK_ERR_UNSUPPORTED;
+    if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_decode(q, *kc, nullptr, vc, k_tail, v_tail, tail_cap, n_tail, G, SPARK_F_DEGENERATE, 0,
+                                  out, workspace, geo, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 

@@ -50,6 +50,9 @@ struct DecArgs {
     const void *q;
     const uint32_t *mask;
     const void *vals;
+    const uint32_t *vmask;  // pruned value cache (packed-V kernels only)
+    const void *vvals;
+    int Tv;
     const float *qn;
     const double *stats;
     const void *v;
@@ -237,9 +240,15 @@ struct WarpSmem {
     float *pdup;   // [kWT][G][2] p duplicated into fp32 pairs (CUDA-core P.V)
     float *qc;     // [G] Qc = sum_j q'_j c_j of the current head
     uint64_t *bars;
-    uint8_t *lst;  // [T][kWT] kept channel indices of the tile's tokens
     unsigned char *stages;
     uint32_t stage_bytes;
+    uint32_t vstage_off;  // offset of the value cache's part of a stage
+    __device__ __forceinline__ const uint32_t *svmask(int st) const {
+        return reinterpret_cast<const uint32_t *>(stages + (size_t)st * stage_bytes + vstage_off);
+    }
+    __device__ __forceinline__ const E *svvals(int st) const {
+        return reinterpret_cast<const E *>(stages + (size_t)st * stage_bytes + vstage_off + kWT * 16);
+    }
     __device__ __forceinline__ const uint32_t *smask(int st) const {
         return reinterpret_cast<const uint32_t *>(stages + (size_t)st * stage_bytes);
     }
@@ -502,8 +511,9 @@ __device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, 
 // spilling warps on the G = 4 workloads
 __host__ __device__ constexpr int dec_max_warps(int G) { return G > 2 ? 12 : kMaxWarps; }
 
-template <typename E, int G, int kF>
+template <typename E, int G, int kF, bool kPV>
 __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArgs a) {
+    static_assert(!kPV || (sizeof(E) == 2 && kF == SPARK_F_DEGENERATE), "packed values: bf16, Degenerate F");
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= a.nwarp) return;
@@ -519,9 +529,9 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         ws.pdup = ws.tabc + kD;
         ws.qc = ws.pdup + kWT * G * 2;
         ws.bars = reinterpret_cast<uint64_t *>(ws.qc + 16);
-        ws.lst = reinterpret_cast<uint8_t *>(ws.bars + kMaxStagesW);
-        ws.stages = base + dec_table_bytes(G, a.T, es);
-        ws.stage_bytes = (uint32_t)dec_stage_bytes(a.T, es);
+        ws.stages = base + dec_table_bytes(G, es);
+        ws.vstage_off = (uint32_t)dec_stage_bytes(a.T, es);
+        ws.stage_bytes = ws.vstage_off + (kPV ? (uint32_t)dec_stage_bytes(a.Tv, es) : 0u);
     }
     if (lane == 0) {
         for (int st = 0; st < a.nstage; ++st) mbar_init(smem_u32(ws.bars + st), 1);
@@ -580,9 +590,16 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         const uint32_t vb = (uint32_t)kWT * (uint32_t)a.T * (uint32_t)es;  // one whole 32-token group
         const uint32_t bar = smem_u32(ws.bars + st);
         unsigned char *dst = ws.stages + (size_t)st * ws.stage_bytes;
-        mbar_expect_tx(bar, mb + vb);
+        const uint32_t vvb = kPV ? (uint32_t)kWT * (uint32_t)a.Tv * (uint32_t)es : 0u;
+        mbar_expect_tx(bar, mb + vb + (kPV ? mb + vvb : 0u));
         bulk_g2s(smem_u32(dst), a.mask + ((size_t)bh * a.S + t0) * kMaskWords, mb, bar);
         if (vb) bulk_g2s(smem_u32(dst + kWT * 16), gvals + (size_t)bh * a.S32 * a.T + (size_t)t0 * a.T, vb, bar);
+        if constexpr (kPV) {
+            bulk_g2s(smem_u32(dst + ws.vstage_off), a.vmask + ((size_t)bh * a.S + t0) * kMaskWords, mb, bar);
+            if (vvb)
+                bulk_g2s(smem_u32(dst + ws.vstage_off + kWT * 16),
+                         static_cast<const E *>(a.vvals) + (size_t)bh * a.S32 * a.Tv + (size_t)t0 * a.Tv, vvb, bar);
+        }
     };
 
     Cursor ic{gw, 0, 0, 0, 0};
@@ -704,8 +721,8 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             const long t0 = t_item + (long)tile * kWT;
             const int n = (int)min((long)kWT, t_end - t0);
             // this tile's V rows start moving (registers or shared memory) under
-            // the q.k~ below
-            pv.begin(ws, vbase + (size_t)t0 * kD, n);
+            // the q.k~ below; a pruned value cache arrives with the stage
+            if constexpr (!kPV) pv.begin(ws, vbase + (size_t)t0 * kD, n);
 
             const int st = (int)(consumed % a.nstage);
             const uint32_t par = (uint32_t)((consumed / a.nstage) & 1);
@@ -774,6 +791,41 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }
             }
+            if constexpr (kPV) {
+                // expand the pruned values into the swizzled V tile: the warp
+                // zeroes the tile (512 contiguous bytes per store, no bank
+                // conflict), then each lane writes its token's kept values with
+                // the same top-down mask walk as q.k~ (pruned entries stay 0)
+                const uint32_t tile = smem_u32(ws.vt);
+#pragma unroll
+                for (int c = 0; c < kWT * kD * 2 / 512; ++c)
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(tile + 512u * c + 16u * lane),
+                                 "r"(0u)
+                                 : "memory");
+                __syncwarp();
+                if (valid && a.Tv > 0) {
+                    const uint4 mw = *reinterpret_cast<const uint4 *>(ws.svmask(st) + lane * kMaskWords);
+                    uint32_t cur = mw.w, n1 = mw.z, n2 = mw.y, n3 = mw.x;
+                    uint32_t bq = 0x00204060u;
+                    queue_nonempty(cur, n1, n2, n3, bq);
+                    const uint16_t *vp =
+                        reinterpret_cast<const uint16_t *>(ws.svvals(st)) + lane + (a.Tv - 1) * kWT;
+                    const uint32_t vrow = smem_u32(ws.vt);
+#pragma unroll 4
+                    for (int i = 0; i < a.Tv; ++i) {
+                        const uint32_t pos = bit_top(cur);
+                        const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
+                        cur ^= shl_clamped(1u, pos);
+                        const bool e = cur == 0u;
+                        cur = e ? n1 : cur;
+                        n1 = e ? n2 : n1;
+                        n2 = e ? n3 : n2;
+                        bq = e ? (bq >> 8) : bq;
+                        const uint32_t adr = vrow + vswz(lane, j >> 3) + 2u * (uint32_t)(j & 7);
+                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(adr), "h"(vp[-i * kWT]) : "memory");
+                    }
+                }
+            }
             // the stage is read: hand it to the tile nstage ahead
             __syncwarp();
             ++consumed;
@@ -832,10 +884,10 @@ __global__ void __launch_bounds__(kD) combine_kernel(const float *__restrict__ a
     out[row * kD + d] = (L > 0.f) ? o / L : 0.f;
 }
 
-DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms) {
+DecodeGeom decode_geometry(long BH, int S, int T, int Tv, int es, int G, int num_sms) {
     DecodeGeom g{};
-    const size_t stage = dec_stage_bytes(T, es);
-    const size_t table = dec_table_bytes(G, T, es);
+    const size_t stage = dec_stage_bytes(T, es) + (Tv >= 0 ? dec_stage_bytes(Tv, es) : 0);
+    const size_t table = dec_table_bytes(G, es);
     const size_t budget = 227 * 1024;
     const int max_w = dec_max_warps(G);
     auto warps_for = [&](int ns) {
@@ -877,7 +929,7 @@ DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms) {
     return g;
 }
 
-template <typename E, int G, int kF>
+template <typename E, int G, int kF, bool kPV>
 static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, float *out, cudaStream_t st) {
     DecArgs a = a0;
     a.chunk = geo.chunk;
@@ -886,7 +938,7 @@ static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, flo
     a.nstage = geo.nstage;
     a.nwarp = geo.nwarp;
     a.warp_bytes = geo.warp_bytes;
-    auto kern = decode_kernel<E, G, kF>;
+    auto kern = decode_kernel<E, G, kF, kPV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)geo.smem);
     if (e != cudaSuccess) return e;
     kern<<<geo.ctas, geo.nwarp * 32, geo.smem, st>>>(a);
@@ -894,13 +946,13 @@ static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, flo
     return cudaGetLastError();
 }
 
-template <typename E, int kF>
+template <typename E, int kF, bool kPV = false>
 static cudaError_t dispatch_g(const DecArgs &a, const DecodeGeom &geo, int G, float *out, cudaStream_t st) {
     switch (G) {
-    case 1: return launch_decode_t<E, 1, kF>(a, geo, out, st);
-    case 2: return launch_decode_t<E, 2, kF>(a, geo, out, st);
-    case 4: return launch_decode_t<E, 4, kF>(a, geo, out, st);
-    case 8: return launch_decode_t<E, 8, kF>(a, geo, out, st);
+    case 1: return launch_decode_t<E, 1, kF, kPV>(a, geo, out, st);
+    case 2: return launch_decode_t<E, 2, kF, kPV>(a, geo, out, st);
+    case 4: return launch_decode_t<E, 4, kF, kPV>(a, geo, out, st);
+    case 8: return launch_decode_t<E, 8, kF, kPV>(a, geo, out, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -916,8 +968,8 @@ static cudaError_t dispatch_f(const DecArgs &a, const DecodeGeom &geo, int G, in
     }
 }
 
-cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const void *k_tail,
-                          const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
+cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const spark_kcache *vc,
+                          const void *k_tail, const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
                           unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st) {
     const long BH = (long)kc.B * kc.Hkv;
     if (BH == 0) return cudaSuccess;
@@ -940,6 +992,12 @@ cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, 
     a.tail_cap = tail_cap;
     a.n_tail = n_tail;
     a.seed = seed;
+    if (vc) {  // pruned value cache: bf16, Degenerate F (checked by the caller)
+        a.vmask = vc->mask;
+        a.vvals = vc->vals;
+        a.Tv = vc->T;
+        return dispatch_g<__nv_bfloat16, SPARK_F_DEGENERATE, true>(a, geo, G, out, st);
+    }
     if (kc.dtype == SPARK_BF16) return dispatch_f<__nv_bfloat16>(a, geo, G, recovery, out, st);
     return dispatch_f<float>(a, geo, G, recovery, out, st);
 }

@@ -615,6 +615,30 @@ cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const s
     return launch_prune_t<float>(k, q_obs, G, W, kc, ws, st, nullptr);
 }
 
+__global__ void fill_ones_kernel(float *__restrict__ qn) { qn[(size_t)blockIdx.x * kD + threadIdx.x] = 1.f; }
+
+// Value-channel pruning: the key kernel with every channel norm 1, so the
+// saliency is |v| exactly (a multiply by 1 is exact).
+cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws, cudaStream_t st) {
+    const long BH = (long)vc.B * vc.Hkv;
+    if (BH == 0) return cudaSuccess;
+    fill_ones_kernel<<<(unsigned)BH, kD, 0, st>>>(vc.qn);
+    double *partial = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
+    const int nch = prune_chunks(vc.S);
+    if (nch > 0) {
+        if (vc.dtype == SPARK_BF16)
+            prune_kernel<__nv_bfloat16, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(v), vc.qn, vc.mask, static_cast<__nv_bfloat16 *>(vc.vals),
+                partial, vc.S, vc.T, nch, GroupArgs{});
+        else
+            prune_kernel<float, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+                static_cast<const float *>(v), vc.qn, vc.mask, static_cast<float *>(vc.vals), partial, vc.S, vc.T,
+                nch, GroupArgs{});
+    }
+    stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, vc.S, vc.T, vc.stats);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups,
                                  const int *group_T, const spark_kcache &kc, void *ws, cudaStream_t st) {
     GroupArgs ga{};

@@ -59,13 +59,15 @@ __host__ __device__ inline size_t dec_stage_bytes(int T, int es) {
 // [kWT][G][2] (fp32 values), Qc [16], mbarriers and the tile's kept-channel
 // lists [T][kWT] bytes; rounded to 128 bytes so that the stages start aligned.
 __host__ __device__ inline size_t dec_vtile_bytes(int es) { return es == 2 ? (size_t)kWT * kD * 2 : 0; }
-__host__ __device__ inline size_t dec_table_bytes(int G, int T, int es) {
+__host__ __device__ inline size_t dec_table_bytes(int G, int es) {
     const size_t b = dec_vtile_bytes(es) + (size_t)G * kWT * 4 + (size_t)kD * G * 4 + kD * 4 +
-                     (size_t)kWT * G * 8 + 64 + kMaxStagesW * 8 + (size_t)kWT * (T > 0 ? T : 1);
+                     (size_t)kWT * G * 8 + 64 + kMaxStagesW * 8;
     return (b + 127) / 128 * 128;
 }
 
-DecodeGeom decode_geometry(long BH, int S, int T, int es, int G, int num_sms);
+// Tv >= 0: the stage also carries a pruned value cache (mask + Tv values per
+// token); Tv < 0: values are read dense
+DecodeGeom decode_geometry(long BH, int S, int T, int Tv, int es, int G, int num_sms);
 
 // partials: acc [BH][units][G][D] fp32, then (m, l) [BH][units][G][2] fp32
 inline size_t decode_workspace(long BH, const DecodeGeom &g, int G) {

@@ -162,6 +162,39 @@ SPARK_API int spark_prune_grouped(const void *k, const void *q_obs, int G, int W
                                   size_t ws_bytes, void *stream);
 
 /*
+ * Value-channel pruning ([W] 4.4: the value cache is pruned too, with a
+ * norm-based heuristic).  The library's reading (the pages name only
+ * "norm-based"): the saliency of value channel j of token t is |v[t,j]|,
+ * i.e. spark_prune's rule with every channel norm set to 1; each token keeps
+ * its out->T value channels of largest |v| (ties -> lower channel).
+ *   v    [B][Hkv][S][D] dtype  values
+ *   out  a cache descriptor exactly as for spark_prune (out->T is the value
+ *        budget T_v = round((1 - lambda_v) * D)); mask and vals receive the
+ *        pruned value cache, qn is filled with 1.0, stats hold N, sum |v| and
+ *        sum v^2 over the pruned entries (unused by decode)
+ * Workspace: spark_workspace_bytes(SPARK_OP_PRUNE, ...).  Decode reads a
+ * pruned value entry as 0 (spark_decode_attn_kv).
+ */
+SPARK_API int spark_prune_values(const void *v, const spark_kcache *out, void *workspace, size_t ws_bytes,
+                                 void *stream);
+
+/*
+ * Decode attention over a pruned key cache kc and a pruned value cache vc
+ * (spark_prune_values), plus a dense tail: as spark_decode_attn with
+ * recovery F = Degenerate, except that the value row of a prompt token is
+ * its kept values with 0 on pruned channels.  kc and vc must have the same
+ * B, Hkv, S and dtype; bf16 only (SPARK_ERR_UNSUPPORTED for fp32).  Tail
+ * values are dense.  Workspace: spark_workspace_bytes_kv(...).
+ */
+SPARK_API int spark_decode_attn_kv(const void *q, const spark_kcache *kc, const spark_kcache *vc,
+                                   const void *k_tail, const void *v_tail, int tail_cap, int n_tail, int G,
+                                   float *out, void *workspace, size_t ws_bytes, void *stream);
+
+/* Workspace bytes of spark_decode_attn_kv for key budget T and value budget
+ * Tv (the tail capacity as n_tail); 0 on bad arguments. */
+SPARK_API size_t spark_workspace_bytes_kv(int B, int Hkv, int G, int S, int D, int T, int Tv, int n_tail);
+
+/*
  * spark_prune without a workspace.  Not part of the SparK method: the paper
  * has no counterpart; this is a calling convention for this library.
  *

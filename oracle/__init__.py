@@ -179,8 +179,8 @@ def prune_values(v, Tv: int, lib=None):
     (vmask, vvals, stats) in the layouts of prune()."""
     v = _f32(v)
     D = v.shape[-1]
-    BH = v.size // (v.shape[-2] * D) if v.shape[-2] > 0 else 0
-    return prune(v, np.ones((BH, D), np.float32), Tv, lib=lib)
+    BH = int(np.prod(v.shape[:-2]))
+    return prune(v.reshape(BH, v.shape[-2], D), np.ones((BH, D), np.float32), Tv, lib=lib)
 
 
 def recover_values(vmask, vvals, bh: int, lib=None) -> np.ndarray:

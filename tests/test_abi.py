@@ -186,3 +186,22 @@ def test_prune_grouped_rejects_bad_budgets(L):
 def test_group_budget_matches_oracle():
     for rates in ([0.25, 0.5, 0.75, 1.0], [0.5] * 5, [0.1, 0.3, 0.5, 0.7, 0.9], [0.0] * 8, [1.0] * 3, [0.33] * 7):
         assert B.spark_group_budget(128, rates) == oracle.group_budget(128, rates)
+
+
+def test_value_pruning_entry_points_reject_bad_args(L):
+    # every call here must fail validation: the pointers are not real
+    kc, vc = _kc(), _kc(T=64)
+    f = lambda k=kc, v=vc, **a: L.spark_decode_attn_kv(
+        a.get("q", 16), ctypes.byref(k), ctypes.byref(v), 16, 16, a.get("cap", 8), a.get("n", 0), a.get("G", 4),
+        a.get("out", 16), a.get("ws", 256), 1 << 20, None)
+    assert f(v=_kc(T=64, S=32)) == B.SPARK_ERR_ARG                      # shapes differ
+    assert f(k=_kc(dtype=B.SPARK_F32), v=_kc(T=64, dtype=B.SPARK_F32)) == B.SPARK_ERR_UNSUPPORTED
+    assert f(G=3) == B.SPARK_ERR_UNSUPPORTED
+    assert f(n=9) == B.SPARK_ERR_ARG
+    assert f(q=None) == B.SPARK_ERR_ARG
+    assert f(ws=None) == B.SPARK_ERR_WORKSPACE
+    assert L.spark_workspace_bytes_kv(1, 2, 4, 64, 128, 26, 129, 8) == 0
+    assert L.spark_workspace_bytes_kv(1, 2, 3, 64, 128, 26, 64, 8) == 0
+    assert L.spark_prune_values(16, ctypes.byref(_kc(T=129)), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert L.spark_prune_values(None, ctypes.byref(vc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert L.spark_prune_values(16, ctypes.byref(vc), None, 1 << 20, None) == B.SPARK_ERR_WORKSPACE
