@@ -312,6 +312,10 @@ def run_gpu(args):
     kernel_name = {"prune": "prune_kernel", "decode": "decode_kernel"}[dom]
     traffic = _traffic_record(kernel_name, wl.name)
 
+    variants = None
+    if not args.no_variants:
+        variants = run_variants(job, wl, stream, peak, peak_kind)
+
     e2e = None
     if not args.no_e2e:  # every rank: the e2e timing has its own barrier and max
         e2e = run_e2e(job, wl, min(args.steps, args.e2e_steps), dist_on, world)
@@ -345,11 +349,65 @@ def run_gpu(args):
                          "bytes_per_launch": bm[dom],
                          "timing": "CUDA events around the entry point on its stream "
                                    "(the two small kernels launched with it included)"},
+            "variants": variants,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": job.launches_per_step * args.steps,
         }
         print(json.dumps(line), flush=True)
     sd.finalize()
+
+
+def run_variants(job, wl, stream, peak, peak_kind, iters=5):
+    """Method variants on the same prompt, timed outside the step with CUDA
+    events on the launching stream: SparK-g grouped pruning with the pages'
+    g = 4 rates (0.25, 0.5, 0.75, 1.0), and value-channel pruning at
+    lambda_v = 0.5 with decode over the pruned key and value caches (bf16)."""
+    sp = job.sp
+    S = job.S_kept
+    k = job.k_ev if wl.keep else job.k
+    v = job.v_ev if wl.keep else job.v
+    es = 2 if wl.dtype == "bf16" else 4
+
+    def timed(f):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                f()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(iters):
+                f()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters * 1e3
+
+    out = {}
+    rates = [0.25, 0.5, 0.75, 1.0]
+    Tg = sp.spark_group_budget(wl.D, rates)
+    kg = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, sum(Tg), wl.torch_dtype, device=job.dev)
+    us = timed(lambda: sp.spark_prune_grouped(k, job.q_obs, wl.G, wl.W, Tg, kg, job.wsp, stream))
+    nbytes = wl.BH * S * (wl.D * es + 16 + sum(Tg) * es)
+    gbs = nbytes / (us / 1e6) / 1e9
+    out["spark_g"] = {"rates": rates, "group_T": Tg, "T": sum(Tg), "us_per_call": us, "gbs": gbs,
+                      f"frac_{peak_kind}": gbs / peak, "bytes_per_call": nbytes,
+                      "timing": "CUDA events around spark_prune_grouped on its stream, outside the step"}
+    del kg
+    if wl.dtype == "bf16":
+        Tv = sp.spark_lambda_to_T(0.5, wl.D)
+        vc = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, Tv, wl.torch_dtype, device=job.dev)
+        us_p = timed(lambda: sp.spark_prune_values(v, vc, job.wsp, stream))
+        wkv = sp.workspace(sp.spark_workspace_bytes_kv(wl.rows, wl.Hkv, wl.G, S, wl.D, job.T, Tv, 0), job.dev)
+        outb = torch.empty_like(job.out)
+        us_d = timed(lambda: sp.spark_decode_attn_kv(job.q, job.kc, vc, None, None, 0, 0, wl.G, outb, wkv,
+                                                     stream))
+        if sp.spark_device_status(wkv) != 0:
+            raise RuntimeError("device status after the value-pruned decode")
+        nb = wl.BH * S * (16 + job.T * es + 16 + Tv * es)
+        out["spark_v"] = {"lambda_k": wl.lam, "lambda_v": 0.5, "T": job.T, "Tv": Tv,
+                          "prune_values_us": us_p, "decode_us": us_d, "decode_bytes": nb,
+                          "decode_gbs": nb / (us_d / 1e6) / 1e9,
+                          "decode_token_heads_per_s": wl.BH * S / (us_d / 1e6),
+                          "timing": "CUDA events on the stream, outside the step; no tail"}
+    return out
 
 
 def run_e2e(job, wl, steps, dist_on, world):
@@ -459,6 +517,7 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip the SparK-g variant timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
