@@ -202,11 +202,13 @@ __device__ __forceinline__ uint32_t bit_top(uint32_t x) {
     return p;
 }
 
-// x << n with shift counts of 32 and above giving 0 (PTX shl clamps).
-__device__ __forceinline__ uint32_t shl_clamped(uint32_t x, uint32_t n) {
-    uint32_t r;
-    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
-    return r;
+// (1 << n) - 1: the bits below position n, all ones for n >= 32 (bmsk with
+// clamping), so `x & bit_mask_below(bit_top(x))` clears x's top bit and
+// leaves 0 at 0.
+__device__ __forceinline__ uint32_t bit_mask_below(uint32_t n) {
+    uint32_t m;
+    asm("bmsk.clamp.b32 %0, 0, %1;" : "=r"(m) : "r"(n));
+    return m;
 }
 
 // Stable compaction of the queue (q0, q1, q2, q3) so that its non-empty words
@@ -774,11 +776,14 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 uint32_t bq = 0x00204060u;  // bases 96, 64, 32, 0 from the low byte up
                 queue_nonempty(cur, n1, n2, n3, bq);
                 const E *vp = ws.svals(st) + lane + (a.T - 1) * kWT;
+                float2 s2[G / 2 > 0 ? G / 2 : 1];  // head pairs: packed fp32x2 FMAs
+#pragma unroll
+                for (int g = 0; g < (G / 2 > 0 ? G / 2 : 1); ++g) s2[g] = make_float2(0.f, 0.f);
 #pragma unroll 4
                 for (int i = 0; i < a.T; ++i) {
                     const uint32_t pos = bit_top(cur);        // 0xffffffff when cur == 0
                     const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
-                    cur ^= shl_clamped(1u, pos);
+                    cur &= bit_mask_below(pos);  // clear the top bit
                     const bool e = cur == 0u;
                     cur = e ? n1 : cur;
                     n1 = e ? n2 : n1;
@@ -787,8 +792,22 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     const float x = Elem<E>::to_f(vp[-i * kWT]) - ws.tabc[j];
                     QVec<G> qv;
                     qv.load(ws.tabq + j * G);
+                    if constexpr (G % 2 == 0) {
+                        const float2 x2 = make_float2(x, x);
 #pragma unroll
-                    for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
+                        for (int g = 0; g < G; g += 2)
+                            s2[g / 2] = __ffma2_rn(make_float2(qv.v[g], qv.v[g + 1]), x2, s2[g / 2]);
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
+                    }
+                }
+                if constexpr (G % 2 == 0) {
+#pragma unroll
+                    for (int g = 0; g < G; g += 2) {
+                        s[g] = s2[g / 2].x;
+                        s[g + 1] = s2[g / 2].y;
+                    }
                 }
             }
             if constexpr (kPV) {
@@ -815,7 +834,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     for (int i = 0; i < a.Tv; ++i) {
                         const uint32_t pos = bit_top(cur);
                         const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
-                        cur ^= shl_clamped(1u, pos);
+                        cur &= bit_mask_below(pos);
                         const bool e = cur == 0u;
                         cur = e ? n1 : cur;
                         n1 = e ? n2 : n1;
