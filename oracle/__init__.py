@@ -82,6 +82,8 @@ def _bind(lib):
     lib.oracle_prune_grouped.restype = None
     lib.oracle_recover_values.argtypes = [P, P, L, L, I, I, P]
     lib.oracle_recover_values.restype = None
+    lib.oracle_think_prune.argtypes = [P, P, L, L, I, I, P, P, P]
+    lib.oracle_think_prune.restype = None
     return lib
 
 
@@ -170,6 +172,24 @@ def prune_grouped(k, qn, Tg, lib=None):
     stats = np.zeros((BH, 4), np.float64)
     lib.oracle_prune_grouped(_ptr(k), _ptr(qn), BH, S, D, len(tg), _ptr(tg), _ptr(mask), _ptr(vals),
                              _ptr(stats))
+    return mask, vals, stats
+
+
+def think_prune(k, qn, T: int, lib=None):
+    """ThinK structured pruning (reading R18): one channel mask per (b, h),
+    channels ranked by qn_j * ||k^j||_2 over the tokens.  Returns (mask, vals,
+    stats) in the layouts of prune(); stats = {N, 0, 0, 0} (no recovery)."""
+    lib = lib or load()
+    k = _f32(k)
+    qn = _f32(qn)
+    D = k.shape[-1]
+    S = k.shape[-2]
+    BH = int(np.prod(k.shape[:-2]))
+    nw = (D + 31) // 32
+    mask = np.zeros((BH, S, nw), np.uint32)
+    vals = np.zeros((BH, S, T), np.float32)
+    stats = np.zeros((BH, 4), np.float64)
+    lib.oracle_think_prune(_ptr(k), _ptr(qn), BH, S, D, T, _ptr(mask), _ptr(vals), _ptr(stats))
     return mask, vals, stats
 
 

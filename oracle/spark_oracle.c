@@ -295,6 +295,74 @@ void oracle_recover_values(const uint32_t *vmask, const float *vvals, long bh, l
     }
 }
 
+/*
+ * ThinK, the structured channel-pruning comparator ([W] 1 and Fig. 2(c): one
+ * channel mask shared by all tokens of a head, no recovery; [W] 4.2 compares
+ * SparK with it at lambda = 0.5 and 0.8).  Reading R18 (the pages give no
+ * ThinK formula): the relaxed objective of [W] 3.1 with one mask for the
+ * whole key block of a (b, h) ranks channel j by
+ *     score_j = qn_j * ||k^j||_2,   ||k^j||_2 = sqrt(sum_t k_tj^2)  (fp64)
+ * over the S prompt tokens; the T channels of largest score (ties -> lower
+ * channel) are kept for every token.  The cache is the plain one (every
+ * token's mask equal, kept values in ascending channel order); without
+ * recovery a pruned entry reads as 0, which the cache states with
+ * stats = {N = S*(D-T), 0, 0, mu = 0}.
+ */
+typedef struct {
+    double s;
+    int j;
+} chan_dscore;
+
+static int by_dscore_desc(const void *pa, const void *pb)
+{
+    const chan_dscore *a = (const chan_dscore *)pa, *b = (const chan_dscore *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->j < b->j) ? -1 : ((a->j > b->j) ? 1 : 0);  /* lower channel first */
+}
+
+void oracle_think_prune(const float *k, const float *qn, long BH, long S, int D, int T, uint32_t *mask,
+                        float *vals, double *stats)
+{
+    const int nw = (D + 31) / 32;
+    chan_dscore *ord = (chan_dscore *)malloc(sizeof(chan_dscore) * (size_t)D);
+    unsigned char *keep = (unsigned char *)malloc((size_t)D);
+    for (long bh = 0; bh < BH; ++bh) {
+        for (int j = 0; j < D; ++j) {
+            double ss = 0.0;
+            for (long t = 0; t < S; ++t) {
+                const double x = (double)k[(bh * S + t) * D + j];
+                ss += x * x;
+            }
+            ord[j].s = (double)qn[bh * D + j] * sqrt(ss);
+            ord[j].j = j;
+        }
+        qsort(ord, (size_t)D, sizeof(chan_dscore), by_dscore_desc);
+        memset(keep, 0, (size_t)D);
+        for (int r = 0; r != T; ++r)  /* the T best channels */
+            keep[ord[r].j] = 1;
+        for (long t = 0; t < S; ++t) {
+            uint32_t *mrow = mask + (bh * S + t) * nw;
+            float *vrow = vals + (bh * S + t) * (long)T;
+            for (int q = 0; q < nw; ++q)
+                mrow[q] = 0u;
+            int pos = 0;
+            for (int j = 0; j < D; ++j)
+                if (keep[j]) {
+                    mrow[j / 32] |= 1u << (j % 32);
+                    vrow[pos] = k[(bh * S + t) * D + j];
+                    ++pos;
+                }
+        }
+        stats[bh * 4 + 0] = (double)S * (double)(D - T);
+        stats[bh * 4 + 1] = 0.0;
+        stats[bh * 4 + 2] = 0.0;
+        stats[bh * 4 + 3] = 0.0;
+    }
+    free(ord);
+    free(keep);
+}
+
 /* Recovery F = Degenerate, [W] 3.3 steps 2-4 and the F table: the sampled
  * score is mu_pruned, and the key is back-solved from it as
  * k~ = w~ / ||q^j||_2 (R5).  Kept channels are the stored key values.

@@ -16,7 +16,8 @@ PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_snapkv_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_sampling_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_group_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_vprune_pins.py")]
+        os.path.join(ROOT, "tests", "test_oracle_vprune_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_think_pins.py")]
 
 MUTANTS = {
     "tie_rule_reversed": ("return (a->j > b->j) - (a->j < b->j);",
@@ -70,6 +71,13 @@ MUTANTS = {
     # V-channel pruning (reading R16)
     "values_pruned_not_dropped": ("? (double)vrow[pos++] : 0.0;", "? (double)vrow[pos++] : 1e-3;"),
     "values_index_not_advanced": ("? (double)vrow[pos++] : 0.0;", "? (double)vrow[pos] : 0.0;"),
+    # ThinK comparator (reading R18)
+    "think_no_query_norm": ("ord[j].s = (double)qn[bh * D + j] * sqrt(ss);", "ord[j].s = sqrt(ss);"),
+    "think_sum_not_squared": ("ss += x * x;", "ss += fabs(x);"),
+    "think_ties_reversed": ("return (a->j < b->j) ? -1 : ((a->j > b->j) ? 1 : 0);",
+                            "return (a->j > b->j) ? -1 : ((a->j < b->j) ? 1 : 0);"),
+    "think_recovers_mean": ("stats[bh * 4 + 3] = 0.0;\n    }\n    free(ord);",
+                            "stats[bh * 4 + 3] = 1.0;\n    }\n    free(ord);"),
     "lambda_truncates": ("return (int)llround((1.0 - (double)lambda) * (double)D);",
                          "return (int)((1.0 - (double)lambda) * (double)D);"),
 }
