@@ -360,8 +360,9 @@ def run_gpu(args):
 def run_variants(job, wl, stream, peak, peak_kind, iters=5):
     """Method variants on the same prompt, timed outside the step with CUDA
     events on the launching stream: SparK-g grouped pruning with the pages'
-    g = 4 rates (0.25, 0.5, 0.75, 1.0), and value-channel pruning at
-    lambda_v = 0.5 with decode over the pruned key and value caches (bf16)."""
+    g = 4 rates (0.25, 0.5, 0.75, 1.0), the ThinK structured comparator at the
+    same T (prune + decode), and value-channel pruning at lambda_v = 0.5 with
+    decode over the pruned key and value caches (bf16)."""
     sp = job.sp
     S = job.S_kept
     k = job.k_ev if wl.keep else job.k
@@ -391,6 +392,20 @@ def run_variants(job, wl, stream, peak, peak_kind, iters=5):
                       f"frac_{peak_kind}": gbs / peak, "bytes_per_call": nbytes,
                       "timing": "CUDA events around spark_prune_grouped on its stream, outside the step"}
     del kg
+    # ThinK comparator at the same T: structured prune, then the same decode
+    kt_ = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, job.T, wl.torch_dtype, device=job.dev)
+    wst = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_THINK, wl.rows, wl.Hkv, wl.G, S, wl.D, job.T, 0),
+                       job.dev)
+    us_tp = timed(lambda: sp.spark_prune_think(k, job.q_obs, wl.G, wl.W, kt_, wst, stream))
+    wsd_t = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_DECODE, wl.rows, wl.Hkv, wl.G, S, wl.D, job.T, 0),
+                         job.dev)
+    outt = torch.empty_like(job.out)
+    us_td = timed(lambda: sp.spark_decode_attn(job.q, kt_, v, None, None, 0, 0, wl.G, outt, wsd_t, stream=stream))
+    nb_t = wl.BH * S * (16 + job.T * es + wl.D * es)
+    out["think"] = {"T": job.T, "prune_us": us_tp, "prune_bytes": wl.BH * S * (2 * wl.D * es + 16 + job.T * es),
+                    "decode_us": us_td, "decode_gbs": nb_t / (us_td / 1e6) / 1e9,
+                    "timing": "CUDA events on the stream, outside the step; no tail"}
+    del kt_, wst, wsd_t
     if wl.dtype == "bf16":
         Tv = sp.spark_lambda_to_T(0.5, wl.D)
         vc = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, Tv, wl.torch_dtype, device=job.dev)

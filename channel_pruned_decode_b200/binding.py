@@ -29,9 +29,10 @@ SPARK_F_EXPONENTIAL = 2
 SPARK_OP_PRUNE = 0
 SPARK_OP_DECODE = 1
 SPARK_OP_SNAPKV = 2
+SPARK_OP_THINK = 3
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
-           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_prune_values", "spark_decode_attn",
+           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_prune_values", "spark_prune_think", "spark_decode_attn",
            "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_tail_append", "spark_device_status",
            "spark_status_str", "spark_snapkv_evict")
 
@@ -76,6 +77,8 @@ def lib():
         L.spark_prune_grouped.restype = I
         L.spark_prune_values.argtypes = [P, ctypes.POINTER(spark_kcache), P, Z, P]
         L.spark_prune_values.restype = I
+        L.spark_prune_think.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P, Z, P]
+        L.spark_prune_think.restype = I
         L.spark_decode_attn_kv.argtypes = [P, ctypes.POINTER(spark_kcache), ctypes.POINTER(spark_kcache), P, P, I,
                                            I, I, P, P, Z, P]
         L.spark_decode_attn_kv.restype = I
@@ -209,6 +212,15 @@ def spark_prune_grouped(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, gr
     rc = lib().spark_prune_grouped(_ptr(k), _ptr(q_obs), G, W, len(group_T), tg, ctypes.byref(s), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_prune_grouped")
+
+
+def spark_prune_think(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, kc: KCache, ws: torch.Tensor,
+                      stream=None) -> None:
+    """ThinK structured pruning (comparator): one channel mask per head (see spark.h)."""
+    s = kc.struct()
+    rc = lib().spark_prune_think(_ptr(k), _ptr(q_obs), G, W, ctypes.byref(s), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_prune_think")
 
 
 def spark_prune_values(v: torch.Tensor, vc: KCache, ws: torch.Tensor, stream=None) -> None:

@@ -12,7 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libspark.so")
 
-SOURCES = ["api.cu", "prune.cu", "decode.cu", "snapkv.cu"]
+SOURCES = ["api.cu", "prune.cu", "decode.cu", "snapkv.cu", "think.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -14,6 +14,9 @@ cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, 
                           const void *k_tail, const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
                           unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st);
 cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws, cudaStream_t st);
+cudaError_t launch_think(const void *k, const void *q_obs, int G, int W, const spark_kcache &kc, void *ws,
+                         cudaStream_t st);
+size_t think_workspace(long BH, int S);
 cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
                           int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st);
 
@@ -103,6 +106,7 @@ size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D, int T,
     const long BH = (long)B * Hkv;
     if (op == SPARK_OP_PRUNE) return round256(prune_workspace(BH, S));
     if (op == SPARK_OP_SNAPKV) return round256(snapkv_workspace(BH, S, 0));
+    if (op == SPARK_OP_THINK) return round256(think_workspace(BH, S));
     if (op == SPARK_OP_DECODE) {
         if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
         // the geometry depends on the element size only through the stage
@@ -185,6 +189,21 @@ size_t spark_workspace_bytes_kv(int B, int Hkv, int G, int S, int D, int T, int 
     if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
     const DecodeGeom g = decode_geometry((long)B * Hkv, S, T, Tv, 2, G, num_sms());
     return round256(decode_workspace((long)B * Hkv, g, G));
+}
+
+int spark_prune_think(const void *k, const void *q_obs, int G, int W, const spark_kcache *out, void *workspace,
+                      size_t ws_bytes, void *stream) {
+    int rc = check_cache(out);
+    if (rc != SPARK_OK) return rc;
+    if (G < 1 || W < 1) return SPARK_ERR_ARG;
+    const long BH = (long)out->B * out->Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
+    if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < think_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_think(k, q_obs, G, W, *out, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 
 int spark_prune_values(const void *v, const spark_kcache *out, void *workspace, size_t ws_bytes, void *stream) {

@@ -609,6 +609,15 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
     return cudaGetLastError();
 }
 
+cudaError_t launch_qnorm(const void *q_obs, int G, int W, long BH, int dtype, float *qn, cudaStream_t st) {
+    if (BH == 0) return cudaSuccess;
+    if (dtype == SPARK_BF16)
+        qnorm_kernel<__nv_bfloat16><<<(unsigned)BH, kD, 0, st>>>(static_cast<const __nv_bfloat16 *>(q_obs), G, W, qn);
+    else
+        qnorm_kernel<float><<<(unsigned)BH, kD, 0, st>>>(static_cast<const float *>(q_obs), G, W, qn);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_prune(const void *k, const void *q_obs, int G, int W, const spark_kcache &kc,
                          void *ws, cudaStream_t st) {
     if (kc.dtype == SPARK_BF16) return launch_prune_t<__nv_bfloat16>(k, q_obs, G, W, kc, ws, st, nullptr);

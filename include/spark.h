@@ -65,7 +65,7 @@ typedef enum {
     SPARK_F_EXPONENTIAL = 2   /* w~ ~ Exp(1/mu) (mean mu)                     */
 } spark_recovery;
 
-typedef enum { SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1, SPARK_OP_SNAPKV = 2 } spark_op;
+typedef enum { SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1, SPARK_OP_SNAPKV = 2, SPARK_OP_THINK = 3 } spark_op;
 
 /*
  * The packed key cache of [W] 3.3 step 1 / Fig. 3: per token the kept key
@@ -193,6 +193,22 @@ SPARK_API int spark_decode_attn_kv(const void *q, const spark_kcache *kc, const 
 /* Workspace bytes of spark_decode_attn_kv for key budget T and value budget
  * Tv (the tail capacity as n_tail); 0 on bad arguments. */
 SPARK_API size_t spark_workspace_bytes_kv(int B, int Hkv, int G, int S, int D, int T, int Tv, int n_tail);
+
+/*
+ * ThinK, the structured channel-pruning comparator of the pages ([W] 1 and
+ * Fig. 2(c): one channel mask shared by all tokens of a head, no recovery;
+ * [W] 4.2).  The library's reading (the pages give no ThinK formula): per
+ * (b, h), channel j is ranked by qn[j] * sqrt(sum_t k[t,j]^2) (fp64, qn as in
+ * spark_prune), and the out->T channels of largest score (ties -> lower
+ * channel) are kept for every token.  The cache has spark_prune's layout
+ * (every token's mask equal) and stats = {S*(D-T), 0, 0, 0}: mu = 0, so
+ * spark_decode_attn reads a pruned entry as 0 (no recovery).
+ * Arguments as for spark_prune; workspace
+ * spark_workspace_bytes(SPARK_OP_THINK, ...).  Reads k twice (channel norms,
+ * then the kept values).
+ */
+SPARK_API int spark_prune_think(const void *k, const void *q_obs, int G, int W, const spark_kcache *out,
+                                void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * spark_prune without a workspace.  Not part of the SparK method: the paper

@@ -205,3 +205,14 @@ def test_value_pruning_entry_points_reject_bad_args(L):
     assert L.spark_prune_values(16, ctypes.byref(_kc(T=129)), 256, 1 << 20, None) == B.SPARK_ERR_ARG
     assert L.spark_prune_values(None, ctypes.byref(vc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
     assert L.spark_prune_values(16, ctypes.byref(vc), None, 1 << 20, None) == B.SPARK_ERR_WORKSPACE
+
+
+def test_prune_think_rejects_bad_args(L):
+    kc = _kc()
+    f = L.spark_prune_think
+    assert f(16, 16, 0, 32, ctypes.byref(kc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert f(16, 16, 4, 0, ctypes.byref(kc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert f(None, 16, 4, 32, ctypes.byref(kc), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+    assert f(16, 16, 4, 32, ctypes.byref(kc), None, 1 << 20, None) == B.SPARK_ERR_WORKSPACE
+    assert f(16, 16, 4, 32, ctypes.byref(kc), 256, 64, None) == B.SPARK_ERR_WORKSPACE
+    assert f(16, 16, 4, 32, ctypes.byref(_kc(T=129)), 256, 1 << 20, None) == B.SPARK_ERR_ARG
