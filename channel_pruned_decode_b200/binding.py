@@ -33,7 +33,7 @@ SPARK_OP_THINK = 3
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
            "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_prune_values", "spark_prune_think", "spark_decode_attn",
-           "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_tail_append", "spark_device_status",
+           "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_selftest_wait_timeout", "spark_tail_append", "spark_device_status",
            "spark_status_str", "spark_snapkv_evict")
 
 
@@ -79,6 +79,8 @@ def lib():
         L.spark_prune_values.restype = I
         L.spark_prune_think.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P, Z, P]
         L.spark_prune_think.restype = I
+        L.spark_selftest_wait_timeout.argtypes = [P, I, P]
+        L.spark_selftest_wait_timeout.restype = I
         L.spark_decode_attn_kv.argtypes = [P, ctypes.POINTER(spark_kcache), ctypes.POINTER(spark_kcache), P, P, I,
                                            I, I, P, P, Z, P]
         L.spark_decode_attn_kv.restype = I
@@ -221,6 +223,11 @@ def spark_prune_think(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, kc: 
     rc = lib().spark_prune_think(_ptr(k), _ptr(q_obs), G, W, ctypes.byref(s), _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_prune_think")
+
+
+def spark_selftest_wait_timeout(ws: torch.Tensor, limit_us: int, stream=None) -> None:
+    """Make one bounded device wait run out on purpose (status word test)."""
+    _check(lib().spark_selftest_wait_timeout(_ptr(ws), limit_us, _stream(stream)), "spark_selftest_wait_timeout")
 
 
 def spark_prune_values(v: torch.Tensor, vc: KCache, ws: torch.Tensor, stream=None) -> None:

@@ -56,6 +56,20 @@ static int check_cache(const spark_kcache *kc) {
     return SPARK_OK;
 }
 
+// Self-test of the bounded-wait path: one warp waits on an mbarrier that
+// nothing ever arrives on, gives up after limit_ns, and records the timeout in
+// the status word exactly as the decode pipeline does.
+__global__ void wait_selftest_kernel(uint32_t *status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    const bool ok = mbar_wait_limit(smem_u32(&bar), 0u, limit_ns);
+    if (__all_sync(0xffffffffu, !ok) && threadIdx.x == 0) atomicOr(status, kDevTimeout);
+}
+
 __global__ void tail_append_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
                                    uint4 *__restrict__ k_tail, uint4 *__restrict__ v_tail,
                                    int row_vec, int tail_cap, int slot) {
@@ -278,6 +292,14 @@ int spark_tail_append(const void *k_new, const void *v_new, void *k_tail, void *
     tail_append_kernel<<<(unsigned)BH, 32 * ((row_vec + 31) / 32), 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), static_cast<uint4 *>(k_tail),
         static_cast<uint4 *>(v_tail), row_vec, tail_cap, slot);
+    return cudaGetLastError() == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_selftest_wait_timeout(void *workspace, int limit_us, void *stream) {
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (limit_us < 1 || limit_us > 1000000) return SPARK_ERR_ARG;
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t *>(workspace),
+                                                                          1000ull * (unsigned long long)limit_us);
     return cudaGetLastError() == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 

@@ -117,16 +117,22 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Wait for phase `parity` of an mbarrier, giving up after ~1 s of device
-// time.  Returns false on timeout (the caller records it and winds down).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Wait for phase `parity` of an mbarrier, giving up after `limit_ns` of
+// device time (and after at most 2^26 polls).  Returns false on timeout (the
+// caller records it and winds down).
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t it = 0; it < (1u << 26); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u && global_ns() - t0 > 1000000000ull) return false;
+        if ((it & 63u) == 63u && global_ns() - t0 > limit_ns) return false;
     }
     return false;
+}
+
+// the pipeline's waits give up after ~1 s
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    return mbar_wait_limit(bar, parity, 1000000000ull);
 }
 
 // Async bulk copy global -> shared, completion counted on `bar` (bytes).

@@ -306,6 +306,17 @@ SPARK_API int spark_tail_append(const void *k_new, const void *v_new, void *k_ta
  * clear != 0, reset it to zero.  Returns SPARK_ERR_CUDA if a copy fails. */
 SPARK_API int spark_device_status(void *workspace, int *status, int clear, void *stream);
 
+/*
+ * Self-test of failure detection (not part of the SparK method): launches one
+ * warp that waits on an mbarrier nothing arrives on, gives up after limit_us
+ * microseconds (1 <= limit_us <= 1e6) -- the same bounded wait the decode
+ * pipeline uses, with a shorter limit -- and records SPARK_ERR_TIMEOUT in the
+ * workspace's status word, which spark_device_status then reports.  No fault,
+ * trap or hang is involved; the context stays usable.  Returns SPARK_ERR_ARG
+ * for a limit out of range, SPARK_ERR_WORKSPACE for a missing workspace.
+ */
+SPARK_API int spark_selftest_wait_timeout(void *workspace, int limit_us, void *stream);
+
 /* Static description of a status code. */
 SPARK_API const char *spark_status_str(int status);
 
