@@ -10,7 +10,8 @@
 //   qnorm_kernel   one CTA per (row, kv head), one thread per channel: the
 //                  fp64 sum of squares over the G*W window rows of the group,
 //                  rounded once to fp32.
-//   prune_kernel   one CTA per 256-token chunk of one (row, kv head).  Four
+//   prune_kernel   one CTA per chunk of 256 to 1024 tokens (8 to 32 groups of
+//                  32, more for large launches) of one (row, kv head).  Four
 //                  lanes own one token (32 channels each): exact fp32 keys
 //                  w = qn_j * |k_j| in registers, plus 16-bit search keys
 //                  fp16(w * 2^-floor(log2 max qn)), two channels per word.
@@ -306,7 +307,7 @@ struct GroupArgs {
 template <typename E, bool kGrouped>
 __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
-                 E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks,
+                 E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks, int gpc,
                  GroupArgs ga) {
     using Raw = typename RawT<E>::type;
     // per-warp staging of the kept values: [kept index][8 tokens of the warp]
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     Raw *vt = vtile[warp];
     uint32_t tau = 1u;
     double acc_w = 0.0, acc_w2 = 0.0;
-    const long g_first = (long)chunk * kPruneGroups;
+    const long g_first = (long)chunk * gpc;
     const E *krow = k + ((size_t)bh * S + g_first * 32 + tl) * kD + 32 * s;  // this lane's slice, group 0
     E *gvals = vals + (size_t)bh * S32 * T + (size_t)g_first * 32 * T;      // group 0's values
 
@@ -397,7 +398,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     auto group = [&](int gi, KSlice<E> &cur, KSlice<E> &nxt) {
         const long t = (g_first + gi) * 32 + tl;
         const bool valid = t < S;
-        if (gi + 1 < kPruneGroups && t + 32 < S) nxt.load(krow + (size_t)(gi + 1) * 32 * kD);
+        if (gi + 1 < gpc && t + 32 < S) nxt.load(krow + (size_t)(gi + 1) * 32 * kD);
         else nxt.zero();
 
         // exact fp32 saliency keys w_j = qn_j * |k_j| (packed fp32 multiplies,
@@ -532,7 +533,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     KSlice<E> ka, kb;
     if (g_first * 32 + tl < S) ka.load(krow);
     else ka.zero();
-    for (int gi = 0; gi < kPruneGroups; gi += 2) {
+    for (int gi = 0; gi < gpc; gi += 2) {
         if ((g_first + gi) * 32 >= S) break;  // uniform across the CTA
         group(gi, ka, kb);
         if ((g_first + gi + 1) * 32 >= S) break;
@@ -594,16 +595,17 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
     if (BH == 0) return cudaSuccess;
     double *partial = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
     qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn);
-    const int nch = prune_chunks(kc.S);
+    const int gpc = prune_groups_per_cta(BH, kc.S);
+    const int nch = prune_chunks(kc.S, gpc);
     if (nch > 0) {
         if (ga)
             prune_kernel<E, true><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-                nch, *ga);
+                nch, gpc, *ga);
         else
             prune_kernel<E, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-                nch, GroupArgs{});
+                nch, gpc, GroupArgs{});
     }
     stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.S, kc.T, kc.stats);
     return cudaGetLastError();
@@ -633,16 +635,17 @@ cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws,
     if (BH == 0) return cudaSuccess;
     fill_ones_kernel<<<(unsigned)BH, kD, 0, st>>>(vc.qn);
     double *partial = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
-    const int nch = prune_chunks(vc.S);
+    const int gpc = prune_groups_per_cta(BH, vc.S);
+    const int nch = prune_chunks(vc.S, gpc);
     if (nch > 0) {
         if (vc.dtype == SPARK_BF16)
             prune_kernel<__nv_bfloat16, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16 *>(v), vc.qn, vc.mask, static_cast<__nv_bfloat16 *>(vc.vals),
-                partial, vc.S, vc.T, nch, GroupArgs{});
+                partial, vc.S, vc.T, nch, gpc, GroupArgs{});
         else
             prune_kernel<float, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const float *>(v), vc.qn, vc.mask, static_cast<float *>(vc.vals), partial, vc.S, vc.T,
-                nch, GroupArgs{});
+                nch, gpc, GroupArgs{});
     }
     stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, vc.S, vc.T, vc.stats);
     return cudaGetLastError();

@@ -18,14 +18,25 @@ constexpr uint32_t kDevTimeout = 1u;  // status bit: a bounded wait ran out
 
 // ----------------------------------------------------------------- prune
 constexpr int kPruneThreads = 128;    // 4 lanes per token, 32 tokens per group
-constexpr int kPruneGroups = 8;       // 32-token groups per CTA (256 tokens)
+constexpr int kPruneGroups = 8;       // fewest 32-token groups per CTA (256 tokens)
+constexpr int kPruneGroupsMax = 32;   // most (1024 tokens) for large launches
 constexpr int kMaxGroups = 8;         // SparK-g channel groups
 
-inline int prune_chunks(int S) {
-    const int per = 32 * kPruneGroups;
+// 32-token groups per prune CTA: 8, doubled (up to 32) while the launch still
+// has >= 2368 CTAs (16 per SM at 4 resident per SM), which amortises each
+// CTA's setup and the cold start of its threshold estimates.
+inline int prune_groups_per_cta(long BH, int S) {
+    int g = kPruneGroups;
+    while (g < kPruneGroupsMax && BH * (long)((S + 64L * g - 1) / (64L * g)) >= 2368) g *= 2;
+    return g;
+}
+
+inline int prune_chunks(int S, int groups_per_cta = kPruneGroups) {
+    const int per = 32 * groups_per_cta;
     return S > 0 ? (S + per - 1) / per : 0;
 }
 
+// sized for the smallest chunks, so any groups-per-CTA choice fits
 inline size_t prune_workspace(long BH, int S) {
     return kWsHeader + (size_t)BH * (size_t)prune_chunks(S) * 2 * sizeof(double);
 }
