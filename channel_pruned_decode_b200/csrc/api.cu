@@ -20,8 +20,12 @@ size_t think_workspace(long BH, int S);
 cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
                           int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st);
 
+size_t snapkv_partials_bytes(long BH);
+
+// scores (fp32) and pooled keys (u32) per prefix token, then the per-split
+// softmax partials
 static size_t snapkv_workspace(long BH, int S, int W) {
-    return kWsHeader + (size_t)BH * (size_t)(S - W) * 8;
+    return kWsHeader + (size_t)BH * (size_t)(S - W) * 8 + snapkv_partials_bytes(BH);
 }
 
 static int elem_size(int dtype) {
