@@ -157,7 +157,7 @@ class Job:
             self.wsp = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_PRUNE, R, H, G, wl.keep, D, self.T, 0), dev)
             self.wsd = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_DECODE, R, H, G, wl.keep, D, self.T,
                                                              self.cap), dev)
-            self.launches_per_step += 3  # scores, select, gather
+            self.launches_per_step += 4  # two score passes, select, gather
 
     def step(self, stream, ev=None):
         sp, wl = self.sp, self.wl
