@@ -362,14 +362,290 @@ __global__ void snap_gather_kernel(const uint4 *__restrict__ k, const uint4 *__r
     v_out[((size_t)bh * keep + i) * row_vec + c] = v[((size_t)bh * S + t) * row_vec + c];
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 version of the two score passes.  Per CTA: 256 threads (8 warps);
+// a 128 x 128 query tile (window rows, zero-padded) and a ring of two 128-key
+// tiles in shared memory, K-major with the 128-byte swizzle that the UMMA
+// descriptors describe; two 128-column fp32 accumulators in tensor memory.
+// Thread 0 issues the tcgen05.mma instructions and commits them to an
+// mbarrier; every thread then reads half of one accumulator row (tcgen05.ld:
+// warp w reads TMEM lanes 32*(w%4).. and columns 64*(w/4)..).  Pass 0
+// computes S = Q K^T (a row is a window row: its running max and exp-sum are
+// kept per half and merged at the end); pass 1 computes S^T = K Q^T (a row is
+// a key: its probability sum over the window rows is summed per half, then
+// the halves are added).
+constexpr int kTcKeys = 128;                  // keys per tile (MMA M or N)
+constexpr int kTcThreads = 256;  // two warps per TMEM lane quarter, one per column half
+constexpr uint32_t kTcTileBytes = 128 * 256;  // 128 rows x 128 bf16
+constexpr uint32_t kTcCols = 256;             // two accumulators
+
+// byte offset of 16-byte chunk cc (0..15) of row r in a K-major 128B-swizzled
+// tile: two K-blocks of 64 elements, 128 bytes per row, chunks XOR-ed with the
+// row's low 3 bits inside each 8-row, 1024-byte atom
+__device__ __forceinline__ uint32_t tc_off(int r, int cc) {
+    return (uint32_t)((cc >> 3) * (128 * 128) + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
+}
+
+// UMMA shared-memory descriptor of the K-major SW128 tile at `addr` (1024-byte
+// aligned atoms; the 8-row groups 1024 bytes apart), for the 16-element K step
+// `ks`: start address, stride byte offset 1024, version 1, layout SWIZZLE_128B
+__device__ __forceinline__ uint64_t tc_desc(uint32_t tile_addr, int ks) {
+    const uint32_t a = tile_addr + (uint32_t)(ks >> 2) * (128 * 128) + (uint32_t)(ks & 3) * 32;
+    return (uint64_t)((a >> 4) & 0x3fff) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, N = 128, M = 128
+constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t da, uint64_t db, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        :
+        : "r"(d_tmem), "l"(da), "l"(db), "r"(kTcIdesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kTcThreads, 2)
+    snap_tc_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ q_obs, int S, int G,
+                   int W, int nsplit, float *__restrict__ ml, float *__restrict__ scores,
+                   uint32_t *__restrict__ status) {
+    extern __shared__ unsigned char sm_raw[];
+    __shared__ uint64_t bars[2];
+    __shared__ uint32_t tmem_base_s;
+    __shared__ float rowm[kSnapMaxRows], rowil[kSnapMaxRows];  // merged row max and 1 / exp-sum (pass 1)
+    __shared__ float half_a[kSnapMaxRows], half_b[kSnapMaxRows];  // the upper column half's partial results
+    __shared__ int fail_s;
+    // 1024-byte aligned tiles: queries, then two key buffers
+    const uint32_t base = (smem_u32(sm_raw) + 1023u) & ~1023u;
+    const uint32_t sq = base, sk0 = base + kTcTileBytes;
+
+    const long bh = blockIdx.x / nsplit;
+    const int split = blockIdx.x % nsplit;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int R = G * W;
+    const long P = (long)S - W;
+    const __nv_bfloat16 *kb = k + (size_t)bh * S * kD;
+    const __nv_bfloat16 *qb = q_obs + (size_t)bh * R * kD;
+    const int ntile = (S + kTcKeys - 1) / kTcKeys;
+    const int per = (ntile + nsplit - 1) / nsplit;
+    const int tile_lo = min(ntile, split * per), tile_hi = min(ntile, tile_lo + per);
+    float *mlh = ml + (size_t)bh * nsplit * kSnapMaxRows * 2;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
+                     "r"(kTcCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fail_s = 0;
+    }
+    // queries (rows past R are zero)
+    for (int i = tid; i < 128 * 16; i += kTcThreads) {
+        const int r = i >> 4, cc = i & 15;
+        cp_async16(sq + tc_off(r, cc), qb + (size_t)min(r, R - 1) * kD + cc * 8, r < R);
+    }
+    auto load_tile = [&](int tile) {
+        const uint32_t dst = sk0 + (uint32_t)(tile & 1) * kTcTileBytes;
+        for (int i = tid; i < kTcKeys * 16; i += kTcThreads) {
+            const int r = i >> 4, cc = i & 15;
+            const long t = (long)tile * kTcKeys + r;
+            cp_async16(dst + tc_off(r, cc), kb + (size_t)min(t, (long)S - 1) * kD + cc * 8, t < S);
+        }
+    };
+    if (kMode == 1) {
+        // merged row statistics in split order (split 0 holds key 0, which
+        // every row sees); rows past R contribute nothing (1 / l = 0)
+        if (tid < kSnapMaxRows) {
+            float m = -INFINITY, l = 0.f;
+            if (tid < R) {
+                for (int sp = 0; sp < nsplit; ++sp) {
+                    const float ma = mlh[((size_t)sp * kSnapMaxRows + tid) * 2];
+                    const float la = mlh[((size_t)sp * kSnapMaxRows + tid) * 2 + 1];
+                    const float n = fmaxf(m, ma);
+                    l = (m == -INFINITY ? 0.f : l * exp2f(m - n)) + (ma == -INFINITY ? 0.f : la * exp2f(ma - n));
+                    m = n;
+                }
+            }
+            rowm[tid] = tid < R ? m : 0.f;
+            rowil[tid] = tid < R ? 1.f / l : 0.f;
+        }
+    }
+    if (tile_lo < tile_hi) load_tile(tile_lo);
+    cp_async_commit();
+    if (tile_lo + 1 < tile_hi) load_tile(tile_lo + 1);
+    cp_async_commit();
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = tmem_base_s;
+
+    // MMA of `tile` into accumulator tile & 1: pass 0 A = queries, B = keys;
+    // pass 1 A = keys, B = queries
+    auto issue = [&](int tile) {
+        if (tid == 0) {
+            const uint32_t kt = sk0 + (uint32_t)(tile & 1) * kTcTileBytes;
+            const uint32_t a_t = kMode == 0 ? sq : kt, b_t = kMode == 0 ? kt : sq;
+            const uint32_t d = tmem + (uint32_t)(tile & 1) * 128u;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) tc_mma(d, tc_desc(a_t, ks), tc_desc(b_t, ks), ks > 0 ? 1u : 0u);
+            tc_commit(smem_u32(&bars[tile & 1]));
+        }
+    };
+    // first tile's operands (and the queries) landed: make them visible to the
+    // tensor core's proxy, then issue
+    if (tile_lo < tile_hi) {
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        __syncthreads();
+        issue(tile_lo);
+    }
+
+    const int row = 32 * (warp & 3) + (tid & 31);  // this thread's TMEM lane
+    const int chalf = warp >> 2;                    // its column half
+    float m_run = -INFINITY, l_run = 0.f;          // pass 0: this window row's statistics
+    const long lim_row = P + (row % W);
+    bool failed = false;
+    for (int tile = tile_lo; tile < tile_hi; ++tile) {
+        // next tile's operands -> issue its MMA before this tile's epilogue
+        if (tile + 1 < tile_hi) {
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            __syncthreads();
+            issue(tile + 1);
+        }
+        // this tile's accumulator is complete
+        const uint32_t par = (uint32_t)(((tile - tile_lo) >> 1) & 1);
+        const bool ok = mbar_wait_limit(smem_u32(&bars[tile & 1]), par, 1000000000ull);
+        if (!__all_sync(0xffffffffu, ok)) failed = true;
+        if (__syncthreads_or(failed ? 1 : 0)) {
+            failed = true;
+            break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        // its key buffer is free: fetch the tile after next
+        if (tile + 2 < tile_hi) load_tile(tile + 2);
+        cp_async_commit();
+        const uint32_t taddr =
+            tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(tile & 1) * 128u + (uint32_t)(64 * chalf);
+        const long t0 = (long)tile * kTcKeys;
+        if (kMode == 0) {
+            // S[row][key]: this row's logits for the tile's 128 keys
+            const bool mask = t0 + kTcKeys - 1 > P;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kTcKeys / 2; c0 += 32) {
+                float v[32];
+                tc_ld32(taddr + (uint32_t)c0, v);
+                if (mask) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const long t = t0 + 64 * chalf + c0 + i;
+                        v[i] = (t <= lim_row && t < S) ? v[i] : -INFINITY;
+                    }
+                }
+                float x = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x = fmaxf(x, v[i]);
+                const float n = fmaxf(m_run, x * kSnapScale);
+                const float b = n == -INFINITY ? 0.f : n;
+                float s = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) s += exp2f(fmaf(v[i], kSnapScale, -b));
+                l_run = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - n)) + s;
+                m_run = n;
+            }
+        } else {
+            // S^T[key][row]: this key's probabilities over the window rows
+            const long t = t0 + row;
+            const bool valid_t = t < P;
+            float acc = 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kSnapMaxRows / 2; c0 += 32) {
+                float v[32];
+                tc_ld32(taddr + (uint32_t)c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int c = 64 * chalf + c0 + i;
+                    acc += exp2f(fmaf(v[i], kSnapScale, -rowm[c])) * rowil[c];
+                }
+            }
+            // lower half + upper half, in that order
+            if (chalf == 1) half_a[row] = acc;
+            __syncthreads();
+            if (chalf == 0 && valid_t) scores[(size_t)bh * (P > 0 ? P : 0) + t] = acc + half_a[row];
+        }
+        // accumulator tile & 1 and its key buffer may be reused
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    if (failed && tid == 0) atomicOr(status, kDevTimeout);
+    if (kMode == 0) {
+        // merge the two column halves of each row (lower half first)
+        if (chalf == 1) {
+            half_a[row] = m_run;
+            half_b[row] = l_run;
+        }
+        __syncthreads();
+        if (chalf == 0 && !failed && row < R) {
+            const float mb = half_a[row], lb = half_b[row];
+            const float n = fmaxf(m_run, mb);
+            const float l = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - n)) +
+                            (mb == -INFINITY ? 0.f : lb * exp2f(mb - n));
+            mlh[((size_t)split * kSnapMaxRows + row) * 2] = n;
+            mlh[((size_t)split * kSnapMaxRows + row) * 2 + 1] = l;
+        }
+    }
+    // release the tensor memory (a timed-out MMA is waited for once more,
+    // with a bound, before the columns are freed)
+    if (failed && tid == 0) {
+        for (int b = 0; b < 2; ++b) (void)mbar_wait_limit(smem_u32(&bars[b]), 0u, 1000000ull);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcCols));
+    }
+}
+
+size_t snapkv_tc_smem_bytes() { return 3 * (size_t)kTcTileBytes + 1024; }
+
 size_t snapkv_smem_bytes() {
     return (size_t)kSnapMaxRows * 256 + (size_t)kSnapStages * kSnapKeys * 256 + 8 * kSnapKeys * 4;
 }
 
 // CTAs per head: about six waves of two CTAs per SM over the whole launch,
-// at least four 64-key tiles per CTA, at most kSnapMaxSplit
+// at least four 128-key tiles per CTA, at most kSnapMaxSplit
 int snapkv_splits(long BH, int S, int num_sms) {
-    const int ntile = (S + kSnapKeys - 1) / kSnapKeys;
+    const int ntile = (S + kTcKeys - 1) / kTcKeys;
     long ns = (12L * num_sms + BH - 1) / (BH > 0 ? BH : 1);
     ns = std::min<long>(ns, kSnapMaxSplit);
     ns = std::min<long>(ns, std::max(1, ntile / 4));
@@ -384,18 +660,19 @@ cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long 
     float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
     uint32_t *pooled = reinterpret_cast<uint32_t *>(scores + (size_t)BH * P);
     float *ml = reinterpret_cast<float *>(pooled + (size_t)BH * P);
-    const size_t smem = snapkv_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(snap_pass_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = snapkv_tc_smem_bytes();
+    cudaError_t e = cudaFuncSetAttribute(snap_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(snap_pass_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(snap_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const int ns = snapkv_splits(BH, S, nsm);
     const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(k);
     const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q_obs);
-    snap_pass_kernel<0><<<(unsigned)(BH * ns), kSnapThreads, smem, st>>>(kb, qb, S, G, W, ns, ml, scores);
-    snap_pass_kernel<1><<<(unsigned)(BH * ns), kSnapThreads, smem, st>>>(kb, qb, S, G, W, ns, ml, scores);
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    snap_tc_kernel<0><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(kb, qb, S, G, W, ns, ml, scores, status);
+    snap_tc_kernel<1><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(kb, qb, S, G, W, ns, ml, scores, status);
     snap_select_kernel<<<(unsigned)BH, kSelThreads, 0, st>>>(scores, pooled, S, W, keep, pool, idx_out);
     const int row_vec = kD * 2 / 16;  // bf16 rows
     const int rows_per_cta = 256 / row_vec;
