@@ -84,6 +84,8 @@ def _bind(lib):
     lib.oracle_recover_values.restype = None
     lib.oracle_think_prune.argtypes = [P, P, L, L, I, I, P, P, P]
     lib.oracle_think_prune.restype = None
+    lib.oracle_prune_topp.argtypes = [P, P, L, L, I, ctypes.c_float, I, P, P, P]
+    lib.oracle_prune_topp.restype = None
     return lib
 
 
@@ -130,6 +132,27 @@ def prune(k, qn, T: int, lib=None):
     vals = np.zeros((BH, S, T), np.float32)
     stats = np.zeros((BH, 4), np.float64)
     lib.oracle_prune(_ptr(k), _ptr(qn), BH, S, D, T, _ptr(mask), _ptr(vals), _ptr(stats))
+    return mask, vals, stats
+
+
+def prune_topp(k, qn, p: float, Tcap: int, lib=None):
+    """SparK-p pruning (reading R19): per token the shortest greedy prefix of
+    channels whose fp32 saliency mass reaches fp32(p * total), at most Tcap
+    channels.  k: [BH, S, D]; qn: [BH, D].  Returns (mask, vals [BH, S, Tcap]
+    with the kept values first and zeros after, stats) in the layouts of
+    prune()."""
+    lib = lib or load()
+    k = _f32(k)
+    qn = _f32(qn)
+    D = k.shape[-1]
+    S = k.shape[-2]
+    BH = int(np.prod(k.shape[:-2]))
+    nw = (D + 31) // 32
+    mask = np.zeros((BH, S, nw), np.uint32)
+    vals = np.zeros((BH, S, Tcap), np.float32)
+    stats = np.zeros((BH, 4), np.float64)
+    lib.oracle_prune_topp(_ptr(k), _ptr(qn), BH, S, D, ctypes.c_float(p), Tcap, _ptr(mask), _ptr(vals),
+                          _ptr(stats))
     return mask, vals, stats
 
 

@@ -152,6 +152,118 @@ void oracle_prune(const float *k, const float *qn, long BH, long S, int D,
 }
 
 /*
+ * SparK-p ([W] 5.2): instead of a fixed ratio, every token keeps the fewest
+ * channels whose cumulative saliency reaches a fraction p (0.99 in [W]) of
+ * the token's total.  Reading R19 (the pages fix neither the arithmetic of
+ * the cumulative sum nor the storage):
+ *   - channels are taken in the greedy order of [W] 3.1 (saliency desc,
+ *     lower channel first on ties, R3); the kept set is the shortest prefix
+ *     of that order whose mass reaches the target;
+ *   - the mass of a channel set is an fp32 sum in one fixed order: within
+ *     each block of 32 channels in ascending channel order starting from
+ *     +0, then the block sums pairwise, adjacent blocks first
+ *     ((B0 + B1) + (B2 + B3) for D = 128); channels outside the set add
+ *     nothing;
+ *   - target = fp32(p * mass(all channels)); "reaches" is >=, so a token
+ *     whose saliencies are all 0 keeps nothing;
+ *   - the cache has a capacity of Tcap values per token: a longer prefix is
+ *     cut to its first Tcap channels.  vals keeps the kept values in
+ *     ascending channel order in the first slots of the token's Tcap slots,
+ *     zeros after;
+ *   - statistics over the pruned entries as in oracle_prune.
+ */
+
+/* fp32 mass of the channels with in[j] != 0 (order of R19). */
+static float topp_mass(const float *w, const unsigned char *in, int D)
+{
+    float blk[64];
+    int nb = 0;
+    for (int b0 = 0; b0 < D; b0 += 32) {
+        float acc = 0.0f;
+        for (int j = b0; j < D && j < b0 + 32; ++j)
+            if (in[j])
+                acc = acc + w[j];
+        blk[nb++] = acc;
+    }
+    while (nb > 1) {
+        int m = 0;
+        for (int i = 0; i + 1 < nb; i += 2)
+            blk[m++] = blk[i] + blk[i + 1];
+        if (nb & 1)
+            blk[m++] = blk[nb - 1];
+        nb = m;
+    }
+    return nb ? blk[0] : 0.0f;
+}
+
+void oracle_prune_topp(const float *k, const float *qn, long BH, long S, int D, float p, int Tcap,
+                       uint32_t *mask, float *vals, double *stats)
+{
+    const int nw = (D + 31) / 32;
+    chan_score *order = (chan_score *)malloc(sizeof(chan_score) * (size_t)D);
+    unsigned char *in = (unsigned char *)malloc((size_t)D);
+    float *w = (float *)malloc(sizeof(float) * (size_t)D);
+    for (long bh = 0; bh < BH; ++bh) {
+        double n_pruned = 0.0, sw = 0.0, sw2 = 0.0;
+        for (long t = 0; t < S; ++t) {
+            const float *krow = k + (bh * S + t) * D;
+            for (int j = 0; j < D; ++j) {
+                w[j] = saliency(qn[bh * D + j], krow[j]);
+                order[j].w = w[j];
+                order[j].j = j;
+            }
+            qsort(order, (size_t)D, sizeof(chan_score), by_saliency_desc);
+            memset(in, 1, (size_t)D);
+            const float target = p * topp_mass(w, in, D);
+            /* shortest prefix: the mass of a prefix never decreases as it
+             * grows (each rounding is monotone), so bisect on its length */
+            int lo = 0, hi = D;  /* mass(prefix hi) >= target always holds */
+            while (lo < hi) {
+                const int mid = lo + (hi - lo) / 2;
+                memset(in, 0, (size_t)D);
+                for (int r = 0; r < mid; ++r)
+                    in[order[r].j] = 1;
+                if (topp_mass(w, in, D) >= target)
+                    hi = mid;
+                else
+                    lo = mid + 1;
+            }
+            const int n_keep = lo < Tcap ? lo : Tcap;
+            memset(in, 0, (size_t)D);
+            for (int r = 0; r < n_keep; ++r)
+                in[order[r].j] = 1;
+
+            uint32_t *mrow = mask + (bh * S + t) * nw;
+            for (int q = 0; q < nw; ++q)
+                mrow[q] = 0u;
+            float *vrow = vals + (bh * S + t) * (long)Tcap;
+            for (int r = 0; r < Tcap; ++r)
+                vrow[r] = 0.0f;
+            int slot = 0;
+            for (int j = 0; j < D; ++j) {
+                if (in[j]) {
+                    mrow[j / 32] |= 1u << (j % 32);
+                    vrow[slot] = krow[j];
+                    slot += 1;
+                } else {
+                    const double x = (double)w[j];
+                    n_pruned += 1.0;
+                    sw += x;
+                    sw2 += x * x;
+                }
+            }
+        }
+        stats[bh * 4 + 0] = n_pruned;
+        stats[bh * 4 + 1] = sw;
+        stats[bh * 4 + 2] = sw2;
+        stats[bh * 4 + 3] = (n_pruned > 0.0) ? sw / n_pruned : 0.0;
+    }
+    free(order);
+    free(in);
+    free(w);
+}
+
+/*
  * SparK-g ([W] 5.2): channels are split into g groups by importance and each
  * group has its own pruning rate, low-importance groups pruned harder
  * (g = 4 with rates (0.25, 0.5, 0.75, 1.0) in [W]).  Reading R15 (the pages
