@@ -30,9 +30,11 @@ SPARK_OP_PRUNE = 0
 SPARK_OP_DECODE = 1
 SPARK_OP_SNAPKV = 2
 SPARK_OP_THINK = 3
+SPARK_OP_TOPP = 4
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
-           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_prune_values", "spark_prune_think", "spark_decode_attn",
+           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_prune_values", "spark_prune_think", "spark_prune_topp", "spark_decode_attn",
+           "spark_decode_attn_topp",
            "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_selftest_wait_timeout", "spark_tail_append", "spark_device_status",
            "spark_status_str", "spark_snapkv_evict")
 
@@ -79,6 +81,11 @@ def lib():
         L.spark_prune_values.restype = I
         L.spark_prune_think.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P, Z, P]
         L.spark_prune_think.restype = I
+        L.spark_prune_topp.argtypes = [P, P, I, I, ctypes.c_float, ctypes.POINTER(spark_kcache), P, Z, P]
+        L.spark_prune_topp.restype = I
+        L.spark_decode_attn_topp.argtypes = [P, ctypes.POINTER(spark_kcache), P, P, P, I, I, I, I,
+                                             ctypes.c_ulonglong, P, P, Z, P]
+        L.spark_decode_attn_topp.restype = I
         L.spark_selftest_wait_timeout.argtypes = [P, I, P]
         L.spark_selftest_wait_timeout.restype = I
         L.spark_decode_attn_kv.argtypes = [P, ctypes.POINTER(spark_kcache), ctypes.POINTER(spark_kcache), P, P, I,
@@ -223,6 +230,27 @@ def spark_prune_think(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, kc: 
     rc = lib().spark_prune_think(_ptr(k), _ptr(q_obs), G, W, ctypes.byref(s), _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_prune_think")
+
+
+def spark_prune_topp(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, p: float, kc: KCache,
+                     ws: torch.Tensor, stream=None) -> None:
+    """SparK-p: per token the fewest greedy-order channels whose saliency mass
+    reaches p of the total, at most kc.T of them (see spark.h)."""
+    s = kc.struct()
+    rc = lib().spark_prune_topp(_ptr(k), _ptr(q_obs), G, W, ctypes.c_float(p), ctypes.byref(s), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_prune_topp")
+
+
+def spark_decode_attn_topp(q: torch.Tensor, kc: KCache, v: torch.Tensor, k_tail, v_tail, tail_cap: int,
+                           n_tail: int, G: int, out: torch.Tensor, ws: torch.Tensor,
+                           recovery: int = SPARK_F_DEGENERATE, seed: int = 0, stream=None) -> None:
+    """spark_decode_attn over a SparK-p cache (masks with at most kc.T bits)."""
+    s = kc.struct()
+    rc = lib().spark_decode_attn_topp(_ptr(q), ctypes.byref(s), _ptr(v), _ptr(k_tail), _ptr(v_tail), tail_cap,
+                                      n_tail, G, recovery, seed, _ptr(out), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_decode_attn_topp")
 
 
 def spark_selftest_wait_timeout(ws: torch.Tensor, limit_us: int, stream=None) -> None:

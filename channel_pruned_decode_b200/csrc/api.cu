@@ -14,6 +14,8 @@ cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, 
                           const void *k_tail, const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
                           unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st);
 cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws, cudaStream_t st);
+cudaError_t launch_prune_topp(const void *k, const void *q_obs, int G, int W, float p, const spark_kcache &kc,
+                              void *ws, cudaStream_t st);
 cudaError_t launch_think(const void *k, const void *q_obs, int G, int W, const spark_kcache &kc, void *ws,
                          cudaStream_t st);
 size_t think_workspace(long BH, int S);
@@ -125,6 +127,7 @@ size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D, int T,
     if (op == SPARK_OP_PRUNE) return round256(prune_workspace(BH, S));
     if (op == SPARK_OP_SNAPKV) return round256(snapkv_workspace(BH, S, 0));
     if (op == SPARK_OP_THINK) return round256(think_workspace(BH, S));
+    if (op == SPARK_OP_TOPP) return round256(topp_workspace(BH, S));
     if (op == SPARK_OP_DECODE) {
         if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
         // the geometry depends on the element size only through the stage
@@ -176,10 +179,27 @@ int spark_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_gr
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 
-int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, const void *k_tail,
-                      const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
-                      unsigned long long seed, float *out, void *workspace, size_t ws_bytes,
-                      void *stream) {
+int spark_prune_topp(const void *k, const void *q_obs, int G, int W, float p, const spark_kcache *out,
+                     void *workspace, size_t ws_bytes, void *stream) {
+    int rc = check_cache(out);
+    if (rc != SPARK_OK) return rc;
+    if (G < 1 || W < 1) return SPARK_ERR_ARG;
+    if (!(p >= 0.0f && p <= 1.0f)) return SPARK_ERR_ARG;
+    const long BH = (long)out->B * out->Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
+    if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < topp_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_prune_topp(k, q_obs, G, W, p, *out, workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+// argument checks and launch shared by spark_decode_attn and
+// spark_decode_attn_topp; `f` is the kernel's recovery selector
+static int decode_entry(const void *q, const spark_kcache *kc, const void *v, const void *k_tail,
+                        const void *v_tail, int tail_cap, int n_tail, int G, int recovery, int f,
+                        unsigned long long seed, float *out, void *workspace, size_t ws_bytes, void *stream) {
     int rc = check_cache(kc);
     if (rc != SPARK_OK) return rc;
     if (G != 1 && G != 2 && G != 4 && G != 8) return G < 1 ? SPARK_ERR_ARG : SPARK_ERR_UNSUPPORTED;
@@ -197,9 +217,28 @@ int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, cons
     const DecodeGeom geo = decode_geometry(BH, kc->S, kc->T, -1, es, G, num_sms());
     if (BH * (long)geo.units >= (1L << 31)) return SPARK_ERR_UNSUPPORTED;  // 32-bit item indices
     if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
-    cudaError_t e = launch_decode(q, *kc, v, nullptr, k_tail, v_tail, tail_cap, n_tail, G, recovery, seed, out,
+    cudaError_t e = launch_decode(q, *kc, v, nullptr, k_tail, v_tail, tail_cap, n_tail, G, f, seed, out,
                                   workspace, geo, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_decode_attn(const void *q, const spark_kcache *kc, const void *v, const void *k_tail,
+                      const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
+                      unsigned long long seed, float *out, void *workspace, size_t ws_bytes,
+                      void *stream) {
+    return decode_entry(q, kc, v, k_tail, v_tail, tail_cap, n_tail, G, recovery, recovery, seed, out, workspace,
+                        ws_bytes, stream);
+}
+
+int spark_decode_attn_topp(const void *q, const spark_kcache *kc, const void *v, const void *k_tail,
+                           const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
+                           unsigned long long seed, float *out, void *workspace, size_t ws_bytes,
+                           void *stream) {
+    // Gaussian / Exponential F walk all channels and read the kept values in
+    // order, which already handles fewer kept channels than slots
+    const int f = recovery == SPARK_F_DEGENERATE ? kRecoveryDegVar : recovery;
+    return decode_entry(q, kc, v, k_tail, v_tail, tail_cap, n_tail, G, recovery, f, seed, out, workspace,
+                        ws_bytes, stream);
 }
 
 size_t spark_workspace_bytes_kv(int B, int Hkv, int G, int S, int D, int T, int Tv, int n_tail) {

@@ -30,7 +30,9 @@
 //            mask from the top channel down (a queue of the non-empty mask
 //            words, one bfind and one bit clear per step, no branch) and
 //            accumulates q'_g (k_j - c_j) for the G heads of the group from
-//            the q' / c tables (q' = q * log2(e)/sqrt(D));
+//            the q' / c tables (q' = q * log2(e)/sqrt(D)); a SparK-p cache,
+//            whose masks may hold fewer bits than its T value slots, takes
+//            the same T steps with those past the token's count adding 0;
 //   softmax  warp max (integer REDUX on an order-preserving map) updates the
 //            running max; p = 2^(s - m) goes to shared memory;
 //   P.V      bf16: tensor cores -- the V tile is the B operand
@@ -513,6 +515,12 @@ __device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, 
 // spilling warps on the G = 4 workloads
 __host__ __device__ constexpr int dec_max_warps(int G) { return G > 2 ? 12 : kMaxWarps; }
 
+// kF: the recovery F (spark_recovery), or kDegVar: Degenerate F over a cache
+// whose masks may hold fewer bits than its T value slots (SparK-p: the kept
+// values fill the first slots of each token, zeros after).
+constexpr int kDegVar = kRecoveryDegVar;
+__host__ __device__ constexpr bool is_degenerate(int f) { return f == SPARK_F_DEGENERATE || f == kDegVar; }
+
 template <typename E, int G, int kF, bool kPV>
 __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArgs a) {
     static_assert(!kPV || (sizeof(E) == 2 && kF == SPARK_F_DEGENERATE), "packed values: bf16, Degenerate F");
@@ -642,7 +650,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         if (bh != tab_bh) {
             const E *q = static_cast<const E *>(a.q) + (size_t)bh * G * kD;
             const double mu = a.stats[bh * 4 + 3];
-            if constexpr (kF != SPARK_F_DEGENERATE) {
+            if constexpr (!is_degenerate(kF)) {
                 const double n = a.stats[bh * 4 + 0];
                 const double var = n > 0.0 ? a.stats[bh * 4 + 2] / n - mu * mu : 0.0;
                 f_mu = (float)mu;
@@ -656,7 +664,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 const int j = lane + 32 * i;
                 const float qnj = a.qn[bh * kD + j];
                 // Degenerate: c_j = mu / qn_j (folded into Qc); sampling: 1 / qn_j
-                const float c = qnj > 0.f ? (kF == SPARK_F_DEGENERATE ? (float)(mu / (double)qnj)
+                const float c = qnj > 0.f ? (is_degenerate(kF) ? (float)(mu / (double)qnj)
                                                                        : (float)(1.0 / (double)qnj))
                                           : 0.f;
                 ws.tabc[j] = c;
@@ -664,7 +672,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 for (int g = 0; g < G; ++g) {
                     const float qq = Elem<E>::to_f(q[(size_t)g * kD + j]) * kQScale;
                     ws.tabq[j * G + g] = qq;
-                    if constexpr (kF == SPARK_F_DEGENERATE) part[g] = fmaf(qq, c, part[g]);
+                    if constexpr (is_degenerate(kF)) part[g] = fmaf(qq, c, part[g]);
                 }
             }
 #pragma unroll
@@ -740,7 +748,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             float s[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) s[g] = 0.f;
-            if constexpr (kF != SPARK_F_DEGENERATE) {
+            if constexpr (!is_degenerate(kF)) {
                 // every channel: kept -> stored value, pruned -> sampled score / qn_j
                 const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
                 const uint32_t wds[4] = {mw.x, mw.y, mw.z, mw.w};
@@ -776,6 +784,13 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 uint32_t bq = 0x00204060u;  // bases 96, 64, 32, 0 from the low byte up
                 queue_nonempty(cur, n1, n2, n3, bq);
                 const E *vp = ws.svals(st) + lane + (a.T - 1) * kWT;
+                // kDegVar: this token's kept count; value i from the top
+                // sits in slot cnt - 1 - i, steps past cnt add nothing
+                int cnt = a.T;
+                if constexpr (kF == kDegVar) {
+                    cnt = min(__popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w), a.T);
+                    vp = ws.svals(st) + lane;
+                }
                 float2 s2[G / 2 > 0 ? G / 2 : 1];  // head pairs: packed fp32x2 FMAs
 #pragma unroll
                 for (int g = 0; g < (G / 2 > 0 ? G / 2 : 1); ++g) s2[g] = make_float2(0.f, 0.f);
@@ -789,7 +804,13 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     n1 = e ? n2 : n1;
                     n2 = e ? n3 : n2;
                     bq = e ? (bq >> 8) : bq;
-                    const float x = Elem<E>::to_f(vp[-i * kWT]) - ws.tabc[j];
+                    float x;
+                    if constexpr (kF == kDegVar) {
+                        const int r = cnt - 1 - i;
+                        x = r >= 0 ? Elem<E>::to_f(vp[max(r, 0) * kWT]) - ws.tabc[j] : 0.f;
+                    } else {
+                        x = Elem<E>::to_f(vp[-i * kWT]) - ws.tabc[j];
+                    }
                     QVec<G> qv;
                     qv.load(ws.tabq + j * G);
                     if constexpr (G % 2 == 0) {
@@ -983,6 +1004,7 @@ static cudaError_t dispatch_f(const DecArgs &a, const DecodeGeom &geo, int G, in
     case SPARK_F_DEGENERATE: return dispatch_g<E, SPARK_F_DEGENERATE>(a, geo, G, out, st);
     case SPARK_F_GAUSSIAN: return dispatch_g<E, SPARK_F_GAUSSIAN>(a, geo, G, out, st);
     case SPARK_F_EXPONENTIAL: return dispatch_g<E, SPARK_F_EXPONENTIAL>(a, geo, G, out, st);
+    case kDegVar: return dispatch_g<E, kDegVar>(a, geo, G, out, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -6,7 +6,7 @@
 // per-token unstructured mask) and 3.3 step 1 (the cache stores the pruned
 // key, the channel mask and the saliency statistics).
 //
-// Three launches on the caller's stream:
+// spark_prune makes three launches on the caller's stream:
 //   qnorm_kernel   one CTA per (row, kv head), one thread per channel: the
 //                  fp64 sum of squares over the G*W window rows of the group,
 //                  rounded once to fp32.
@@ -28,7 +28,9 @@
 //                  fp64 per-lane accumulators and one fp64 partial per CTA.
 //   stats_kernel   fixed-order fp64 sum of the CTA partials per head, then
 //                  N = S*(D-T) and mu_pruned = sum w / N.
-// All reductions have a fixed order, so reruns are bit-identical.
+// All reductions have a fixed order, so reruns are bit-identical.  SparK-g
+// uses prune_kernel with per-group selections; SparK-p (per-token top-p
+// selection) has its own kernel, prune_topp_kernel, described with it below.
 #include "spark_internal.cuh"
 
 #include <cuda_fp16.h>
@@ -658,6 +660,361 @@ cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W,
     for (int q = 0; q < n_groups; ++q) ga.T[q] = group_T[q];
     if (kc.dtype == SPARK_BF16) return launch_prune_t<__nv_bfloat16>(k, q_obs, G, W, kc, ws, st, &ga);
     return launch_prune_t<float>(k, q_obs, G, W, kc, ws, st, &ga);
+}
+
+// ---------------------------------------------------------------------------
+// SparK-p ("KV Cache 还能再砍一刀：SparK ..." section 5.2): every token keeps
+// the fewest channels, taken in the greedy order of section 3.1 (saliency
+// desc, lower channel first), whose saliency mass reaches p of its total,
+// at most Tcap of them.  The library's arithmetic for the mass of a channel
+// set (the pages leave it open): each lane adds its 32 channels in
+// ascending order in fp32 from +0, then the quad adds
+// (lane 0 + lane 1) + (lane 2 + lane 3); fp32 addition is commutative, so
+// every lane of the quad holds the same bits.  target = fp32(p * total).
+//
+// A set {16-bit key >= P} is a threshold set of the exact keys (the 16-bit
+// key is monotone in them), hence a greedy prefix, and its mass M(P) does
+// not increase with P (each rounding is monotone).  The search finds the
+// largest level lo with M(lo) >= target by binary lifting, tracking the
+// lowest failing level hi: over [0, 2^15) for the first token of a quad
+// (M(0) is the total, nothing reaches 2^15), otherwise over a 2^11-level
+// window around a running estimate, redone over [0, 2^15) when the window
+// did not bracket lo.  It leaves early once {key >= lo} and {key >= hi}
+// differ by one channel for every quad of the warp: that channel ends the
+// prefix.  Otherwise the band between them is added one channel at a time
+// in greedy order (exact keys desc, lower channel first) until the mass
+// reaches the target.  A prefix longer than Tcap is replaced by the top-Tcap
+// set (select_top_t).
+
+// this lane's channels whose 16-bit key is >= P (bit i = channel i)
+__device__ __forceinline__ uint32_t ge16_bits(const uint32_t (&kp)[16], uint32_t P) {
+    const uint32_t p2 = P * 0x10001u;
+    uint32_t m = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m |= hge2_mask(kp[i], p2) & (0x00010001u << i);
+    return m;
+}
+
+// fp32 mass of the quad's channels in m, in the order described above
+__device__ __forceinline__ float quad_mass(const uint32_t (&key)[32], uint32_t m) {
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc = ((m >> i) & 1u) ? __fadd_rn(acc, __uint_as_float(key[i])) : acc;
+    const float a = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
+    return __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
+}
+
+// search state of one quad: M(lo) >= target > M(hi) once both are known
+struct TopPBracket {
+    uint32_t lo, hi;
+    int clo, chi;    // channel counts of {key >= lo}, {key >= hi}
+    bool klo, khi;   // lo / hi established by a probe (or known bounds)
+};
+
+// Binary lifting of lo over [lo, lo + 2^K) for the active quads; every loop
+// trip is warp-uniform (the shuffles of quad_sum / quad_mass see all lanes).
+__device__ __forceinline__ void topp_lift(const uint32_t (&key)[32], const uint32_t (&kp)[16], float target,
+                                          int K, bool active, TopPBracket &b) {
+    bool done = !active || (b.klo && b.khi && b.clo - b.chi <= 1);
+    for (int bit = K - 1; bit >= 0; --bit) {
+        if (__all_sync(0xffffffffu, done)) break;
+        const uint32_t P = b.lo + (1u << bit);
+        const uint32_t m = ge16_bits(kp, P);
+        const int c = quad_sum(__popc(m));
+        const float M = quad_mass(key, m);
+        if (!done) {
+            if (M >= target) {
+                b.lo = P;
+                b.clo = c;
+                b.klo = true;
+            } else {
+                b.hi = P;
+                b.chi = c;
+                b.khi = true;
+            }
+            done = b.klo && b.khi && b.clo - b.chi <= 1;
+        }
+    }
+}
+
+// the whole 16-bit key range: M(0) = total >= target, no key reaches 2^15
+__device__ __forceinline__ void topp_full_range(TopPBracket &b) {
+    b.lo = 0u;
+    b.hi = 0x8000u;
+    b.clo = kD;
+    b.chi = 0;
+    b.klo = b.khi = true;
+}
+
+template <typename E>
+__global__ void __launch_bounds__(kPruneThreads, 3)
+    prune_topp_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
+                      E *__restrict__ vals, double *__restrict__ partial, int S, int Tcap, int n_chunks, int gpc,
+                      float p) {
+    using Raw = typename RawT<E>::type;
+    __shared__ __align__(16) Raw vtile[kPruneThreads / 32][kD * 8];
+    __shared__ double red[3][kPruneThreads / 32];
+    __shared__ uint32_t qmax[kPruneThreads / 32];
+    __shared__ __align__(16) float qs[4 * 36];
+
+    const long bh = blockIdx.x / n_chunks;
+    const int chunk = blockIdx.x % n_chunks;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int s = lane & 3;
+    const int tq = lane >> 2;
+    const int tl = warp * 8 + tq;
+    const long S32 = ((long)S + 31) / 32 * 32;
+
+    {
+        const float q = __ldg(qn + bh * kD + tid);
+        qs[(tid >> 5) * 36 + (tid & 31)] = q;
+        const uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(q) & 0x7fffffffu);
+        if (lane == 0) qmax[warp] = mx;
+    }
+    __syncthreads();
+    float scale = 1.f, inv_scale = 1.f;
+    {
+        uint32_t mx = qmax[0];
+#pragma unroll
+        for (int w = 1; w < kPruneThreads / 32; ++w) mx = max(mx, qmax[w]);
+        const int e = (int)(mx >> 23);
+        if (e > 0 && e < 255) {
+            const int x = min(max(127 - e, -64), 64);
+            scale = __uint_as_float((uint32_t)(127 + x) << 23);
+            inv_scale = __uint_as_float((uint32_t)(127 - x) << 23);
+        }
+    }
+    const float2 scale2 = make_float2(scale, scale);
+
+    Raw *vt = vtile[warp];
+    uint32_t tau = 0u;  // running estimate of the quad's mass level
+    double acc_w = 0.0, acc_w2 = 0.0, acc_n = 0.0;
+    const long g_first = (long)chunk * gpc;
+    const E *krow = k + ((size_t)bh * S + g_first * 32 + tl) * kD + 32 * s;
+    E *gvals = vals + (size_t)bh * S32 * Tcap + (size_t)g_first * 32 * Tcap;
+
+    auto group = [&](int gi, KSlice<E> &cur, KSlice<E> &nxt) {
+        const long t = (g_first + gi) * 32 + tl;
+        const bool valid = t < S;
+        if (gi + 1 < gpc && t + 32 < S) nxt.load(krow + (size_t)(gi + 1) * 32 * kD);
+        else nxt.zero();
+
+        uint32_t key[32];
+        float2 wsc[16];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 q4 = *reinterpret_cast<const float4 *>(qs + s * 36 + 4 * c);
+            const float2 w01 = __fmul2_rn(make_float2(q4.x, q4.y), cur.abs_pair(2 * c));
+            const float2 w23 = __fmul2_rn(make_float2(q4.z, q4.w), cur.abs_pair(2 * c + 1));
+            key[4 * c + 0] = __float_as_uint(w01.x);
+            key[4 * c + 1] = __float_as_uint(w01.y);
+            key[4 * c + 2] = __float_as_uint(w23.x);
+            key[4 * c + 3] = __float_as_uint(w23.y);
+            wsc[2 * c] = __fmul2_rn(w01, scale2);
+            wsc[2 * c + 1] = __fmul2_rn(w23, scale2);
+        }
+        uint32_t kp[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float a = (i & 1) ? wsc[i >> 1].y : wsc[i >> 1].x;
+            const float b = (i & 1) ? wsc[8 + (i >> 1)].y : wsc[8 + (i >> 1)].x;
+            const __half2 h = __floats2half2_rn(a, b);
+            kp[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+
+        // target = p * total; a token with target 0 (p = 0 or no saliency)
+        // keeps nothing
+        const float total = quad_mass(key, 0xffffffffu);
+        const float target = __fmul_rn(p, total);
+        const bool active = valid && target > 0.f && Tcap > 0;
+
+        TopPBracket b;
+        if (gi == 0) {
+            topp_full_range(b);
+        } else {
+            b.lo = min(tau > 1024u ? tau - 1024u : 0u, kTop16 - 2048u);
+            b.hi = b.lo + 2048u;
+            b.clo = kD;
+            b.chi = 0;
+            b.klo = b.khi = false;
+        }
+        topp_lift(key, kp, target, gi == 0 ? 15 : 11, active, b);
+        const bool suspect = active && !(b.klo && b.khi);
+        if (__any_sync(0xffffffffu, suspect)) {
+            if (suspect) topp_full_range(b);
+            topp_lift(key, kp, target, 15, suspect, b);
+        }
+
+        uint32_t m = active ? ge16_bits(kp, b.lo) : 0u;
+        const bool band = active && b.clo - b.chi >= 2;
+        if (__any_sync(0xffffffffu, band)) {
+            // the prefix {key >= hi} falls short; add the band's channels in
+            // greedy order until the mass reaches the target
+            uint32_t mA = ge16_bits(kp, min(b.hi, kTop16));
+            uint32_t mB = band ? (m & ~mA) : 0u;
+            bool open = band;
+            for (int it = 0; it < kD && __any_sync(0xffffffffu, open); ++it) {
+                uint32_t bk = 0u;
+                int bi = -1;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool take = ((mB >> i) & 1u) && (bi < 0 || key[i] > bk);
+                    bk = take ? key[i] : bk;
+                    bi = take ? i : bi;
+                }
+                // quad arg-max of (exact key desc, channel asc)
+                uint32_t wk = bk;
+                int wc = bi < 0 ? 4 * kD : 32 * s + bi;
+#pragma unroll
+                for (int o = 1; o <= 2; o <<= 1) {
+                    const uint32_t ok = __shfl_xor_sync(0xffffffffu, wk, o);
+                    const int oc = __shfl_xor_sync(0xffffffffu, wc, o);
+                    const bool better = oc < 4 * kD && (wc >= 4 * kD || ok > wk || (ok == wk && oc < wc));
+                    wk = better ? ok : wk;
+                    wc = better ? oc : wc;
+                }
+                if (open && wc < 4 * kD && (wc >> 5) == s) {
+                    mA |= 1u << (wc & 31);
+                    mB &= ~(1u << (wc & 31));
+                }
+                const float M = quad_mass(key, mA);
+                if (open && (M >= target || wc >= 4 * kD)) open = false;
+            }
+            m = band ? mA : m;
+        }
+        const int n_keep = quad_sum(__popc(m));
+        if (active) tau = gi == 0 ? b.lo : (uint32_t)((int)tau + (((int)b.lo - (int)tau) >> 1));
+
+        // capacity: a longer prefix becomes the top-Tcap set
+        const bool cap = active && n_keep > Tcap;
+        if (__any_sync(0xffffffffu, cap)) {
+            const uint32_t base = min(b.lo, kTop16 - (1u << kLiftCold));
+            uint32_t lo_cap;
+            const uint32_t mc = select_top_t(key, kp, Tcap, s, inv_scale, base, kLiftCold, !cap, 0xffffffffu, lo_cap);
+            m = cap ? mc : m;
+        }
+        if (valid) mask[((size_t)bh * S + t) * kMaskWords + s] = m;
+
+        // zero the warp's Tcap staging rows, then stage the kept values
+        {
+            constexpr int kRowB = 8 * (int)sizeof(Raw);  // bytes of one staging row
+            uint4 *z = reinterpret_cast<uint4 *>(vt);
+            for (int c = lane; c < Tcap * kRowB / 16; c += 32) z[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+        Raw *dst = vt + quad_excl_scan(__popc(m), s) * 8 + tq;
+        float sw = 0.f, sw2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if ((m >> i) & 1u) {
+                *dst = (Raw)cur.raw(i);
+                dst += 8;
+            } else {
+                const float w = __uint_as_float(key[i]);
+                sw = __fadd_rn(sw, w);
+                sw2 = __fmaf_rn(w, w, sw2);
+            }
+        }
+        if (valid) {
+            acc_w = __dadd_rn(acc_w, (double)sw);
+            acc_w2 = __dadd_rn(acc_w2, (double)sw2);
+            acc_n = __dadd_rn(acc_n, (double)(32 - __popc(m)));
+        }
+        __syncwarp();
+        constexpr int kParts = (int)sizeof(E) / 2;
+        unsigned char *g = reinterpret_cast<unsigned char *>(gvals + (size_t)gi * 32 * Tcap + warp * 8);
+        const unsigned char *src = reinterpret_cast<const unsigned char *>(vt);
+        for (int c = lane; c < Tcap * kParts; c += 32) {
+            const int row = c / kParts, part = c % kParts;
+            __stcs(reinterpret_cast<uint4 *>(g + (size_t)row * 32 * sizeof(E) + part * 16),
+                   *reinterpret_cast<const uint4 *>(src + row * 8 * sizeof(E) + part * 16));
+        }
+        __syncwarp();
+    };
+
+    KSlice<E> ka, kb;
+    if (g_first * 32 + tl < S) ka.load(krow);
+    else ka.zero();
+    for (int gi = 0; gi < gpc; gi += 2) {
+        if ((g_first + gi) * 32 >= S) break;
+        group(gi, ka, kb);
+        if ((g_first + gi + 1) * 32 >= S) break;
+        group(gi + 1, kb, ka);
+    }
+
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        acc_w = __dadd_rn(acc_w, __shfl_xor_sync(0xffffffffu, acc_w, o));
+        acc_w2 = __dadd_rn(acc_w2, __shfl_xor_sync(0xffffffffu, acc_w2, o));
+        acc_n = __dadd_rn(acc_n, __shfl_xor_sync(0xffffffffu, acc_n, o));
+    }
+    if (lane == 0) {
+        red[0][warp] = acc_w;
+        red[1][warp] = acc_w2;
+        red[2][warp] = acc_n;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double a = 0.0, b2 = 0.0, n = 0.0;
+        for (int i = 0; i < kPruneThreads / 32; ++i) {
+            a = __dadd_rn(a, red[0][i]);
+            b2 = __dadd_rn(b2, red[1][i]);
+            n = __dadd_rn(n, red[2][i]);
+        }
+        partial[((size_t)bh * n_chunks + chunk) * 3 + 0] = a;
+        partial[((size_t)bh * n_chunks + chunk) * 3 + 1] = b2;
+        partial[((size_t)bh * n_chunks + chunk) * 3 + 2] = n;
+    }
+}
+
+// SparK-p statistics: the pruned count is data-dependent, summed like the
+// saliency sums (exact: integers below 2^53).
+__global__ void stats_topp_kernel(const double *__restrict__ partial, int n_chunks, long BH,
+                                  double *__restrict__ stats) {
+    const long bh = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (bh >= BH) return;
+    double a = 0.0, b = 0.0, n = 0.0;
+    for (int c = lane; c < n_chunks; c += 32) {
+        a = __dadd_rn(a, partial[((size_t)bh * n_chunks + c) * 3 + 0]);
+        b = __dadd_rn(b, partial[((size_t)bh * n_chunks + c) * 3 + 1]);
+        n = __dadd_rn(n, partial[((size_t)bh * n_chunks + c) * 3 + 2]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a = __dadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+        b = __dadd_rn(b, __shfl_xor_sync(0xffffffffu, b, o));
+        n = __dadd_rn(n, __shfl_xor_sync(0xffffffffu, n, o));
+    }
+    if (lane == 0) {
+        stats[bh * 4 + 0] = n;
+        stats[bh * 4 + 1] = a;
+        stats[bh * 4 + 2] = b;
+        stats[bh * 4 + 3] = n > 0.0 ? a / n : 0.0;
+    }
+}
+
+template <typename E>
+static cudaError_t launch_prune_topp_t(const void *k, const void *q_obs, int G, int W, float p,
+                                       const spark_kcache &kc, void *ws, cudaStream_t st) {
+    const long BH = (long)kc.B * kc.Hkv;
+    if (BH == 0) return cudaSuccess;
+    double *partial = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
+    qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn);
+    const int gpc = prune_groups_per_cta(BH, kc.S);
+    const int nch = prune_chunks(kc.S, gpc);
+    if (nch > 0)
+        prune_topp_kernel<E><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+            static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T, nch, gpc,
+            p);
+    stats_topp_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.stats);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prune_topp(const void *k, const void *q_obs, int G, int W, float p, const spark_kcache &kc,
+                              void *ws, cudaStream_t st) {
+    if (kc.dtype == SPARK_BF16) return launch_prune_topp_t<__nv_bfloat16>(k, q_obs, G, W, p, kc, ws, st);
+    return launch_prune_topp_t<float>(k, q_obs, G, W, p, kc, ws, st);
 }
 
 // ---------------------------------------------------------------------------

@@ -41,7 +41,16 @@ inline size_t prune_workspace(long BH, int S) {
     return kWsHeader + (size_t)BH * (size_t)prune_chunks(S) * 2 * sizeof(double);
 }
 
+// SparK-p: a third partial per chunk (the data-dependent pruned count)
+inline size_t topp_workspace(long BH, int S) {
+    return kWsHeader + (size_t)BH * (size_t)prune_chunks(S) * 3 * sizeof(double);
+}
+
 // ---------------------------------------------------------------- decode
+// recovery selector of the decode kernel beyond spark_recovery: Degenerate F
+// over a SparK-p cache (masks may hold fewer bits than the T value slots)
+constexpr int kRecoveryDegVar = 3;
+
 // Each warp of a persistent CTA is an independent flash-decoding worker.  Its
 // ring of shared-memory stages holds the mask and kept values of one 32-token
 // tile each; the tile's dense V rows go straight to registers.

@@ -65,7 +65,9 @@ typedef enum {
     SPARK_F_EXPONENTIAL = 2   /* w~ ~ Exp(1/mu) (mean mu)                     */
 } spark_recovery;
 
-typedef enum { SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1, SPARK_OP_SNAPKV = 2, SPARK_OP_THINK = 3 } spark_op;
+typedef enum {
+    SPARK_OP_PRUNE = 0, SPARK_OP_DECODE = 1, SPARK_OP_SNAPKV = 2, SPARK_OP_THINK = 3, SPARK_OP_TOPP = 4
+} spark_op;
 
 /*
  * The packed key cache of [W] 3.3 step 1 / Fig. 3: per token the kept key
@@ -160,6 +162,40 @@ SPARK_API int spark_prune(const void *k, const void *q_obs, int G, int W,
 SPARK_API int spark_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups,
                                   const int *group_T, const spark_kcache *out, void *workspace,
                                   size_t ws_bytes, void *stream);
+
+/*
+ * SparK-p ([W] 5.2: instead of a fixed ratio, each token keeps the fewest
+ * channels whose cumulative saliency reaches p -- 99 % in [W] -- of its
+ * total).  Same arguments, saliencies w and statistics as spark_prune, plus
+ *   p     fraction in [0, 1] (SPARK_ERR_ARG otherwise, NaN included)
+ *   out   out->T is the capacity Tcap: the number of value slots per token
+ * Per token, channels are ordered by (w desc, channel asc); the kept set is
+ * the shortest prefix of that order whose mass reaches fp32(p * total), cut
+ * to its first Tcap channels when longer.  The library's arithmetic for the
+ * mass of a channel set (the pages leave it open): an fp32 sum, within each
+ * block of 32 channels in ascending channel order from +0, then
+ * (B0 + B1) + (B2 + B3); "reaches" is >=, so a token whose saliencies are
+ * all 0 (or p = 0) keeps nothing.  The mask holds the kept channels (at most
+ * Tcap bits); the kept values fill the first slots of the token's Tcap slots
+ * in ascending channel order (layout of spark_kcache with T = Tcap), the
+ * other slots are 0.  stats: N = number of pruned entries (data-dependent),
+ * sum w, sum w^2 over them, mu = sum w / N.  Decode this cache with
+ * spark_decode_attn_topp.  Workspace: spark_workspace_bytes(SPARK_OP_TOPP,
+ * ...).
+ */
+SPARK_API int spark_prune_topp(const void *k, const void *q_obs, int G, int W, float p,
+                               const spark_kcache *out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Decode attention over a SparK-p cache (spark_prune_topp): exactly
+ * spark_decode_attn (same arguments, workspace and results), for a cache
+ * whose masks may hold fewer bits than its T value slots, the kept values
+ * first.  Degenerate F adds no term for the empty slots.
+ */
+SPARK_API int spark_decode_attn_topp(const void *q, const spark_kcache *kc, const void *v,
+                                     const void *k_tail, const void *v_tail, int tail_cap,
+                                     int n_tail, int G, int recovery, unsigned long long seed,
+                                     float *out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * Value-channel pruning ([W] 4.4: the value cache is pruned too, with a

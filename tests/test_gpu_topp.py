@@ -1,0 +1,156 @@
+"""GPU parity of SparK-p (spark_prune_topp / spark_decode_attn_topp) against
+the oracle's prune_topp on the same seeded inputs.  The mass of a channel set
+is defined in fp32 in one fixed order on both sides, so masks, kept values
+(zero padding included) and the pruned count are compared bit for bit, the
+saliency sums to fp32-partial rounding, and decode within the attention
+tolerance.  Full-size heads are checked on sampled tokens."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from channel_pruned_decode_b200 import (KCache, spark_decode_attn, spark_decode_attn_topp, spark_prune_topp,
+                                        spark_workspace_bytes, workspace, SPARK_F_GAUSSIAN, SPARK_OP_DECODE,
+                                        SPARK_OP_TOPP)
+from channel_pruned_decode_b200.synth import WORKLOADS, make_decode_step, make_prefill, scaled
+from tests._parity import assert_out_close, mask_np, run_prune, to_np, unpack_vals
+from tests.test_gpu_parity import STATS_RTOL
+
+pytestmark = pytest.mark.gpu
+D = 128
+DEV = "cuda"
+
+
+def run_topp(k, q_obs, G, W, p, Tcap):
+    R, Hkv, S, _ = k.shape
+    kc = KCache.empty(R, Hkv, S, D, Tcap, k.dtype, device=k.device)
+    ws = workspace(spark_workspace_bytes(SPARK_OP_TOPP, R, Hkv, G, S, D, Tcap, 0))
+    spark_prune_topp(k, q_obs, G, W, p, kc, ws)
+    torch.cuda.synchronize()
+    return kc
+
+
+def check_topp(kc, k_np, q_np, G, p, what):
+    BH, S, Tcap = kc.B * kc.Hkv, kc.S, kc.T
+    qn = oracle.qnorm(q_np.reshape(BH * G, -1, D), G)
+    assert np.array_equal(kc.qn.cpu().numpy().reshape(BH, D).view(np.uint32), qn.view(np.uint32)), what
+    m_o, v_o, s_o = oracle.prune_topp(k_np.reshape(BH, S, D), qn, p, Tcap)
+    s_g = kc.stats.cpu().numpy().reshape(BH, 4)
+    assert np.array_equal(s_g[:, 0], s_o[:, 0]), f"{what}: pruned count"
+    np.testing.assert_allclose(s_g[:, 1:], s_o[:, 1:], rtol=STATS_RTOL, atol=0, err_msg=what)
+    if S == 0:
+        return qn, m_o, v_o, s_o
+    m_g = mask_np(kc)
+    bad = np.argwhere(np.any(m_g != m_o, axis=-1))
+    assert len(bad) == 0, f"{what}: {len(bad)} tokens differ, first {bad[:4].tolist()}"
+    if Tcap > 0:
+        assert np.array_equal(unpack_vals(kc).view(np.uint32), v_o.view(np.uint32)), f"{what}: vals"
+    return qn, m_o, v_o, s_o
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("S,p,Tcap", [(1, 0.99, 128), (33, 0.99, 128), (1000, 0.99, 128), (2049, 0.9, 96),
+                                      (700, 0.99, 40), (300, 0.5, 128), (257, 1.0, 128), (129, 0.0, 64),
+                                      (100, 0.99, 0), (0, 0.99, 64)])
+def test_topp_parity_and_decode(dtype, S, p, Tcap):
+    G = 4
+    wl = scaled(WORKLOADS["tiny"], S=S, G=G, Hkv=3, dtype="f32" if dtype == torch.float32 else "bf16",
+                seed=700 + S + Tcap)
+    pre = make_prefill(wl, DEV)
+    what = f"topp S={S} p={p} Tcap={Tcap} {dtype}"
+    kc = run_topp(pre["k"], pre["q_obs"], G, wl.W, p, Tcap)
+    qn, m, vals, st = check_topp(kc, to_np(pre["k"]), to_np(pre["q_obs"]), G, p, what)
+    BH = wl.rows * wl.Hkv
+    q = make_decode_step(wl, 1, DEV)["q"]
+    out = torch.empty((wl.rows, wl.Hkv * G, D), dtype=torch.float32, device=DEV)
+    ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, G, S, D, Tcap, 0))
+    spark_decode_attn_topp(q, kc, pre["v"], None, None, 0, 0, G, out, ws)
+    torch.cuda.synchronize()
+    o_ref = oracle.decode(to_np(q).reshape(BH * G, D), m, vals, qn, st, to_np(pre["v"]).reshape(BH, S, D), G=G)
+    assert_out_close(out.cpu().numpy().reshape(BH * G, D), o_ref, what + " decode")
+
+
+def test_topp_extreme_tokens():
+    """All-zero tokens, single dominant channels, saliencies spanning many
+    octaves and exact ties."""
+    G, S, Hkv = 2, 512, 2
+    wl = scaled(WORKLOADS["tiny"], S=S, G=G, Hkv=Hkv, dtype="bf16", seed=91)
+    pre = make_prefill(wl, DEV)
+    k = pre["k"].float()
+    k[0, 0, 0:40] = 0.0                                  # no saliency at all
+    k[0, 0, 40:80] = 0.0
+    k[0, 0, 40:80, 7] = 3.0                              # one channel holds everything
+    k[0, 1, 0:64] *= torch.logspace(-20, 20, D, base=2.0, device=DEV)   # many octaves
+    k[0, 1, 64:128] = torch.round(k[0, 1, 64:128] * 2) / 2              # many exact ties
+    k = k.to(torch.bfloat16)
+    for p, Tcap in ((0.99, 128), (0.999, 50), (1.0, 128)):
+        kc = run_topp(k, pre["q_obs"], G, wl.W, p, Tcap)
+        check_topp(kc, to_np(k), to_np(pre["q_obs"]), G, p, f"extreme p={p} Tcap={Tcap}")
+
+
+def test_topp_decode_gaussian_and_tail():
+    """Sampling F and the dense tail over a SparK-p cache."""
+    G = 4
+    wl = scaled(WORKLOADS["tiny"], S=777, G=G, Hkv=2, dtype="bf16", seed=44)
+    pre = make_prefill(wl, DEV)
+    kc = run_topp(pre["k"], pre["q_obs"], G, wl.W, 0.99, 100)
+    qn, m, vals, st = check_topp(kc, to_np(pre["k"]), to_np(pre["q_obs"]), G, 0.99, "topp tail")
+    BH = wl.rows * wl.Hkv
+    cap, n_tail = 16, 5
+    kt = torch.randn((wl.rows, wl.Hkv, cap, D), device=DEV).to(torch.bfloat16)
+    vt = torch.randn((wl.rows, wl.Hkv, cap, D), device=DEV).to(torch.bfloat16)
+    q = make_decode_step(wl, 2, DEV)["q"]
+    for rec in (0, SPARK_F_GAUSSIAN):
+        out = torch.empty((wl.rows, wl.Hkv * G, D), dtype=torch.float32, device=DEV)
+        ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, G, wl.S, D, kc.T, cap))
+        spark_decode_attn_topp(q, kc, pre["v"], kt, vt, cap, n_tail, G, out, ws, recovery=rec, seed=5)
+        torch.cuda.synchronize()
+        args = (to_np(q).reshape(BH * G, D), m, vals, qn, st, to_np(pre["v"]).reshape(BH, wl.S, D),
+                to_np(kt).reshape(BH, cap, D), to_np(vt).reshape(BH, cap, D), n_tail, G)
+        o_ref = oracle.decode(*args) if rec == 0 else oracle.decode_f(*args, mode=rec, seed=5)
+        assert_out_close(out.cpu().numpy().reshape(BH * G, D), o_ref, f"topp decode F={rec}")
+
+
+def test_topp_decode_equals_plain_decode_on_full_masks():
+    """On a plain SparK cache (exactly T bits per token) the SparK-p decode
+    takes the same arithmetic steps as spark_decode_attn."""
+    wl = scaled(WORKLOADS["llama1l"], S=4096)
+    pre = make_prefill(wl, DEV)
+    kc = run_prune(pre["k"], pre["q_obs"], wl.G, wl.W, 64)
+    q = make_decode_step(wl, 0, DEV)["q"]
+    outs = []
+    for fn in (spark_decode_attn, spark_decode_attn_topp):
+        out = torch.empty((wl.rows, wl.Hkv * wl.G, D), dtype=torch.float32, device=DEV)
+        ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, wl.G, wl.S, D, 64, 0))
+        fn(q, kc, pre["v"], None, None, 0, 0, wl.G, out, ws)
+        torch.cuda.synchronize()
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_topp_full_size_sampled():
+    """One layer of the long-context workload (8 heads x 131072 tokens) in
+    the launch configuration of the benchmark: sampled tokens against the
+    oracle, every mask within the capacity."""
+    wl = scaled(WORKLOADS["long"], L=1)
+    pre = make_prefill(wl, DEV)
+    Tcap = 96
+    kc = run_topp(pre["k"], pre["q_obs"], wl.G, wl.W, 0.99, Tcap)
+    BH, S = wl.rows * wl.Hkv, wl.S
+    qn = oracle.qnorm(to_np(pre["q_obs"]).reshape(BH * wl.G, -1, D), wl.G)
+    m_g = mask_np(kc)
+    pc = np.zeros(m_g.shape[:2], np.int64)
+    for wd in range(4):
+        x = m_g[..., wd].astype(np.uint64)
+        pc += np.array([bin(int(v)).count("1") for v in x.ravel()]).reshape(x.shape)
+    assert pc.max() <= Tcap
+    st = kc.stats.cpu().numpy().reshape(BH, 4)
+    assert np.array_equal(st[:, 0], (D - pc).sum(1).astype(np.float64))
+    rng = np.random.default_rng(1)
+    vals_g = unpack_vals(kc)
+    k_np = to_np(pre["k"]).reshape(BH, S, D)
+    for bh in range(BH):
+        ts = np.sort(rng.choice(S, 256, replace=False))
+        m_o, v_o, _ = oracle.prune_topp(k_np[bh, ts][None], qn[bh:bh + 1], 0.99, Tcap)
+        assert np.array_equal(m_g[bh, ts], m_o[0]), f"head {bh}"
+        assert np.array_equal(vals_g[bh, ts].view(np.uint32), v_o[0].view(np.uint32)), f"head {bh}"
