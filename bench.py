@@ -361,8 +361,9 @@ def run_variants(job, wl, stream, peak, peak_kind, iters=5):
     """Method variants on the same prompt, timed outside the step with CUDA
     events on the launching stream: SparK-g grouped pruning with the pages'
     g = 4 rates (0.25, 0.5, 0.75, 1.0), the ThinK structured comparator at the
-    same T (prune + decode), and value-channel pruning at lambda_v = 0.5 with
-    decode over the pruned key and value caches (bf16)."""
+    same T (prune + decode), SparK-p at p = 0.99 with the full 128-slot
+    capacity (prune + decode), and value-channel pruning at lambda_v = 0.5
+    with decode over the pruned key and value caches (bf16)."""
     sp = job.sp
     S = job.S_kept
     k = job.k_ev if wl.keep else job.k
@@ -406,6 +407,28 @@ def run_variants(job, wl, stream, peak, peak_kind, iters=5):
                     "decode_us": us_td, "decode_gbs": nb_t / (us_td / 1e6) / 1e9,
                     "timing": "CUDA events on the stream, outside the step; no tail"}
     del kt_, wst, wsd_t
+    # SparK-p at the pages' p = 0.99, full capacity (no cut): prune + decode
+    Tcap = wl.D
+    kp_ = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, Tcap, wl.torch_dtype, device=job.dev)
+    wsp_p = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_TOPP, wl.rows, wl.Hkv, wl.G, S, wl.D, Tcap, 0),
+                         job.dev)
+    us_pp = timed(lambda: sp.spark_prune_topp(k, job.q_obs, wl.G, wl.W, 0.99, kp_, wsp_p, stream))
+    n_pruned = float(kp_.stats.reshape(-1, 4)[:, 0].sum().item())
+    mean_kept = wl.D - n_pruned / max(wl.BH * S, 1)
+    wsd_p = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_DECODE, wl.rows, wl.Hkv, wl.G, S, wl.D, Tcap, 0),
+                         job.dev)
+    outp = torch.empty_like(job.out)
+    us_pd = timed(lambda: sp.spark_decode_attn_topp(job.q, kp_, v, None, None, 0, 0, wl.G, outp, wsd_p,
+                                                    stream=stream))
+    if sp.spark_device_status(wsd_p) != 0:
+        raise RuntimeError("device status after the SparK-p decode")
+    nb_pp = wl.BH * S * (wl.D * es + 16 + Tcap * es)
+    nb_pd = wl.BH * S * (16 + Tcap * es + wl.D * es)
+    out["spark_p"] = {"p": 0.99, "Tcap": Tcap, "mean_kept": mean_kept, "mean_prune_rate": 1 - mean_kept / wl.D,
+                      "prune_us": us_pp, "prune_bytes": nb_pp, "prune_gbs": nb_pp / (us_pp / 1e6) / 1e9,
+                      "decode_us": us_pd, "decode_bytes": nb_pd, "decode_gbs": nb_pd / (us_pd / 1e6) / 1e9,
+                      "timing": "CUDA events on the stream, outside the step; no tail"}
+    del kp_, wsp_p, wsd_p
     if wl.dtype == "bf16":
         Tv = sp.spark_lambda_to_T(0.5, wl.D)
         vc = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, Tv, wl.torch_dtype, device=job.dev)

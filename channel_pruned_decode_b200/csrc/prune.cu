@@ -257,6 +257,29 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     // u / scale) in fp32 bit patterns brackets the T-th largest key.
     uint32_t lo32 = lo == 0u ? 0u : __float_as_uint(half_bits_to_float(lo - 1u) * inv_scale);
     uint32_t hi32 = hi >= kTop16 ? 0x7f800001u : __float_as_uint(half_bits_to_float(hi) * inv_scale);
+    {
+        // Narrow the bracket to the keys inside it: with no key in [lo32,
+        // kmin) or (kmax, hi32), count(>= kmin) = count(>= lo32) >= T and
+        // count(>= kmax + 1) = count(>= hi32) < T.  A band of equal keys
+        // (bf16 values under unit norms are exact in fp16) leaves a bracket
+        // one wide, and the tie scan below settles it.
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const bool in = ((gm >> i) & 1u) && (key[i] - lo32 < hi32 - lo32);
+            kmin = in ? min(kmin, key[i]) : kmin;
+            kmax = in ? max(kmax, key[i]) : kmax;
+        }
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+            kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        }
+        if (!exact && kmax >= kmin) {
+            lo32 = kmin;
+            hi32 = kmax + 1u;
+        }
+    }
     bool exact32 = exact;
     bool done2 = exact || (hi32 - lo32 <= 1u);
     while (__any_sync(0xffffffffu, !done2)) {
