@@ -32,7 +32,8 @@
 //            accumulates q'_g (k_j - c_j) for the G heads of the group from
 //            the q' / c tables (q' = q * log2(e)/sqrt(D)); a SparK-p cache,
 //            whose masks may hold fewer bits than its T value slots, takes
-//            the same T steps with those past the token's count adding 0;
+//            as many steps as the warp's largest kept count, those past a
+//            token's own count adding 0;
 //   softmax  warp max (integer REDUX on an order-preserving map) updates the
 //            running max; p = 2^(s - m) goes to shared memory;
 //   P.V      bf16: tensor cores -- the V tile is the B operand
@@ -786,16 +787,17 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 const E *vp = ws.svals(st) + lane + (a.T - 1) * kWT;
                 // kDegVar: this token's kept count; value i from the top
                 // sits in slot cnt - 1 - i, steps past cnt add nothing
-                int cnt = a.T;
+                int cnt = a.T, steps = a.T;
                 if constexpr (kF == kDegVar) {
                     cnt = min(__popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w), a.T);
                     vp = ws.svals(st) + lane;
+                    steps = (int)__reduce_max_sync(0xffffffffu, (unsigned)cnt);  // the warp's longest walk
                 }
                 float2 s2[G / 2 > 0 ? G / 2 : 1];  // head pairs: packed fp32x2 FMAs
 #pragma unroll
                 for (int g = 0; g < (G / 2 > 0 ? G / 2 : 1); ++g) s2[g] = make_float2(0.f, 0.f);
 #pragma unroll 4
-                for (int i = 0; i < a.T; ++i) {
+                for (int i = 0; i < steps; ++i) {
                     const uint32_t pos = bit_top(cur);        // 0xffffffff when cur == 0
                     const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
                     cur &= bit_mask_below(pos);  // clear the top bit
