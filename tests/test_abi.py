@@ -216,3 +216,36 @@ def test_prune_think_rejects_bad_args(L):
     assert f(16, 16, 4, 32, ctypes.byref(kc), None, 1 << 20, None) == B.SPARK_ERR_WORKSPACE
     assert f(16, 16, 4, 32, ctypes.byref(kc), 256, 64, None) == B.SPARK_ERR_WORKSPACE
     assert f(16, 16, 4, 32, ctypes.byref(_kc(T=129)), 256, 1 << 20, None) == B.SPARK_ERR_ARG
+
+
+def test_prune_topp_rejects_bad_args(L):
+    kc = _kc()
+
+    def f(p=0.99, k=16, G=4, c=None, ws=256, wsb=1 << 20):
+        return L.spark_prune_topp(k, 16, G, 32, ctypes.c_float(p), ctypes.byref(c or kc), ws, wsb, None)
+    for p in (1.5, -0.1, float("nan")):
+        assert f(p=p) == B.SPARK_ERR_ARG
+    assert f(G=0) == B.SPARK_ERR_ARG
+    assert f(k=None) == B.SPARK_ERR_ARG
+    assert f(ws=None) == B.SPARK_ERR_WORKSPACE
+    assert f(wsb=64) == B.SPARK_ERR_WORKSPACE
+    assert f(c=_kc(T=129)) == B.SPARK_ERR_ARG
+    assert f(c=_kc(D=64)) == B.SPARK_ERR_UNSUPPORTED
+    # three fp64 partials per chunk of 256 tokens (the pruned count is the third)
+    assert B.spark_workspace_bytes(B.SPARK_OP_TOPP, 1, 8, 4, 32768, 128, 128, 0) >= 256 + 8 * 128 * 24
+    assert B.spark_workspace_bytes(B.SPARK_OP_TOPP, 1, 8, 4, 32768, 128, 128, 0) > \
+        B.spark_workspace_bytes(B.SPARK_OP_PRUNE, 1, 8, 4, 32768, 128, 128, 0)
+
+
+def test_decode_topp_rejects_bad_args(L):
+    kc = _kc()
+    call = lambda **k: L.spark_decode_attn_topp(
+        k.get("q", 16), ctypes.byref(kc), k.get("v", 16), k.get("kt", 16), k.get("vt", 16),
+        k.get("cap", 8), k.get("n", 0), k.get("G", 4), k.get("rec", 0), 0, k.get("out", 16),
+        k.get("ws", 256), 1 << 20, None)
+    assert call(G=3) == B.SPARK_ERR_UNSUPPORTED
+    assert call(rec=9) == B.SPARK_ERR_ARG
+    assert call(n=9) == B.SPARK_ERR_ARG
+    assert call(q=None) == B.SPARK_ERR_ARG
+    assert call(kt=None) == B.SPARK_ERR_ARG
+    assert call(ws=None) == B.SPARK_ERR_WORKSPACE
