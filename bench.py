@@ -429,6 +429,7 @@ def run_variants(job, wl, stream, peak, peak_kind, iters=5):
                       "decode_us": us_pd, "decode_bytes": nb_pd, "decode_gbs": nb_pd / (us_pd / 1e6) / 1e9,
                       "timing": "CUDA events on the stream, outside the step; no tail"}
     del kp_, wsp_p, wsd_p
+    out["decode_loop"] = run_decode_loop(sp, job.dev)
     if wl.dtype == "bf16":
         Tv = sp.spark_lambda_to_T(0.5, wl.D)
         vc = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, Tv, wl.torch_dtype, device=job.dev)
@@ -446,6 +447,62 @@ def run_variants(job, wl, stream, peak, peak_kind, iters=5):
                           "decode_token_heads_per_s": wl.BH * S / (us_d / 1e6),
                           "timing": "CUDA events on the stream, outside the step; no tail"}
     return out
+
+
+def run_decode_loop(sp, dev, steps=64):
+    """The decode phase of the single-layer Llama-3.1-8B shape (B=1, 8 kv
+    heads x 4, S=32768, lambda=0.5, bf16): 64 steps, each appending the new
+    key/value to the dense tail and decoding.  One step moves ~105 MB, a few
+    microseconds of HBM time, so launches matter: the same 64 steps are timed
+    as individual calls and as one replay of a CUDA graph that captured them."""
+    wl = WORKLOADS["llama1l"]
+    T = sp.spark_lambda_to_T(wl.lam, wl.D)
+    pre = make_prefill(wl, dev)
+    R, H, S, D, G = wl.rows, wl.Hkv, wl.S, wl.D, wl.G
+    kc = sp.KCache.empty(R, H, S, D, T, wl.torch_dtype, device=dev)
+    wsp = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_PRUNE, R, H, G, S, D, T, 0), dev)
+    sp.spark_prune(pre["k"], pre["q_obs"], G, wl.W, kc, wsp)
+    cap = steps
+    kt = torch.zeros((R, H, cap, D), dtype=wl.torch_dtype, device=dev)
+    vt = torch.zeros_like(kt)
+    ws = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_DECODE, R, H, G, S, D, T, cap), dev)
+    stp = [make_decode_step(wl, i, dev) for i in range(steps)]
+    out = torch.empty((R, wl.Hq, D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream()
+
+    def loop():
+        for i in range(steps):
+            sp.spark_tail_append(stp[i]["k_new"], stp[i]["v_new"], kt, vt, R, H, D, cap, i, stream)
+            sp.spark_decode_attn(stp[i]["q"], kc, pre["v"], kt, vt, cap, i + 1, G, out, ws, stream=stream)
+
+    def timed(f, reps=5):
+        with torch.cuda.stream(stream):
+            f()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                f()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps / steps * 1e3
+
+    us_eager = timed(loop)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            loop()
+    torch.cuda.synchronize()
+    us_graph = timed(g.replay)
+    if sp.spark_device_status(ws) != 0:
+        raise RuntimeError("device status after the decode loop")
+    del g
+    es = 2
+    nb = wl.BH * S * (16 + T * es + D * es) + wl.BH * (steps // 2) * 2 * D * es  # cache + mean tail
+    return {"workload": "llama1l: B=1 L=1 Hkv=8 G=4 S=32768 lambda=0.5 (T=64) bf16, 64 decode steps",
+            "us_per_step_eager": us_eager, "us_per_step_graph": us_graph,
+            "launches_per_step": 3, "bytes_per_step": nb, "gbs_graph": nb / (us_graph / 1e6) / 1e9,
+            "timing": "CUDA events around 5 repetitions of the 64 steps on one stream; tail append + decode "
+                      "+ combine per step"}
 
 
 def run_e2e(job, wl, steps, dist_on, world):

@@ -42,7 +42,8 @@
 //            the products keep ~16 bits of p; fp32: lane = 4 value channels,
 //            packed fp32x2 FMAs over the tokens.
 // At the end of an item the warp writes (acc[G][D], m, l) for it;
-// combine_kernel merges a head's items in a fixed order.
+// combine_kernel merges a head's items, eight warps over disjoint item
+// slices with loads in flight, then the warp sums in a fixed order.
 #include "spark_internal.cuh"
 
 #include <algorithm>
@@ -901,29 +902,68 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
     }
 }
 
+// One CTA of kCombineThreads per (row, query head) merges the head's work
+// items: the running maxima first (all threads, then a fixed-order tree),
+// then warp w sums the items w, w + 8, ... with weights 2^(m_u - M) (lane =
+// 4 channels, 16-byte loads, four items in flight), and the eight warp sums
+// are added in warp order.  Items with l = 0 (empty) weigh 0.
+constexpr int kCombineThreads = 256;
 template <int G>
-__global__ void __launch_bounds__(kD) combine_kernel(const float *__restrict__ acc,
-                                                     const float *__restrict__ ml, int units,
-                                                     float *__restrict__ out) {
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const float *__restrict__ acc,
+                                                                  const float *__restrict__ ml, int units,
+                                                                  float *__restrict__ out) {
+    constexpr int kW = kCombineThreads / 32;
+    __shared__ float wmax[kW];
+    __shared__ float wl[kW];
+    __shared__ float4 wo[kW][32];
     const long row = blockIdx.x;  // (bh, g)
     const long bh = row / G;
     const int g = (int)(row % G);
-    const int d = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t base = (size_t)bh * units * G + g;  // item u of this head: base + u * G
     float M = -INFINITY;
-    for (int u = 0; u < units; ++u) M = fmaxf(M, ml[(((size_t)bh * units + u) * G + g) * 2]);
-    float L = 0.f, o = 0.f;
+    for (int u = tid; u < units; u += kCombineThreads) M = fmaxf(M, ml[(base + (size_t)u * G) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) wmax[warp] = M;
+    __syncthreads();
+    M = wmax[0];
+#pragma unroll
+    for (int w = 1; w < kW; ++w) M = fmaxf(M, wmax[w]);
+    float L = 0.f;
+    float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
-        for (int u = 0; u < units; ++u) {
-            const size_t r = ((size_t)bh * units + u) * G + g;
-            const float mu = ml[r * 2], lu = ml[r * 2 + 1];
-            if (lu > 0.f) {
-                const float w = exp2f(mu - M);
-                L = fmaf(lu, w, L);
-                o = fmaf(acc[r * kD + d], w, o);
-            }
+#pragma unroll 4
+        for (int u = warp; u < units; u += kW) {
+            const size_t r = base + (size_t)u * G;
+            const float2 m_l = *reinterpret_cast<const float2 *>(ml + r * 2);
+            const float w = m_l.y > 0.f ? exp2f(m_l.x - M) : 0.f;
+            const float4 a4 = *reinterpret_cast<const float4 *>(acc + r * kD + 4 * lane);
+            L = fmaf(m_l.y, w, L);
+            o4.x = fmaf(a4.x, w, o4.x);
+            o4.y = fmaf(a4.y, w, o4.y);
+            o4.z = fmaf(a4.z, w, o4.z);
+            o4.w = fmaf(a4.w, w, o4.w);
         }
     }
-    out[row * kD + d] = (L > 0.f) ? o / L : 0.f;
+    wo[warp][lane] = o4;
+    if (lane == 0) wl[warp] = L;
+    __syncthreads();
+    if (warp == 0) {
+        float Ls = 0.f;
+        float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kW; ++w) {
+            Ls += wl[w];
+            s4.x += wo[w][lane].x;
+            s4.y += wo[w][lane].y;
+            s4.z += wo[w][lane].z;
+            s4.w += wo[w][lane].w;
+        }
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        *reinterpret_cast<float4 *>(out + row * kD + 4 * lane) =
+            make_float4(s4.x * inv, s4.y * inv, s4.z * inv, s4.w * inv);
+    }
 }
 
 DecodeGeom decode_geometry(long BH, int S, int T, int Tv, int es, int G, int num_sms) {
@@ -984,7 +1024,7 @@ static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, flo
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)geo.smem);
     if (e != cudaSuccess) return e;
     kern<<<geo.ctas, geo.nwarp * 32, geo.smem, st>>>(a);
-    combine_kernel<G><<<(unsigned)(a.BH * G), kD, 0, st>>>(a.acc, a.ml, geo.units, out);
+    combine_kernel<G><<<(unsigned)(a.BH * G), kCombineThreads, 0, st>>>(a.acc, a.ml, geo.units, out);
     return cudaGetLastError();
 }
 
