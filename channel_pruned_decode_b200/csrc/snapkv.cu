@@ -17,7 +17,8 @@
 //       shared-memory tiles.  Pass 0 writes each split's running max and
 //       exp-sum of every window row (online softmax); pass 1 merges them in a
 //       fixed order, recomputes the logits and sums the normalised
-//       probabilities of each key over the rows.
+//       probabilities of each key over the rows (one MUFU exp2 per score,
+//       the row's 1 / l folded into the exponent).
 //   snap_select_kernel  one CTA per head: max-pool, exact radix select of the
 //       (keep-W)-th largest pooled score on its fp32 bit pattern (scores are
 //       >= 0), and an order-preserving compaction (ties to the lower index).
@@ -43,6 +44,14 @@ template <int N> __device__ __forceinline__ void cp_async_wait() {
 
 // log2(e) / sqrt(128)
 constexpr float kSnapScale = 0.12751743074602467f;
+
+// 2^x on the MUFU unit in one instruction (results below 2^-126 flush to 0:
+// a probability that small does not move a sum that holds the row's maximum)
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // exclusive block-wide prefix sum of one int per thread (kSelThreads threads)
 __device__ __forceinline__ int block_excl_scan(int v, int *wsum, int &total) {
@@ -226,7 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     extern __shared__ unsigned char sm_raw[];
     __shared__ uint64_t bars[2];
     __shared__ uint32_t tmem_base_s;
-    __shared__ float rowm[kSnapMaxRows], rowil[kSnapMaxRows];  // merged row max and 1 / exp-sum (pass 1)
+    __shared__ float rowb[kSnapMaxRows];  // pass 1: m + log2(l) of each window row (+inf past R)
     __shared__ float half_a[kSnapMaxRows], half_b[kSnapMaxRows];  // the upper column half's partial results
     __shared__ int fail_s;
     // 1024-byte aligned tiles: queries, then two key buffers
@@ -283,8 +292,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                     m = n;
                 }
             }
-            rowm[tid] = tid < R ? m : 0.f;
-            rowil[tid] = tid < R ? 1.f / l : 0.f;
+            // p = 2^(x - m) / l = 2^(x - (m + log2 l)): one exponent per score
+            rowb[tid] = (tid < R && l > 0.f) ? m + log2f(l) : INFINITY;
         }
     }
     if (tile_lo < tile_hi) load_tile(tile_lo);
@@ -366,7 +375,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 const float b = n == -INFINITY ? 0.f : n;
                 float s = 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) s += exp2f(fmaf(v[i], kSnapScale, -b));
+                for (int i = 0; i < 32; ++i) s += ex2_fast(fmaf(v[i], kSnapScale, -b));
                 l_run = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - n)) + s;
                 m_run = n;
             }
@@ -382,7 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int c = 64 * chalf + c0 + i;
-                    acc += exp2f(fmaf(v[i], kSnapScale, -rowm[c])) * rowil[c];
+                    acc += ex2_fast(fmaf(v[i], kSnapScale, -rowb[c]));
                 }
             }
             // lower half + upper half, in that order
