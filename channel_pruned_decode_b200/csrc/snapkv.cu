@@ -21,7 +21,9 @@
 //       the row's 1 / l folded into the exponent).
 //   snap_select_kernel  one CTA per head: max-pool, exact radix select of the
 //       (keep-W)-th largest pooled score on its fp32 bit pattern (scores are
-//       >= 0), and an order-preserving compaction (ties to the lower index).
+//       >= 0; 8-bit digits, each digit found by a warp scan of the
+//       histogram), and an order-preserving compaction (ties to the lower
+//       index; contiguous token ranges per thread, two block scans).
 //   snap_gather_kernel  copies the kept K and V rows (16-byte vectors).
 #include "spark_internal.cuh"
 
@@ -114,15 +116,45 @@ __global__ void __launch_bounds__(kSelThreads)
             if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
         }
         __syncthreads();
-        if (tid == 0) {
-            int above = 0;
-            int d = 255;
-            for (; d > 0; --d) {
-                if (above + hist[d] >= rem) break;
-                above += hist[d];
+        if (tid < 32) {
+            // the largest digit d whose count from the top, inclusive, reaches
+            // rem: lane l sums digits 255 - 8l ... 248 - 8l, a warp scan gives
+            // the count above each lane's block, and the lane whose block
+            // crosses rem walks its 8 digits (digit 0 if no block crosses)
+            const int lane = tid;
+            int c[8], loc = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                c[j] = hist[255 - 8 * lane - j];
+                loc += c[j];
             }
-            sel[0] = prefix | ((uint32_t)d << shift);
-            sel[1] = (uint32_t)(rem - above);
+            int incl = loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int before = incl - loc;
+            const bool cross = before < rem && incl >= rem;
+            const unsigned who = __ballot_sync(0xffffffffu, cross);
+            if (who == 0u) {
+                if (lane == 31) {  // no block reaches rem: digit 0 with everything above it
+                    sel[0] = prefix;
+                    sel[1] = (uint32_t)(rem - (incl - c[7]));
+                }
+            } else if (cross) {
+                int above = before, d = 255 - 8 * lane;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (above + c[j] >= rem) {
+                        d = 255 - 8 * lane - j;
+                        break;
+                    }
+                    above += c[j];
+                }
+                sel[0] = prefix | ((uint32_t)d << shift);
+                sel[1] = (uint32_t)(rem - above);
+            }
         }
         __syncthreads();
         prefix = sel[0];
@@ -130,20 +162,28 @@ __global__ void __launch_bounds__(kSelThreads)
         pmask |= 255u << shift;
         __syncthreads();
     }
-    // keep: key > prefix, plus the first `rem` keys == prefix in index order
-    int base = 0, eq_base = 0;
-    for (long t0 = 0; t0 < P; t0 += kSelThreads) {
-        const long t = t0 + tid;
-        const uint32_t key = t < P ? pk[t] : 0u;
-        const int eq = (kp > 0 && t < P && key == prefix) ? 1 : 0;
-        int eq_total;
-        const int eq_rank = eq_base + block_excl_scan(eq, wsum, eq_total);
-        const int keepf = (kp > 0 && t < P && (key > prefix || (eq && eq_rank < rem))) ? 1 : 0;
-        int k_total;
-        const int pos = base + block_excl_scan(keepf, wsum, k_total);
-        if (keepf) out[pos] = (int)t;
-        base += k_total;
-        eq_base += eq_total;
+    // keep: key > prefix, plus the first `rem` keys == prefix in index order.
+    // Thread i owns the contiguous tokens [i*E, (i+1)*E), so two block scans
+    // (equal keys before it, kept tokens before it) place every kept index.
+    const long E = (P + kSelThreads - 1) / kSelThreads;
+    const long tb = min(P, (long)tid * E), te = min(P, tb + E);
+    int n_eq = 0;
+    for (long t = tb; t < te; ++t) n_eq += (kp > 0 && pk[t] == prefix) ? 1 : 0;
+    int tot;
+    const int eq_before = block_excl_scan(n_eq, wsum, tot);
+    int n_keep = 0;
+    for (long t = tb, r = eq_before; t < te && kp > 0; ++t) {
+        const uint32_t key = pk[t];
+        const bool eq = key == prefix;
+        n_keep += (key > prefix || (eq && r < rem)) ? 1 : 0;
+        r += eq ? 1 : 0;
+    }
+    int pos = block_excl_scan(n_keep, wsum, tot);
+    for (long t = tb, r = eq_before; t < te && kp > 0; ++t) {
+        const uint32_t key = pk[t];
+        const bool eq = key == prefix;
+        if (key > prefix || (eq && r < rem)) out[pos++] = (int)t;
+        r += eq ? 1 : 0;
     }
     for (int w = tid; w < W; w += kSelThreads) out[kp + w] = (int)(P + w);
 }
