@@ -505,6 +505,84 @@ def run_decode_loop(sp, dev, steps=64):
                       "+ combine per step"}
 
 
+def run_sweep(args):
+    """Every configuration of the workload table on one GPU: prune and one
+    decode step (dense tail of one token) timed with CUDA events on the
+    launching stream (inputs larger than L2 except `tiny`), each against the
+    HBM roofline on its algorithmic bytes.  One JSON object per line."""
+    import channel_pruned_decode_b200 as sp
+    peak, peak_kind = _peaks()
+    dev = "cuda"
+    if not args.sweep_workloads:
+        # one process per configuration: a configuration timed after another
+        # one in the same process can inherit a slow device state (the long
+        # prune after the single-layer one: 8.7 ms instead of 4.8)
+        for name in ("tiny", "llama1l", "lsweep_0.3", "lsweep_0.5", "lsweep_0.8", "long", "evict"):
+            r = subprocess.run([sys.executable, os.path.abspath(__file__), "--sweep", "--sweep-workloads", name],
+                               capture_output=True, text=True)
+            sys.stdout.write(r.stdout)
+            sys.stdout.flush()
+            if r.returncode != 0:
+                sys.stderr.write(r.stderr)
+                raise SystemExit(r.returncode)
+        return
+    names = args.sweep_workloads.split(",")
+    for name in names:
+        wl = WORKLOADS[name]
+        T = sp.spark_lambda_to_T(wl.lam, wl.D)
+        job = Job(wl, dev)
+        stream = torch.cuda.Stream()
+        k, v = job.k, job.v
+        rec = {"workload": _workload_desc(wl, T).split(";")[0], "T": T}
+
+        def timed(f, reps):
+            # warm up for at least 0.2 s of device time (and 3 calls): the
+            # first calls on freshly allocated buffers run up to 2x slower
+            with torch.cuda.stream(stream):
+                t_end, n = time.perf_counter() + 0.2, 0
+                while n < 3 or time.perf_counter() < t_end:
+                    f()
+                    n += 1
+                    if n % 8 == 0:
+                        torch.cuda.synchronize()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(reps):
+                    f()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / reps * 1e3
+
+        reps = 5 if name == "long" else 20
+        if wl.keep:
+            rec["snapkv_us"] = timed(lambda: sp.spark_snapkv_evict(
+                job.k, job.v, job.q_obs, wl.G, wl.W, wl.keep, wl.pool, job.k_ev, job.v_ev, job.idx, job.wse,
+                stream), reps)
+            k, v = job.k_ev, job.v_ev
+            sp.spark_snapkv_evict(job.k, job.v, job.q_obs, wl.G, wl.W, wl.keep, wl.pool, job.k_ev, job.v_ev,
+                                  job.idx, job.wse, stream)
+        S = job.S_kept
+        es = 2 if wl.dtype == "bf16" else 4
+        us_p = timed(lambda: sp.spark_prune(k, job.q_obs, wl.G, wl.W, job.kc, job.wsp, stream), reps)
+        sp.spark_tail_append(job.k_new, job.v_new, job.kt, job.vt, wl.rows, wl.Hkv, wl.D, job.cap, 0, stream)
+        us_d = timed(lambda: sp.spark_decode_attn(job.q, job.kc, v, job.kt, job.vt, job.cap, 1, wl.G, job.out,
+                                                  job.wsd, stream=stream), reps)
+        if sp.spark_device_status(job.wsd) != 0:
+            raise RuntimeError(f"device status after decode ({name})")
+        bp = wl.BH * S * (wl.D * es + 16 + T * es)
+        bd = wl.BH * S * (16 + T * es + wl.D * es) + wl.BH * 2 * wl.D * es
+        rec.update({"prune_us": us_p, "prune_gbs": bp / (us_p / 1e6) / 1e9,
+                    f"prune_frac_{peak_kind}": bp / (us_p / 1e6) / 1e9 / peak,
+                    "decode_us": us_d, "decode_gbs": bd / (us_d / 1e6) / 1e9,
+                    f"decode_frac_{peak_kind}": bd / (us_d / 1e6) / 1e9 / peak,
+                    "decode_token_heads_per_s": wl.BH * (S + 1) / (us_d / 1e6),
+                    "l2": "inputs exceed the 126 MB L2" if bd > 126e6 else "inputs fit in L2 (parity-size case)"})
+        print(json.dumps(rec), flush=True)
+        del job
+        torch.cuda.empty_cache()
+
+
 def run_e2e(job, wl, steps, dist_on, world):
     """Same metric through the public API with pinned HOST inputs: every step
     copies K, V, window queries and the decode query/new key/value to the
@@ -613,11 +691,16 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip the SparK-g variant timing")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time prune and decode on every workload (one JSON line each) instead of the step")
+    ap.add_argument("--sweep-workloads", default="", help="comma-separated subset for --sweep")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_gpu(args)
 
