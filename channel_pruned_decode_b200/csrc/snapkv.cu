@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __shared__ uint32_t tmem_base_s;
     __shared__ float rowb[kSnapMaxRows];  // pass 1: m + log2(l) of each window row (+inf past R)
     __shared__ float half_a[kSnapMaxRows], half_b[kSnapMaxRows];  // the upper column half's partial results
+    __shared__ float half_p[2][kSnapMaxRows];  // pass 1: upper-half sums, one buffer per tile parity
     __shared__ int fail_s;
     // 1024-byte aligned tiles: queries, then two key buffers
     const uint32_t base = (smem_u32(sm_raw) + 1023u) & ~1023u;
@@ -357,10 +358,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             tc_commit(smem_u32(&bars[tile & 1]));
         }
     };
-    // first tile's operands (and the queries) landed: make them visible to the
-    // tensor core's proxy, then issue
+    // the first two tiles' operands (and the queries) landed: make them
+    // visible to the tensor core's proxy, then issue the first MMA
     if (tile_lo < tile_hi) {
-        cp_async_wait<1>();
+        cp_async_wait<0>();
         fence_proxy_async_smem();
         __syncthreads();
         issue(tile_lo);
@@ -371,22 +372,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     float m_run = -INFINITY, l_run = 0.f;          // pass 0: this window row's statistics
     const long lim_row = P + (row % W);
     bool failed = false;
+    // One CTA barrier per tile, at its end: the epilogue is done (its
+    // accumulator and key buffer may be reused), the copies of the tile after
+    // next have landed and are visible to the tensor core, and the threads
+    // agree on any timed-out wait.
     for (int tile = tile_lo; tile < tile_hi; ++tile) {
-        // next tile's operands -> issue its MMA before this tile's epilogue
-        if (tile + 1 < tile_hi) {
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            __syncthreads();
-            issue(tile + 1);
-        }
+        // the next tile's operands are in place: issue its MMA before this
+        // tile's epilogue
+        if (tile + 1 < tile_hi) issue(tile + 1);
         // this tile's accumulator is complete
         const uint32_t par = (uint32_t)(((tile - tile_lo) >> 1) & 1);
         const bool ok = mbar_wait_limit(smem_u32(&bars[tile & 1]), par, 1000000000ull);
         if (!__all_sync(0xffffffffu, ok)) failed = true;
-        if (__syncthreads_or(failed ? 1 : 0)) {
-            failed = true;
-            break;
-        }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         // its key buffer is free: fetch the tile after next
         if (tile + 2 < tile_hi) load_tile(tile + 2);
@@ -394,7 +391,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const uint32_t taddr =
             tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(tile & 1) * 128u + (uint32_t)(64 * chalf);
         const long t0 = (long)tile * kTcKeys;
-        if (kMode == 0) {
+        float acc_lo = 0.f;  // pass 1: this key's lower-half sum (added after the barrier)
+        if (failed) {
+            // skip the epilogue; the barrier below ends the loop
+        } else if (kMode == 0) {
             // S[row][key]: this row's logits for the tile's 128 keys
             const bool mask = t0 + kTcKeys - 1 > P;
 #pragma unroll 1
@@ -421,8 +421,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             }
         } else {
             // S^T[key][row]: this key's probabilities over the window rows
-            const long t = t0 + row;
-            const bool valid_t = t < P;
             float acc = 0.f;
 #pragma unroll 1
             for (int c0 = 0; c0 < kSnapMaxRows / 2; c0 += 32) {
@@ -434,14 +432,25 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                     acc += ex2_fast(fmaf(v[i], kSnapScale, -rowb[c]));
                 }
             }
-            // lower half + upper half, in that order
-            if (chalf == 1) half_a[row] = acc;
-            __syncthreads();
-            if (chalf == 0 && valid_t) scores[(size_t)bh * (P > 0 ? P : 0) + t] = acc + half_a[row];
+            // lower half + upper half, in that order (after the barrier)
+            if (chalf == 1) half_p[tile & 1][row] = acc;
+            acc_lo = acc;
         }
-        // accumulator tile & 1 and its key buffer may be reused
+        // the tile after next landed (its copies were issued before this
+        // epilogue); accumulator tile & 1 and its key buffer may be reused
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-        __syncthreads();
+        if (__syncthreads_or(failed ? 1 : 0)) {
+            failed = true;
+            break;
+        }
+        if (kMode == 1) {
+            // half_p[tile & 1] is rewritten two tiles on, after the next barrier
+            const long t = t0 + row;
+            if (chalf == 0 && t < P) scores[(size_t)bh * (P > 0 ? P : 0) + t] = acc_lo + half_p[tile & 1][row];
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     }
     cp_async_wait<0>();
     if (failed && tid == 0) atomicOr(status, kDevTimeout);
