@@ -281,6 +281,14 @@ struct Flash {
 // for lanes past the tile end).  Leaves p in shared memory in the layout the
 // P.V engine reads and returns the factor each head's accumulator is scaled
 // by (all 1 when no running max moved).
+// 2^x in one MUFU instruction (results below 2^-126 flush to 0: such a
+// weight is zero next to the tile's maximum, whose weight is 1)
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <typename E, int G>
 __device__ __forceinline__ bool tile_softmax(const WarpSmem<E, G> &ws, Flash<G> &f, const float (&s)[G],
                                              float (&alpha)[G]) {
@@ -291,10 +299,10 @@ __device__ __forceinline__ bool tile_softmax(const WarpSmem<E, G> &ws, Flash<G> 
     for (int g = 0; g < G; ++g) {
         const float mt = ord2f(__reduce_max_sync(0xffffffffu, f2ord(s[g])));
         const float m_new = fmaxf(f.m[g], mt);
-        alpha[g] = (m_new == -INFINITY) ? 1.f : exp2f(f.m[g] - m_new);
+        alpha[g] = (m_new == -INFINITY) ? 1.f : ex2_fast(f.m[g] - m_new);
         rescale |= (alpha[g] != 1.f);
         f.m[g] = m_new;
-        p[g] = (m_new == -INFINITY) ? 0.f : exp2f(s[g] - m_new);
+        p[g] = (m_new == -INFINITY) ? 0.f : ex2_fast(s[g] - m_new);
         f.l[g] = fmaf(f.l[g], alpha[g], p[g]);
     }
     if constexpr (sizeof(E) == 2) {
