@@ -154,3 +154,21 @@ def test_topp_full_size_sampled():
         m_o, v_o, _ = oracle.prune_topp(k_np[bh, ts][None], qn[bh:bh + 1], 0.99, Tcap)
         assert np.array_equal(m_g[bh, ts], m_o[0]), f"head {bh}"
         assert np.array_equal(vals_g[bh, ts].view(np.uint32), v_o[0].view(np.uint32)), f"head {bh}"
+
+
+@pytest.mark.parametrize("G", [1, 2, 8])
+def test_topp_group_sizes(G):
+    """The variable-count decode walk for every supported GQA group size (the
+    odd size takes the scalar FMA path, the others packed head pairs)."""
+    wl = scaled(WORKLOADS["tiny"], S=600, G=G, Hkv=2, dtype="bf16", seed=810 + G)
+    pre = make_prefill(wl, DEV)
+    kc = run_topp(pre["k"], pre["q_obs"], G, wl.W, 0.9, 100)
+    qn, m, vals, st = check_topp(kc, to_np(pre["k"]), to_np(pre["q_obs"]), G, 0.9, f"topp G={G}")
+    BH = wl.rows * wl.Hkv
+    q = make_decode_step(wl, 3, DEV)["q"]
+    out = torch.empty((wl.rows, wl.Hkv * G, D), dtype=torch.float32, device=DEV)
+    ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, G, wl.S, D, kc.T, 0))
+    spark_decode_attn_topp(q, kc, pre["v"], None, None, 0, 0, G, out, ws)
+    torch.cuda.synchronize()
+    o_ref = oracle.decode(to_np(q).reshape(BH * G, D), m, vals, qn, st, to_np(pre["v"]).reshape(BH, wl.S, D), G=G)
+    assert_out_close(out.cpu().numpy().reshape(BH * G, D), o_ref, f"topp decode G={G}")
