@@ -95,15 +95,39 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(tmp_path, name):
+def _run_mutant(name, workdir):
+    """Build the oracle with one planted mistake and run the pin suite on it;
+    returns (pin-suite exit code, the tail of its output)."""
     before, after = MUTANTS[name]
     src = open(os.path.join(ROOT, "oracle", "spark_oracle.c")).read()
-    assert src.count(before) == 1, f"mutation site for {name} not unique"
-    mutant_c = tmp_path / "mutant.c"
-    mutant_c.write_text(src.replace(before, after))
-    lib = oracle.build(force=True, src=str(mutant_c), out=str(tmp_path / "libmutant.so"))
+    if src.count(before) != 1:
+        return None, f"mutation site for {name} not unique"
+    d = os.path.join(workdir, name)
+    os.makedirs(d, exist_ok=True)
+    mutant_c = os.path.join(d, "mutant.c")
+    with open(mutant_c, "w") as f:
+        f.write(src.replace(before, after))
+    lib = oracle.build(force=True, src=mutant_c, out=os.path.join(d, "libmutant.so"))
     env = dict(os.environ, ORACLE_LIB=lib)
     r = subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider"],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """All mutants at once, one pin-suite process per mutant on the host's
+    cores (each builds its own copy of the oracle)."""
+    import concurrent.futures as cf
+    work = str(tmp_path_factory.mktemp("mutants"))
+    workers = max(1, min(len(MUTANTS), os.cpu_count() or 1))
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        futs = {name: ex.submit(_run_mutant, name, work) for name in MUTANTS}
+        return {name: f.result() for name, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(mutant_results, name):
+    rc, out = mutant_results[name]
+    assert rc is not None, out
+    assert rc != 0, f"pins did not catch mutant {name}:\n{out}"
