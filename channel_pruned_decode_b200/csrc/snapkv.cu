@@ -27,6 +27,8 @@
 //   snap_gather_kernel  copies the kept K and V rows (16-byte vectors).
 #include "spark_internal.cuh"
 
+#include <cuda.h>  // CUtensorMap and its enums (the encoder is fetched at run time)
+
 #include <algorithm>
 
 namespace spark {
@@ -267,13 +269,27 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// TMA: one box of the 3-D key tensor [head][token][channel] (64 channels x
+// 128 tokens, 128-byte swizzle) into shared memory, completion counted on
+// `bar`.  x = channel offset (0 or 64: 128-byte aligned), y = first token
+// (tokens past S read as zero), z = head.  No multicast.
+__device__ __forceinline__ void tma_load_keys(uint32_t dst, const CUtensorMap *tm, int x, int y, int z,
+                                              uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kTcThreads, 2)
-    snap_tc_kernel(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ q_obs, int S, int G,
-                   int W, int nsplit, float *__restrict__ ml, float *__restrict__ scores,
+    snap_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __nv_bfloat16 *__restrict__ q_obs, int S,
+                   int G, int W, int nsplit, float *__restrict__ ml, float *__restrict__ scores,
                    uint32_t *__restrict__ status) {
     extern __shared__ unsigned char sm_raw[];
-    __shared__ uint64_t bars[2];
+    __shared__ uint64_t bars[2];  // accumulator b complete (MMA commit)
+    __shared__ uint64_t full[2];  // key buffer b landed (TMA)
     __shared__ uint32_t tmem_base_s;
     __shared__ float rowb[kSnapMaxRows];  // pass 1: m + log2(l) of each window row (+inf past R)
     __shared__ float half_a[kSnapMaxRows], half_b[kSnapMaxRows];  // the upper column half's partial results
@@ -288,7 +304,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int tid = threadIdx.x, warp = tid >> 5;
     const int R = G * W;
     const long P = (long)S - W;
-    const __nv_bfloat16 *kb = k + (size_t)bh * S * kD;
     const __nv_bfloat16 *qb = q_obs + (size_t)bh * R * kD;
     const int ntile = (S + kTcKeys - 1) / kTcKeys;
     const int per = (ntile + nsplit - 1) / nsplit;
@@ -303,6 +318,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     if (tid == 0) {
         mbar_init(smem_u32(&bars[0]), 1);
         mbar_init(smem_u32(&bars[1]), 1);
+        mbar_init(smem_u32(&full[0]), 1);
+        mbar_init(smem_u32(&full[1]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fail_s = 0;
     }
@@ -311,14 +328,17 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const int r = i >> 4, cc = i & 15;
         cp_async16(sq + tc_off(r, cc), qb + (size_t)min(r, R - 1) * kD + cc * 8, r < R);
     }
+    // one thread fetches a key tile: two TMA boxes (channels 0-63, 64-127),
+    // which land in the two K-blocks of the swizzled tile
     auto load_tile = [&](int tile) {
         const uint32_t dst = sk0 + (uint32_t)(tile & 1) * kTcTileBytes;
-        for (int i = tid; i < kTcKeys * 16; i += kTcThreads) {
-            const int r = i >> 4, cc = i & 15;
-            const long t = (long)tile * kTcKeys + r;
-            cp_async16(dst + tc_off(r, cc), kb + (size_t)min(t, (long)S - 1) * kD + cc * 8, t < S);
-        }
+        const uint32_t fb = smem_u32(&full[tile & 1]);
+        mbar_expect_tx(fb, kTcTileBytes);
+        tma_load_keys(dst, &tmap_k, 0, tile * kTcKeys, (int)bh, fb);
+        tma_load_keys(dst + 128 * 128, &tmap_k, 64, tile * kTcKeys, (int)bh, fb);
     };
+    // parity of the use of buffer / accumulator `tile & 1` that `tile` makes
+    auto use_parity = [&](int tile) -> uint32_t { return (uint32_t)(((tile - tile_lo) >> 1) & 1); };
     if (kMode == 1) {
         // merged row statistics in split order (split 0 holds key 0, which
         // every row sees); rows past R contribute nothing (1 / l = 0)
@@ -337,14 +357,17 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             rowb[tid] = (tid < R && l > 0.f) ? m + log2f(l) : INFINITY;
         }
     }
-    if (tile_lo < tile_hi) load_tile(tile_lo);
-    cp_async_commit();
-    if (tile_lo + 1 < tile_hi) load_tile(tile_lo + 1);
-    cp_async_commit();
+    cp_async_commit();  // the queries
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
+    __syncthreads();  // barrier initialisation and the TMEM address are visible
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = tmem_base_s;
+    int loaded_hi = tile_lo, waited_hi = tile_lo;  // thread 0: tiles fetched / whose fetch it waited for
+    if (tid == 0) {
+        if (tile_lo < tile_hi) load_tile(tile_lo);
+        if (tile_lo + 1 < tile_hi) load_tile(tile_lo + 1);
+        loaded_hi = min(tile_hi, tile_lo + 2);
+    }
 
     // MMA of `tile` into accumulator tile & 1: pass 0 A = queries, B = keys;
     // pass 1 A = keys, B = queries
@@ -358,36 +381,49 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             tc_commit(smem_u32(&bars[tile & 1]));
         }
     };
-    // the first two tiles' operands (and the queries) landed: make them
-    // visible to the tensor core's proxy, then issue the first MMA
-    if (tile_lo < tile_hi) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        __syncthreads();
-        issue(tile_lo);
+    // the queries landed: make them visible to the tensor core's proxy; the
+    // MMA issuer waits for each key tile's TMA on its own
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncthreads();
+    bool failed = false;
+    if (tile_lo < tile_hi && tid == 0) {
+        if (mbar_wait_limit(smem_u32(&full[tile_lo & 1]), 0u, 1000000000ull)) {
+            waited_hi = tile_lo + 1;
+            issue(tile_lo);
+        } else {
+            failed = true;
+        }
     }
 
     const int row = 32 * (warp & 3) + (tid & 31);  // this thread's TMEM lane
     const int chalf = warp >> 2;                    // its column half
     float m_run = -INFINITY, l_run = 0.f;          // pass 0: this window row's statistics
     const long lim_row = P + (row % W);
-    bool failed = false;
     // One CTA barrier per tile, at its end: the epilogue is done (its
     // accumulator and key buffer may be reused), the copies of the tile after
     // next have landed and are visible to the tensor core, and the threads
     // agree on any timed-out wait.
     for (int tile = tile_lo; tile < tile_hi; ++tile) {
-        // the next tile's operands are in place: issue its MMA before this
-        // tile's epilogue
-        if (tile + 1 < tile_hi) issue(tile + 1);
+        // the next tile's keys landed: issue its MMA before this tile's
+        // epilogue (its accumulator was freed by the previous barrier)
+        if (tid == 0 && tile + 1 < tile_hi && !failed) {
+            if (mbar_wait_limit(smem_u32(&full[(tile + 1) & 1]), use_parity(tile + 1), 1000000000ull)) {
+                waited_hi = tile + 2;
+                issue(tile + 1);
+            } else {
+                failed = true;
+            }
+        }
         // this tile's accumulator is complete
-        const uint32_t par = (uint32_t)(((tile - tile_lo) >> 1) & 1);
-        const bool ok = mbar_wait_limit(smem_u32(&bars[tile & 1]), par, 1000000000ull);
+        const bool ok = mbar_wait_limit(smem_u32(&bars[tile & 1]), use_parity(tile), 1000000000ull);
         if (!__all_sync(0xffffffffu, ok)) failed = true;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        // its key buffer is free: fetch the tile after next
-        if (tile + 2 < tile_hi) load_tile(tile + 2);
-        cp_async_commit();
+        // its key buffer is free (the MMA read it): fetch the tile after next
+        if (tid == 0 && tile + 2 < tile_hi && !failed) {
+            load_tile(tile + 2);
+            loaded_hi = tile + 3;
+        }
         const uint32_t taddr =
             tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(tile & 1) * 128u + (uint32_t)(64 * chalf);
         const long t0 = (long)tile * kTcKeys;
@@ -436,10 +472,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             if (chalf == 1) half_p[tile & 1][row] = acc;
             acc_lo = acc;
         }
-        // the tile after next landed (its copies were issued before this
-        // epilogue); accumulator tile & 1 and its key buffer may be reused
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
+        // accumulator tile & 1 may be reused; the threads agree on timeouts
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         if (__syncthreads_or(failed ? 1 : 0)) {
             failed = true;
@@ -474,6 +507,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     // with a bound, before the columns are freed)
     if (failed && tid == 0) {
         for (int b = 0; b < 2; ++b) (void)mbar_wait_limit(smem_u32(&bars[b]), 0u, 1000000ull);
+        // key tiles still in flight land before the CTA leaves
+        for (int t = waited_hi; t < loaded_hi; ++t)
+            (void)mbar_wait_limit(smem_u32(&full[t & 1]), use_parity(t), 1000000ull);
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -497,6 +533,39 @@ int snapkv_splits(long BH, int S, int num_sms) {
 
 size_t snapkv_partials_bytes(long BH) { return (size_t)BH * kSnapMaxSplit * kSnapMaxRows * 2 * sizeof(float); }
 
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime (no
+// link-time dependency on the driver library)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// Keys as a 3-D tensor [head][token][channel] of bf16; one box is 64
+// channels (128 bytes, the swizzle span) x 128 tokens of one head.  Tokens
+// past S are out of bounds and read as zero.
+static bool make_key_map(CUtensorMap *tm, const void *k, long BH, int S) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)S, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)S * kD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kTcKeys, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
                           int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st) {
     const long P = (long)S - W;
@@ -511,11 +580,12 @@ cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long 
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     const int ns = snapkv_splits(BH, S, nsm);
-    const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(k);
     const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q_obs);
     uint32_t *status = static_cast<uint32_t *>(ws);
-    snap_tc_kernel<0><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(kb, qb, S, G, W, ns, ml, scores, status);
-    snap_tc_kernel<1><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(kb, qb, S, G, W, ns, ml, scores, status);
+    CUtensorMap tmap;
+    if (!make_key_map(&tmap, k, BH, S)) return cudaErrorInvalidValue;
+    snap_tc_kernel<0><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(tmap, qb, S, G, W, ns, ml, scores, status);
+    snap_tc_kernel<1><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(tmap, qb, S, G, W, ns, ml, scores, status);
     snap_select_kernel<<<(unsigned)BH, kSelThreads, 0, st>>>(scores, pooled, S, W, keep, pool, idx_out);
     const int row_vec = kD * 2 / 16;  // bf16 rows
     const int rows_per_cta = 256 / row_vec;
