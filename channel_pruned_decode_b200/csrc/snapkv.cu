@@ -14,7 +14,8 @@
 //   snap_tc_kernel<0/1>  the keys of each (row, kv head) split over several
 //       CTAs; the G*W x S logits are a dense contraction, computed by
 //       tcgen05.mma (bf16 -> fp32 in tensor memory) from 128-byte-swizzled
-//       shared-memory tiles.  Pass 0 writes each split's running max and
+//       shared-memory tiles, the key tiles fetched by TMA.  Pass 0 writes
+//       each split's running max and
 //       exp-sum of every window row (online softmax); pass 1 merges them in a
 //       fixed order, recomputes the logits and sums the normalised
 //       probabilities of each key over the rows (one MUFU exp2 per score,
@@ -207,8 +208,10 @@ __global__ void snap_gather_kernel(const uint4 *__restrict__ k, const uint4 *__r
 // a 128 x 128 query tile (window rows, zero-padded) and a ring of two 128-key
 // tiles in shared memory, K-major with the 128-byte swizzle that the UMMA
 // descriptors describe; two 128-column fp32 accumulators in tensor memory.
-// Thread 0 issues the tcgen05.mma instructions and commits them to an
-// mbarrier; every thread then reads half of one accumulator row (tcgen05.ld:
+// Thread 0 fetches the key tiles by TMA (completion on a per-buffer
+// mbarrier), issues the tcgen05.mma instructions once a tile has landed and
+// commits them to a per-accumulator mbarrier; every thread then reads half of
+// one accumulator row (tcgen05.ld:
 // warp w reads TMEM lanes 32*(w%4).. and columns 64*(w/4)..).  Pass 0
 // computes S = Q K^T (a row is a window row: its running max and exp-sum are
 // kept per half and merged at the end); pass 1 computes S^T = K Q^T (a row is
