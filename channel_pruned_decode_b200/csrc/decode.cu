@@ -912,11 +912,10 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
 
 // One CTA of kCombineThreads per (row, query head) merges the head's work
 // items: the running maxima first (all threads, then a fixed-order tree),
-// then warp w sums the items w, w + 8, ... with weights 2^(m_u - M) (lane =
-// 4 channels, 16-byte loads, four items in flight), and the eight warp sums
-// are added in warp order.  Items with l = 0 (empty) weigh 0.
-constexpr int kCombineThreads = 256;
-template <int G>
+// then warp w sums the items w, w + W, ... (W warps) with weights
+// 2^(m_u - M) (lane = 4 channels, 16-byte loads, four items in flight), and
+// the warp sums are added in warp order.  Items with l = 0 (empty) weigh 0.
+template <int G, int kCombineThreads>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const float *__restrict__ acc,
                                                                   const float *__restrict__ ml, int units,
                                                                   float *__restrict__ out) {
@@ -1032,7 +1031,13 @@ static cudaError_t launch_decode_t(const DecArgs &a0, const DecodeGeom &geo, flo
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)geo.smem);
     if (e != cudaSuccess) return e;
     kern<<<geo.ctas, geo.nwarp * 32, geo.smem, st>>>(a);
-    combine_kernel<G><<<(unsigned)(a.BH * G), kCombineThreads, 0, st>>>(a.acc, a.ml, geo.units, out);
+    // few rows with many items (small batches): more warps per row, so that
+    // each warp merges a handful of items
+    const long rows = a.BH * G;
+    if (rows < 2L * geo.ctas && geo.units > 64)
+        combine_kernel<G, 1024><<<(unsigned)rows, 1024, 0, st>>>(a.acc, a.ml, geo.units, out);
+    else
+        combine_kernel<G, 256><<<(unsigned)rows, 256, 0, st>>>(a.acc, a.ml, geo.units, out);
     return cudaGetLastError();
 }
 
