@@ -63,8 +63,15 @@ def _byte_model(wl, T, n_tail):
     prune = BH * S * (D * es + 16 + T * es) + BH * G * wl.W * D * es + BH * (D * 4 + 32)
     decode = (BH * S * (16 + T * es + D * es) + BH * n_tail * 2 * D * es
               + BH * G * D * (es + 4) + BH * (D * 4 + 32))
-    return {"prune": prune, "decode": decode, "per_token_head_prune": D * es + 16 + T * es,
-            "per_token_head_decode": 16 + T * es + D * es}
+    out = {"prune": prune, "decode": decode, "per_token_head_prune": D * es + 16 + T * es,
+           "per_token_head_decode": 16 + T * es + D * es}
+    if wl.keep:
+        # eviction: the keys read once for the scores, the window queries,
+        # the kept K and V rows read and written, the kept indices written
+        S0 = wl.S
+        out["snapkv"] = (BH * S0 * D * es + BH * G * wl.W * D * es + 4 * BH * wl.keep * D * es
+                         + BH * wl.keep * 4)
+    return out
 
 
 # --------------------------------------------------------------- clocks
@@ -306,11 +313,20 @@ def run_gpu(args):
     peak, peak_kind = _peaks()
     prune_gbs = bm["prune"] / (prune_ms / 1e3) / 1e9
     decode_gbs = bm["decode"] / (decode_ms / 1e3) / 1e9
-    dom = "prune" if prune_ms >= decode_ms else "decode"
-    dom_ms = prune_ms if dom == "prune" else decode_ms
+    spans = {"prune": prune_ms, "decode": decode_ms}
+    if wl.keep:
+        spans["snapkv"] = evict_ms
+    dom = max(spans, key=spans.get)
+    dom_ms = spans[dom]
     achieved = bm[dom] / (dom_ms / 1e3) / 1e9
-    kernel_name = {"prune": "prune_kernel", "decode": "decode_kernel"}[dom]
-    traffic = _traffic_record(kernel_name, wl.name)
+    kernel_name = {"prune": "prune_kernel", "decode": "decode_kernel", "snapkv": "snap_tc_kernel"}[dom]
+    traffic = _traffic_record(kernel_name, wl.name) if dom != "snapkv" else None
+    timing = {"prune": "CUDA events around spark_prune on its stream (qnorm and stats, the two small "
+                       "kernels launched with it, included)",
+              "decode": "CUDA events around spark_decode_attn on its stream (the combine kernel "
+                        "launched with it included)",
+              "snapkv": "CUDA events around spark_snapkv_evict on its stream: both score passes, the "
+                        "select and the gather (the bytes are those of the whole entry point)"}[dom]
 
     variants = None
     if not args.no_variants:
@@ -343,12 +359,16 @@ def run_gpu(args):
                       f"frac_{peak_kind}": prune_gbs / peak, "bytes_per_step": bm["prune"]},
             "tail_append_us": append_ms * 1e3,
             "snapkv_evict_us": evict_ms * 1e3 if wl.keep else None,
+            "snapkv": ({"us_per_step": evict_ms * 1e3, "gbs": bm["snapkv"] / (evict_ms / 1e3) / 1e9,
+                        f"frac_{peak_kind}": bm["snapkv"] / (evict_ms / 1e3) / 1e9 / peak,
+                        "bytes_per_step": bm["snapkv"]} if wl.keep else None),
             "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic,
-                         "bytes_per_launch": bm[dom],
-                         "timing": "CUDA events around the entry point on its stream "
-                                   "(the two small kernels launched with it included)"},
+                         "bytes_per_launch": bm[dom], "entry": {"prune": "spark_prune",
+                                                                "decode": "spark_decode_attn",
+                                                                "snapkv": "spark_snapkv_evict"}[dom],
+                         "timing": timing},
             "variants": variants,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": job.launches_per_step * args.steps,
