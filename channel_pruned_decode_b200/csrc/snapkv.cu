@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __shared__ uint64_t bars[2];  // accumulator b complete (MMA commit)
     __shared__ uint64_t full[2];  // key buffer b landed (TMA)
     __shared__ uint32_t tmem_base_s;
-    __shared__ float rowb[kSnapMaxRows];  // pass 1: m + log2(l) of each window row (+inf past R)
+    __shared__ __align__(16) float rowb[kSnapMaxRows];  // pass 1: m + log2(l) of each window row (+inf past R)
     __shared__ float half_a[kSnapMaxRows], half_b[kSnapMaxRows];  // the upper column half's partial results
     __shared__ float half_p[2][kSnapMaxRows];  // pass 1: upper-half sums, one buffer per tile parity
     __shared__ int fail_s;
@@ -465,10 +465,15 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             for (int c0 = 0; c0 < kSnapMaxRows / 2; c0 += 32) {
                 float v[32];
                 tc_ld32(taddr + (uint32_t)c0, v);
+                // the warp reads the same biases: 16-byte broadcasts
+                const float4 *rb = reinterpret_cast<const float4 *>(rowb + 64 * chalf + c0);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c = 64 * chalf + c0 + i;
-                    acc += ex2_fast(fmaf(v[i], kSnapScale, -rowb[c]));
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 b = rb[i4];
+                    acc += ex2_fast(fmaf(v[4 * i4 + 0], kSnapScale, -b.x));
+                    acc += ex2_fast(fmaf(v[4 * i4 + 1], kSnapScale, -b.y));
+                    acc += ex2_fast(fmaf(v[4 * i4 + 2], kSnapScale, -b.z));
+                    acc += ex2_fast(fmaf(v[4 * i4 + 3], kSnapScale, -b.w));
                 }
             }
             // lower half + upper half, in that order (after the barrier)
