@@ -219,6 +219,17 @@ def _traffic_record(kernel: str, workload: str):
     return rec["bytes_per_launch"] if h == rec["source_sha"] else None
 
 
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(wl, job, units: int | None = None):
     """The CPU oracle, as it stands, on a bounded sample of the workload:
     prune + decode of whole (layer, kv head) units, threads over units."""
@@ -242,19 +253,33 @@ def cpu_baseline(wl, job, units: int | None = None):
         data.append((k[b:b + 1].float().cpu().numpy(), v[b:b + 1].float().cpu().numpy(),
                      qo[b * G:(b + 1) * G].float().cpu().numpy(), q[b * G:(b + 1) * G].float().cpu().numpy()))
 
-    def one(d):
+    def prune_one(d):
         kk, vv, qq, q1 = d
         qn = oracle.qnorm(qq, G, lib=lib)
-        m, vals, st = oracle.prune(kk, qn, job.T, lib=lib)
+        return qn, oracle.prune(kk, qn, job.T, lib=lib)
+
+    def decode_one(d, pr):
+        kk, vv, qq, q1 = d
+        qn, (m, vals, st) = pr
         return oracle.decode(q1, m, vals, qn, st, vv, G=G, lib=lib)
 
+    # one unit on one thread, then the sample on the pool, prune and decode
+    # timed as separate phases
     t0 = time.perf_counter()
+    decode_one(data[0], prune_one(data[0]))
+    single = time.perf_counter() - t0
     with cf.ThreadPoolExecutor(max_workers=min(cores, len(data))) as ex:
-        list(ex.map(one, data))
-    dt = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        prs = list(ex.map(prune_one, data))
+        t1 = time.perf_counter()
+        list(ex.map(decode_one, data, prs))
+        t2 = time.perf_counter()
+    dt = t2 - t0
     return {"value": len(data) * S / dt, "unit": UNIT, "cores": min(cores, len(data)), "kind": "oracle",
             "sample": f"{len(data)} of {BH} (layer, kv head) units, full S={S}: prune + 1 decode step, "
-                      f"{dt:.1f} s wall"}
+                      f"{dt:.1f} s wall",
+            "prune_s": t1 - t0, "decode_s": t2 - t1, "single_thread_unit_s": single,
+            "cpu_model": _cpu_model()}
 
 
 def run_gpu(args):
@@ -693,7 +718,8 @@ def run_reference(args):
         "data": "synthetic", "config": {"workload": _workload_desc(wl, T)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"each step: {len(units)} kv-head units of the first {S_s} of "
-                                   f"S={S} prompt tokens, prune + 1 decode step (threads over units)"},
+                                   f"S={S} prompt tokens, prune + 1 decode step (threads over units)",
+                         "cpu_model": _cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
