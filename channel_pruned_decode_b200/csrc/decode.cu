@@ -26,14 +26,15 @@
 // for bf16 by cp.async into an XOR-swizzled per-warp tile, for fp32 by
 // coalesced 8-byte loads into registers.  No CTA-wide barrier is on the path.
 // Per tile:
-//   q.k~     lane = token; the lane walks exactly T set bits of its 128-bit
-//            mask from the top channel down (a queue of the non-empty mask
-//            words, one bfind and one bit clear per step, no branch) and
-//            accumulates q'_g (k_j - c_j) for the G heads of the group from
-//            the q' / c tables (q' = q * log2(e)/sqrt(D)); a SparK-p cache,
-//            whose masks may hold fewer bits than its T value slots, takes
-//            as many steps as the warp's largest kept count, those past a
-//            token's own count adding 0;
+//   q.k~     lane = token; for T < 72 the lane walks exactly T set bits of
+//            its 128-bit mask from the top channel down (a queue of the
+//            non-empty mask words, one bfind and one bit clear per step, no
+//            branch) and accumulates q'_g (k_j - c_j) for the G heads of the
+//            group from the q' / c tables (q' = q * log2(e)/sqrt(D)); for
+//            larger T, and for a SparK-p cache (masks with fewer bits than
+//            its T value slots), all lanes step through the 128 channels
+//            together, so that the table reads are broadcasts, and a pruned
+//            channel adds q' * 0 -- the same sums in the same order;
 //   softmax  warp max (integer REDUX on an order-preserving map) updates the
 //            running max; p = 2^(s - m) goes to shared memory;
 //   P.V      bf16: tensor cores -- the V tile is the B operand
@@ -525,11 +526,14 @@ __device__ __forceinline__ void write_partial(const DecArgs &a, long bh, int u, 
 // spilling warps on the G = 4 workloads
 __host__ __device__ constexpr int dec_max_warps(int G) { return G > 2 ? 12 : kMaxWarps; }
 
-// kF: the recovery F (spark_recovery), or kDegVar: Degenerate F over a cache
-// whose masks may hold fewer bits than its T value slots (SparK-p: the kept
-// values fill the first slots of each token, zeros after).
-constexpr int kDegVar = kRecoveryDegVar;
-__host__ __device__ constexpr bool is_degenerate(int f) { return f == SPARK_F_DEGENERATE || f == kDegVar; }
+// kF: the recovery F (spark_recovery), or kDegDense: Degenerate F with q.k~
+// taken in channel order (every lane visits the same channel at each step, so
+// the q' / c table reads are broadcasts) instead of walking each token's kept
+// bits.  The channel-order loop also serves caches whose masks hold fewer bits
+// than their T value slots (SparK-p: the kept values fill the first slots of
+// each token, zeros after; selector kRecoveryDegVar on the host side).
+constexpr int kDegDense = kRecoveryDegDense;
+__host__ __device__ constexpr bool is_degenerate(int f) { return f == SPARK_F_DEGENERATE || f == kDegDense; }
 
 template <typename E, int G, int kF, bool kPV>
 __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArgs a) {
@@ -779,6 +783,54 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
 #pragma unroll
                     for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
                 }
+            } else if constexpr (kF == kDegDense) {
+                // All 128 channels from the top down, the same for every lane:
+                // a kept channel takes this token's next packed value from the
+                // end, a pruned one adds q' * 0.  The kept channels meet the
+                // FMAs in the same order as in the walk below, and adding an
+                // exact zero product leaves the sum unchanged, so the scores
+                // are bit-identical to the walk's.  A mask with more bits than
+                // value slots (a cache never written by spark_prune, or a lane
+                // past n) reads nothing.
+                const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
+                const int cnt = __popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w);
+                const bool ok = cnt <= a.T;
+                const uint32_t wds[4] = {ok ? mw.x : 0u, ok ? mw.y : 0u, ok ? mw.z : 0u, ok ? mw.w : 0u};
+                const E *vp = ws.svals(st) + lane + (ok && cnt > 0 ? cnt - 1 : 0) * kWT;
+                float2 s2[G / 2 > 0 ? G / 2 : 1];
+#pragma unroll
+                for (int g = 0; g < (G / 2 > 0 ? G / 2 : 1); ++g) s2[g] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int wi = 3; wi >= 0; --wi) {
+                    const uint32_t w = wds[wi];
+#pragma unroll
+                    for (int b = 31; b >= 0; --b) {
+                        const int j = 32 * wi + b;
+                        float x = 0.f;
+                        if ((w >> b) & 1u) {
+                            x = Elem<E>::to_f(*vp) - ws.tabc[j];
+                            vp -= kWT;
+                        }
+                        QVec<G> qv;
+                        qv.load(ws.tabq + j * G);
+                        if constexpr (G % 2 == 0) {
+                            const float2 x2 = make_float2(x, x);
+#pragma unroll
+                            for (int g = 0; g < G; g += 2)
+                                s2[g / 2] = __ffma2_rn(make_float2(qv.v[g], qv.v[g + 1]), x2, s2[g / 2]);
+                        } else {
+#pragma unroll
+                            for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
+                        }
+                    }
+                }
+                if constexpr (G % 2 == 0) {
+#pragma unroll
+                    for (int g = 0; g < G; g += 2) {
+                        s[g] = s2[g / 2].x;
+                        s[g + 1] = s2[g / 2].y;
+                    }
+                }
             } else if (a.T > 0) {
                 // Walk the T set bits of the 128-bit mask from the top channel
                 // down, pairing the i-th bit from the top with the i-th packed
@@ -794,19 +846,11 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 uint32_t bq = 0x00204060u;  // bases 96, 64, 32, 0 from the low byte up
                 queue_nonempty(cur, n1, n2, n3, bq);
                 const E *vp = ws.svals(st) + lane + (a.T - 1) * kWT;
-                // kDegVar: this token's kept count; value i from the top
-                // sits in slot cnt - 1 - i, steps past cnt add nothing
-                int cnt = a.T, steps = a.T;
-                if constexpr (kF == kDegVar) {
-                    cnt = min(__popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w), a.T);
-                    vp = ws.svals(st) + lane;
-                    steps = (int)__reduce_max_sync(0xffffffffu, (unsigned)cnt);  // the warp's longest walk
-                }
                 float2 s2[G / 2 > 0 ? G / 2 : 1];  // head pairs: packed fp32x2 FMAs
 #pragma unroll
                 for (int g = 0; g < (G / 2 > 0 ? G / 2 : 1); ++g) s2[g] = make_float2(0.f, 0.f);
 #pragma unroll 4
-                for (int i = 0; i < steps; ++i) {
+                for (int i = 0; i < a.T; ++i) {
                     const uint32_t pos = bit_top(cur);        // 0xffffffff when cur == 0
                     const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
                     cur &= bit_mask_below(pos);  // clear the top bit
@@ -815,13 +859,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                     n1 = e ? n2 : n1;
                     n2 = e ? n3 : n2;
                     bq = e ? (bq >> 8) : bq;
-                    float x;
-                    if constexpr (kF == kDegVar) {
-                        const int r = cnt - 1 - i;
-                        x = r >= 0 ? Elem<E>::to_f(vp[max(r, 0) * kWT]) - ws.tabc[j] : 0.f;
-                    } else {
-                        x = Elem<E>::to_f(vp[-i * kWT]) - ws.tabc[j];
-                    }
+                    const float x = Elem<E>::to_f(vp[-i * kWT]) - ws.tabc[j];
                     QVec<G> qv;
                     qv.load(ws.tabq + j * G);
                     if constexpr (G % 2 == 0) {
@@ -1052,14 +1090,22 @@ static cudaError_t dispatch_g(const DecArgs &a, const DecodeGeom &geo, int G, fl
     }
 }
 
+// From this many kept channels per token on, the channel-order loop (128
+// steps of about 10 instructions, broadcast table reads) beats the per-token
+// walk (T steps of about 20, table reads that conflict in shared-memory
+// banks): measured equal at T = 64, the loop 16 % faster at T = 90.
+constexpr int kDenseMinT = 72;
+
 template <typename E>
 static cudaError_t dispatch_f(const DecArgs &a, const DecodeGeom &geo, int G, int recovery, float *out,
                               cudaStream_t st) {
     switch (recovery) {
-    case SPARK_F_DEGENERATE: return dispatch_g<E, SPARK_F_DEGENERATE>(a, geo, G, out, st);
+    case SPARK_F_DEGENERATE:
+        return a.T >= kDenseMinT ? dispatch_g<E, kDegDense>(a, geo, G, out, st)
+                                 : dispatch_g<E, SPARK_F_DEGENERATE>(a, geo, G, out, st);
     case SPARK_F_GAUSSIAN: return dispatch_g<E, SPARK_F_GAUSSIAN>(a, geo, G, out, st);
     case SPARK_F_EXPONENTIAL: return dispatch_g<E, SPARK_F_EXPONENTIAL>(a, geo, G, out, st);
-    case kDegVar: return dispatch_g<E, kDegVar>(a, geo, G, out, st);
+    case kRecoveryDegVar: return dispatch_g<E, kDegDense>(a, geo, G, out, st);
     default: return cudaErrorInvalidValue;
     }
 }

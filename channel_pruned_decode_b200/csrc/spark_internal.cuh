@@ -50,6 +50,8 @@ inline size_t topp_workspace(long BH, int S) {
 // recovery selector of the decode kernel beyond spark_recovery: Degenerate F
 // over a SparK-p cache (masks may hold fewer bits than the T value slots)
 constexpr int kRecoveryDegVar = 3;
+// Degenerate F with the channel-order q.k~ loop (chosen for large T)
+constexpr int kRecoveryDegDense = 4;
 
 // Each warp of a persistent CTA is an independent flash-decoding worker.  Its
 // ring of shared-memory stages holds the mask and kept values of one 32-token
