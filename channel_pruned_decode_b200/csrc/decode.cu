@@ -26,15 +26,15 @@
 // for bf16 by cp.async into an XOR-swizzled per-warp tile, for fp32 by
 // coalesced 8-byte loads into registers.  No CTA-wide barrier is on the path.
 // Per tile:
-//   q.k~     lane = token; for T < 72 the lane walks exactly T set bits of
+//   q.k~     lane = token; for T < 48 the lane walks exactly T set bits of
 //            its 128-bit mask from the top channel down (a queue of the
 //            non-empty mask words, one bfind and one bit clear per step, no
 //            branch) and accumulates q'_g (k_j - c_j) for the G heads of the
 //            group from the q' / c tables (q' = q * log2(e)/sqrt(D)); for
 //            larger T, and for a SparK-p cache (masks with fewer bits than
 //            its T value slots), all lanes step through the 128 channels
-//            together, so that the table reads are broadcasts, and a pruned
-//            channel adds q' * 0 -- the same sums in the same order;
+//            together, so that the table reads are broadcasts, and pruned
+//            channels are predicated off -- the same sums in the same order;
 //   softmax  warp max (integer REDUX on an order-preserving map) updates the
 //            running max; p = 2^(s - m) goes to shared memory;
 //   P.V      bf16: tensor cores -- the V tile is the B operand
@@ -786,12 +786,12 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
             } else if constexpr (kF == kDegDense) {
                 // All 128 channels from the top down, the same for every lane:
                 // a kept channel takes this token's next packed value from the
-                // end, a pruned one adds q' * 0.  The kept channels meet the
-                // FMAs in the same order as in the walk below, and adding an
-                // exact zero product leaves the sum unchanged, so the scores
-                // are bit-identical to the walk's.  A mask with more bits than
-                // value slots (a cache never written by spark_prune, or a lane
-                // past n) reads nothing.
+                // end (the table reads of the lanes that keep it are one
+                // broadcast), a pruned one is skipped by predication.  The kept
+                // channels meet the FMAs in the same order as in the walk
+                // below, so the scores are bit-identical to the walk's.  A mask
+                // with more bits than value slots (a cache never written by
+                // spark_prune, or a lane past n) reads nothing.
                 const uint4 mw = *reinterpret_cast<const uint4 *>(ws.smask(st) + lane * kMaskWords);
                 const int cnt = __popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w);
                 const bool ok = cnt <= a.T;
@@ -804,23 +804,29 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 for (int wi = 3; wi >= 0; --wi) {
                     const uint32_t w = wds[wi];
 #pragma unroll
-                    for (int b = 31; b >= 0; --b) {
-                        const int j = 32 * wi + b;
-                        float x = 0.f;
-                        if ((w >> b) & 1u) {
-                            x = Elem<E>::to_f(*vp) - ws.tabc[j];
-                            vp -= kWT;
-                        }
-                        QVec<G> qv;
-                        qv.load(ws.tabq + j * G);
-                        if constexpr (G % 2 == 0) {
-                            const float2 x2 = make_float2(x, x);
+                    for (int b4 = 7; b4 >= 0; --b4) {
+                        // c_j of four channels in one broadcast read
+                        const float4 c4 = *reinterpret_cast<const float4 *>(ws.tabc + 32 * wi + 4 * b4);
+                        const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-                            for (int g = 0; g < G; g += 2)
-                                s2[g / 2] = __ffma2_rn(make_float2(qv.v[g], qv.v[g + 1]), x2, s2[g / 2]);
-                        } else {
+                        for (int u = 3; u >= 0; --u) {
+                            const int b = 4 * b4 + u;
+                            const int j = 32 * wi + b;
+                            if ((w >> b) & 1u) {  // predicated, no branch
+                                const float x = Elem<E>::to_f(*vp) - cc[u];
+                                vp -= kWT;
+                                QVec<G> qv;
+                                qv.load(ws.tabq + j * G);
+                                if constexpr (G % 2 == 0) {
+                                    const float2 x2 = make_float2(x, x);
 #pragma unroll
-                            for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
+                                    for (int g = 0; g < G; g += 2)
+                                        s2[g / 2] = __ffma2_rn(make_float2(qv.v[g], qv.v[g + 1]), x2, s2[g / 2]);
+                                } else {
+#pragma unroll
+                                    for (int g = 0; g < G; ++g) s[g] = fmaf(qv.v[g], x, s[g]);
+                                }
+                            }
                         }
                     }
                 }
@@ -1091,10 +1097,11 @@ static cudaError_t dispatch_g(const DecArgs &a, const DecodeGeom &geo, int G, fl
 }
 
 // From this many kept channels per token on, the channel-order loop (128
-// steps of about 10 instructions, broadcast table reads) beats the per-token
-// walk (T steps of about 20, table reads that conflict in shared-memory
-// banks): measured equal at T = 64, the loop 16 % faster at T = 90.
-constexpr int kDenseMinT = 72;
+// predicated steps of about 8 instructions, broadcast table reads) beats the
+// per-token walk (T steps of about 20, table reads that conflict in
+// shared-memory banks): measured 25 % slower at T = 26, 12 % faster at T = 64
+// and 27 % at T = 90.
+constexpr int kDenseMinT = 48;
 
 template <typename E>
 static cudaError_t dispatch_f(const DecArgs &a, const DecodeGeom &geo, int G, int recovery, float *out,
