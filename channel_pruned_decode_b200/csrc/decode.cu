@@ -887,37 +887,37 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 }
             }
             if constexpr (kPV) {
-                // expand the pruned values into the swizzled V tile: the warp
-                // zeroes the tile (512 contiguous bytes per store, no bank
-                // conflict), then each lane writes its token's kept values with
-                // the same top-down mask walk as q.k~ (pruned entries stay 0)
-                const uint32_t tile = smem_u32(ws.vt);
+                // expand the pruned values into the swizzled V tile: each lane
+                // builds its token's row 8 channels (16 bytes) at a time, top
+                // channel first, a kept channel taking the token's next packed
+                // value from the end and a pruned one 0, and stores every
+                // chunk (the swizzle keeps the warp's 16-byte stores free of
+                // bank conflicts); a lane past n, or a mask with more bits
+                // than Tv, writes a zero row
+                const uint4 mw = *reinterpret_cast<const uint4 *>(ws.svmask(st) + lane * kMaskWords);
+                const int cnt = __popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w);
+                const bool ok = valid && cnt <= a.Tv;
+                const uint32_t wds[4] = {ok ? mw.x : 0u, ok ? mw.y : 0u, ok ? mw.z : 0u, ok ? mw.w : 0u};
+                const uint16_t *vp = reinterpret_cast<const uint16_t *>(ws.svvals(st)) + lane +
+                                     (ok && cnt > 0 ? cnt - 1 : 0) * kWT;
+                const uint32_t vrow = smem_u32(ws.vt);
 #pragma unroll
-                for (int c = 0; c < kWT * kD * 2 / 512; ++c)
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(tile + 512u * c + 16u * lane),
-                                 "r"(0u)
-                                 : "memory");
-                __syncwarp();
-                if (valid && a.Tv > 0) {
-                    const uint4 mw = *reinterpret_cast<const uint4 *>(ws.svmask(st) + lane * kMaskWords);
-                    uint32_t cur = mw.w, n1 = mw.z, n2 = mw.y, n3 = mw.x;
-                    uint32_t bq = 0x00204060u;
-                    queue_nonempty(cur, n1, n2, n3, bq);
-                    const uint16_t *vp =
-                        reinterpret_cast<const uint16_t *>(ws.svvals(st)) + lane + (a.Tv - 1) * kWT;
-                    const uint32_t vrow = smem_u32(ws.vt);
-#pragma unroll 4
-                    for (int i = 0; i < a.Tv; ++i) {
-                        const uint32_t pos = bit_top(cur);
-                        const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
-                        cur &= bit_mask_below(pos);
-                        const bool e = cur == 0u;
-                        cur = e ? n1 : cur;
-                        n1 = e ? n2 : n1;
-                        n2 = e ? n3 : n2;
-                        bq = e ? (bq >> 8) : bq;
-                        const uint32_t adr = vrow + vswz(lane, j >> 3) + 2u * (uint32_t)(j & 7);
-                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(adr), "h"(vp[-i * kWT]) : "memory");
+                for (int wi = 3; wi >= 0; --wi) {
+                    const uint32_t w = wds[wi];
+#pragma unroll
+                    for (int c8 = 3; c8 >= 0; --c8) {
+                        uint32_t h[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                        for (int u = 7; u >= 0; --u) {
+                            if ((w >> (8 * c8 + u)) & 1u) {  // predicated, no branch
+                                h[u >> 1] |= (uint32_t)*vp << (16 * (u & 1));
+                                vp -= kWT;
+                            }
+                        }
+                        const uint32_t adr = vrow + vswz(lane, 4 * wi + c8);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(h[0]), "r"(h[1]),
+                                     "r"(h[2]), "r"(h[3])
+                                     : "memory");
                     }
                 }
             }
