@@ -9,9 +9,9 @@ import pytest
 import torch
 
 import oracle
-from channel_pruned_decode_b200 import (KCache, spark_decode_attn, spark_decode_attn_topp, spark_prune_topp,
-                                        spark_workspace_bytes, workspace, SPARK_F_GAUSSIAN, SPARK_OP_DECODE,
-                                        SPARK_OP_TOPP)
+from channel_pruned_decode_b200 import (KCache, spark_decode_attn, spark_decode_attn_topp, spark_device_status,
+                                        spark_prune_topp, spark_workspace_bytes, workspace, SPARK_F_GAUSSIAN,
+                                        SPARK_OP_DECODE, SPARK_OP_TOPP)
 from channel_pruned_decode_b200.synth import WORKLOADS, make_decode_step, make_prefill, scaled
 from tests._parity import assert_out_close, mask_np, run_prune, to_np, unpack_vals
 from tests.test_gpu_parity import STATS_RTOL
@@ -111,19 +111,24 @@ def test_topp_decode_gaussian_and_tail():
         assert_out_close(out.cpu().numpy().reshape(BH * G, D), o_ref, f"topp decode F={rec}")
 
 
-def test_topp_decode_equals_plain_decode_on_full_masks():
-    """On a plain SparK cache (exactly T bits per token) the SparK-p decode
-    takes the same arithmetic steps as spark_decode_attn."""
-    wl = scaled(WORKLOADS["llama1l"], S=4096)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("T,G", [(1, 4), (26, 4), (26, 1), (26, 8), (47, 2), (64, 4), (127, 8)])
+def test_topp_decode_equals_plain_decode_on_full_masks(dtype, T, G):
+    """On a plain SparK cache (exactly T bits per token) the SparK-p decode,
+    which always steps through the channels in order, gives the same bits as
+    spark_decode_attn, which walks the T kept bits of each token for T < 48:
+    the kept channels meet the same FMAs in the same order."""
+    wl = scaled(WORKLOADS["llama1l"], S=3000, Hkv=3, G=G, dtype=dtype, seed=T + G)
     pre = make_prefill(wl, DEV)
-    kc = run_prune(pre["k"], pre["q_obs"], wl.G, wl.W, 64)
+    kc = run_prune(pre["k"], pre["q_obs"], wl.G, wl.W, T)
     q = make_decode_step(wl, 0, DEV)["q"]
     outs = []
     for fn in (spark_decode_attn, spark_decode_attn_topp):
         out = torch.empty((wl.rows, wl.Hkv * wl.G, D), dtype=torch.float32, device=DEV)
-        ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, wl.G, wl.S, D, 64, 0))
+        ws = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, wl.G, wl.S, D, T, 0))
         fn(q, kc, pre["v"], None, None, 0, 0, wl.G, out, ws)
         torch.cuda.synchronize()
+        assert spark_device_status(ws) == 0
         outs.append(out)
     assert torch.equal(outs[0], outs[1])
 
