@@ -31,10 +31,11 @@
 //            non-empty mask words, one bfind and one bit clear per step, no
 //            branch) and accumulates q'_g (k_j - c_j) for the G heads of the
 //            group from the q' / c tables (q' = q * log2(e)/sqrt(D)); for
-//            larger T, and for a SparK-p cache (masks with fewer bits than
-//            its T value slots), all lanes step through the 128 channels
-//            together, so that the table reads are broadcasts, and pruned
-//            channels are predicated off -- the same sums in the same order;
+//            larger T (the value-pruned decode included), and for a SparK-p
+//            cache (masks with fewer bits than its T value slots), all lanes
+//            step through the 128 channels together, so that the table reads
+//            are broadcasts, and pruned channels are predicated off -- the
+//            same sums in the same order;
 //   softmax  warp max (integer REDUX on an order-preserving map) updates the
 //            running max; p = 2^(s - m) goes to shared memory;
 //   P.V      bf16: tensor cores -- the V tile is the B operand
@@ -537,7 +538,7 @@ __host__ __device__ constexpr bool is_degenerate(int f) { return f == SPARK_F_DE
 
 template <typename E, int G, int kF, bool kPV>
 __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArgs a) {
-    static_assert(!kPV || (sizeof(E) == 2 && kF == SPARK_F_DEGENERATE), "packed values: bf16, Degenerate F");
+    static_assert(!kPV || (sizeof(E) == 2 && is_degenerate(kF)), "packed values: bf16, Degenerate F");
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= a.nwarp) return;
@@ -1145,7 +1146,8 @@ cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, 
         a.vmask = vc->mask;
         a.vvals = vc->vals;
         a.Tv = vc->T;
-        return dispatch_g<__nv_bfloat16, SPARK_F_DEGENERATE, true>(a, geo, G, out, st);
+        return a.T >= kDenseMinT ? dispatch_g<__nv_bfloat16, kDegDense, true>(a, geo, G, out, st)
+                                 : dispatch_g<__nv_bfloat16, SPARK_F_DEGENERATE, true>(a, geo, G, out, st);
     }
     if (kc.dtype == SPARK_BF16) return dispatch_f<__nv_bfloat16>(a, geo, G, recovery, out, st);
     return dispatch_f<float>(a, geo, G, recovery, out, st);
