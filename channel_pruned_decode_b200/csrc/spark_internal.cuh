@@ -76,10 +76,10 @@ __host__ __device__ inline size_t dec_stage_bytes(int T, int es) {
     return (size_t)kWT * 16 + (size_t)kWT * T * es;
 }
 
-// Per-warp tables: bf16 values add a swizzled V tile [kWT][kD] (8 KB) and
-// p as [G][kWT] fp32; then q' [kD][G], c [kD], p as duplicated pairs
-// [kWT][G][2] (fp32 values), Qc [16], mbarriers and the tile's kept-channel
-// lists [T][kWT] bytes; rounded to 128 bytes so that the stages start aligned.
+// Per-warp tables: bf16 values add a swizzled V tile [kWT][kD] (8 KB); then
+// p as [G][kWT] fp32, q' [kD][G], c [kD], p as duplicated pairs [kWT][G][2]
+// (fp32 values), Qc [16] and the ring's mbarriers; rounded to 128 bytes so
+// that the stages start aligned.
 __host__ __device__ inline size_t dec_vtile_bytes(int es) { return es == 2 ? (size_t)kWT * kD * 2 : 0; }
 __host__ __device__ inline size_t dec_table_bytes(int G, int es) {
     const size_t b = dec_vtile_bytes(es) + (size_t)G * kWT * 4 + (size_t)kD * G * 4 + kD * 4 +
