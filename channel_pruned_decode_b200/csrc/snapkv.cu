@@ -255,9 +255,9 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                  : "memory");
 }
 
-// 32 consecutive fp32 accumulator columns of this thread's TMEM lane
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane (the
+// caller waits for the load with tc_wait_ld)
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
         "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -267,9 +267,20 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
           "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
           "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Wait for this thread's TMEM loads.  The registers pass through the asm
+// ("+r"), so no use of them can be scheduled before the wait.
+__device__ __forceinline__ void tc_wait_ld(uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+          "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),
+          "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+          "+r"(r[30]), "+r"(r[31])
+        :
+        : "memory");
 }
 
 // TMA: one box of the 3-D key tensor [head][token][channel] (64 channels x
@@ -436,10 +447,17 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         } else if (kMode == 0) {
             // S[row][key]: this row's logits for the tile's 128 keys
             const bool mask = t0 + kTcKeys - 1 > P;
-#pragma unroll 1
+            // both 32-column chunks in flight before one wait
+            uint32_t rr[2][32];
+            tc_ld32(taddr, rr[0]);
+            tc_ld32(taddr + 32u, rr[1]);
+            tc_wait_ld(rr[0]);  // waits for both loads
+            tc_wait_ld(rr[1]);  // (already complete: orders the second chunk's uses)
+#pragma unroll
             for (int c0 = 0; c0 < kTcKeys / 2; c0 += 32) {
                 float v[32];
-                tc_ld32(taddr + (uint32_t)c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[c0 >> 5][i]);
                 if (mask) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -461,10 +479,16 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         } else {
             // S^T[key][row]: this key's probabilities over the window rows
             float acc = 0.f;
-#pragma unroll 1
+            uint32_t rr[2][32];
+            tc_ld32(taddr, rr[0]);
+            tc_ld32(taddr + 32u, rr[1]);
+            tc_wait_ld(rr[0]);  // waits for both loads
+            tc_wait_ld(rr[1]);  // (already complete: orders the second chunk's uses)
+#pragma unroll
             for (int c0 = 0; c0 < kSnapMaxRows / 2; c0 += 32) {
                 float v[32];
-                tc_ld32(taddr + (uint32_t)c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[c0 >> 5][i]);
                 // the warp reads the same biases: 16-byte broadcasts
                 const float4 *rb = reinterpret_cast<const float4 *>(rowb + 64 * chalf + c0);
 #pragma unroll
