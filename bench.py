@@ -232,7 +232,9 @@ def _cpu_model() -> str:
 
 def cpu_baseline(wl, job, units: int | None = None):
     """The CPU oracle, as it stands, on a bounded sample of the workload:
-    prune + decode of whole (layer, kv head) units, threads over units."""
+    prune + decode (with the step's one-token tail) of whole (layer, kv head)
+    units, threads over units; the same oracle outputs then check the GPU's
+    results for those units (sampled parity)."""
     import concurrent.futures as cf
 
     import numpy as np
@@ -240,28 +242,38 @@ def cpu_baseline(wl, job, units: int | None = None):
     import oracle
 
     lib = oracle.load()
-    BH, S, D, G = wl.BH, wl.S, wl.D, wl.G
+    BH, D, G = wl.BH, wl.D, wl.G
+    S = job.S_kept  # the tokens the GPU pruned (after eviction, if any)
     cores = os.cpu_count() or 1
     units = units or min(BH, cores)
     sel = list(range(0, BH, max(1, BH // units)))[:units]
-    k = job.k.reshape(BH, S, D)
-    v = job.v.reshape(BH, S, D)
+    # one untimed GPU step, so that the cache, the tail and the output hold
+    # this step's results whatever ran before
+    stream = torch.cuda.current_stream()
+    job.step(stream)
+    torch.cuda.synchronize()
+    k_src, v_src = (job.k_ev, job.v_ev) if wl.keep else (job.k, job.v)
+    k = k_src.reshape(BH, S, D)
+    v = v_src.reshape(BH, S, D)
+    kt = job.kt.reshape(BH, job.cap, D)
+    vt = job.vt.reshape(BH, job.cap, D)
     qo = job.q_obs.reshape(BH * G, wl.W, D)
     q = job.q.reshape(BH * G, D)
     data = []
     for b in sel:
         data.append((k[b:b + 1].float().cpu().numpy(), v[b:b + 1].float().cpu().numpy(),
-                     qo[b * G:(b + 1) * G].float().cpu().numpy(), q[b * G:(b + 1) * G].float().cpu().numpy()))
+                     qo[b * G:(b + 1) * G].float().cpu().numpy(), q[b * G:(b + 1) * G].float().cpu().numpy(),
+                     kt[b:b + 1].float().cpu().numpy(), vt[b:b + 1].float().cpu().numpy()))
 
     def prune_one(d):
-        kk, vv, qq, q1 = d
+        kk, vv, qq, q1, kt1, vt1 = d
         qn = oracle.qnorm(qq, G, lib=lib)
         return qn, oracle.prune(kk, qn, job.T, lib=lib)
 
     def decode_one(d, pr):
-        kk, vv, qq, q1 = d
+        kk, vv, qq, q1, kt1, vt1 = d
         qn, (m, vals, st) = pr
-        return oracle.decode(q1, m, vals, qn, st, vv, G=G, lib=lib)
+        return oracle.decode(q1, m, vals, qn, st, vv, kt1, vt1, 1, G=G, lib=lib)
 
     # one unit on one thread, then the sample on the pool, prune and decode
     # timed as separate phases
@@ -272,14 +284,46 @@ def cpu_baseline(wl, job, units: int | None = None):
         t0 = time.perf_counter()
         prs = list(ex.map(prune_one, data))
         t1 = time.perf_counter()
-        list(ex.map(decode_one, data, prs))
+        outs = list(ex.map(decode_one, data, prs))
         t2 = time.perf_counter()
     dt = t2 - t0
     return {"value": len(data) * S / dt, "unit": UNIT, "cores": min(cores, len(data)), "kind": "oracle",
-            "sample": f"{len(data)} of {BH} (layer, kv head) units, full S={S}: prune + 1 decode step, "
-                      f"{dt:.1f} s wall",
+            "sample": f"{len(data)} of {BH} (layer, kv head) units, full S={S}"
+                      f"{' (the tokens kept by the GPU eviction)' if wl.keep else ''}: prune + 1 decode step "
+                      f"with the one-token tail, {dt:.1f} s wall",
             "prune_s": t1 - t0, "decode_s": t2 - t1, "single_thread_unit_s": single,
-            "cpu_model": _cpu_model()}
+            "cpu_model": _cpu_model(), "parity": _sample_parity(job, sel, prs, outs, S)}
+
+
+def _sample_parity(job, sel, prs, outs, S):
+    """The GPU's cache and decode output of the sampled units against the
+    oracle's: tokens whose mask differs, tokens whose packed values differ,
+    the largest relative error of the statistics, the largest absolute error
+    of the decode output."""
+    import numpy as np
+
+    BH, G, D, T = job.wl.BH, job.wl.G, job.wl.D, job.T
+    st = torch.as_tensor(sel, device=job.kc.mask.device)
+    m_g = job.kc.mask.reshape(BH, S, 4)[st].cpu().numpy().view(np.uint32)
+    S32 = (S + 31) // 32 * 32
+    v_g = (job.kc.vals.reshape(BH, S32 // 32, T, 32)[st].float().permute(0, 1, 3, 2)
+           .reshape(len(sel), S32, T)[:, :S].cpu().numpy()) if T > 0 else np.zeros((len(sel), S, 0), np.float32)
+    s_g = job.kc.stats.reshape(BH, 4)[st].cpu().numpy()
+    rows = torch.as_tensor(np.concatenate([np.arange(b * G, (b + 1) * G) for b in sel]), device=job.out.device)
+    o_g = job.out.reshape(BH * G, D)[rows].cpu().numpy().reshape(len(sel), G, D)
+    mask_bad = vals_bad = 0
+    stats_rel = out_abs = ref_abs = 0.0
+    for i, ((qn, (m_o, v_o, s_o)), o_o) in enumerate(zip(prs, outs)):
+        same = np.all(m_g[i] == m_o[0], axis=-1)
+        mask_bad += int((~same).sum())
+        vals_bad += int((~np.all(v_g[i][same] == v_o[0][same], axis=-1)).sum())
+        den = np.maximum(np.abs(s_o[0, 1:3]), 1e-300)
+        stats_rel = max(stats_rel, float(np.max(np.abs(s_g[i, 1:3] - s_o[0, 1:3]) / den)))
+        out_abs = max(out_abs, float(np.max(np.abs(o_g[i].astype(np.float64) - o_o.reshape(G, D)))))
+        ref_abs = max(ref_abs, float(np.max(np.abs(o_o))))
+    return {"units": len(sel), "tokens": len(sel) * S, "mask_mismatch_tokens": mask_bad,
+            "vals_mismatch_tokens": vals_bad, "stats_max_rel_err": stats_rel,
+            "decode_max_abs_err": out_abs, "decode_max_abs_ref": ref_abs}
 
 
 def run_gpu(args):
