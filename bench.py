@@ -200,8 +200,9 @@ def _max_over_ranks(x: float, dist_on: bool) -> float:
 
 
 def _traffic_record(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel (else None)."""
+    """The committed ncu record of a kernel (DRAM bytes per launch, issue and
+    pipe counters), if it was taken on the current source of the kernel
+    (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -216,7 +217,7 @@ def _traffic_record(kernel: str, workload: str):
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except Exception:
         return None
-    return rec["bytes_per_launch"] if h == rec["source_sha"] else None
+    return rec if h == rec["source_sha"] else None
 
 
 def _cpu_model() -> str:
@@ -389,7 +390,12 @@ def run_gpu(args):
     dom_ms = spans[dom]
     achieved = bm[dom] / (dom_ms / 1e3) / 1e9
     kernel_name = {"prune": "prune_kernel", "decode": "decode_kernel", "snapkv": "snap_tc_kernel"}[dom]
-    traffic = _traffic_record(kernel_name, wl.name) if dom != "snapkv" else None
+    rec = _traffic_record(kernel_name, wl.name) if dom != "snapkv" else None
+    traffic = rec["bytes_per_launch"] if rec else None
+    # what bounds the kernel, from the same capture: the HBM fraction above
+    # is the roofline; these say which on-chip resource is the limit instead
+    limiter = ({"source": "ncu --set full of the same kernel source (" + rec["captured_on"] + ")",
+                **rec.get("ncu_counters", {})} if rec else None)
     timing = {"prune": "CUDA events around spark_prune on its stream (qnorm and stats, the two small "
                        "kernels launched with it, included)",
               "decode": "CUDA events around spark_decode_attn on its stream (the combine kernel "
@@ -433,7 +439,7 @@ def run_gpu(args):
                         "bytes_per_step": bm["snapkv"]} if wl.keep else None),
             "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic,
+                         "traffic": traffic, "limiter": limiter,
                          "bytes_per_launch": bm[dom], "entry": {"prune": "spark_prune",
                                                                 "decode": "spark_decode_attn",
                                                                 "snapkv": "spark_snapkv_evict"}[dom],

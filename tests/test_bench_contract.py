@@ -71,3 +71,15 @@ def test_byte_model_eviction():
     # keys read once for the scores, kept K and V rows read and written
     assert bm["snapkv"] >= BH * S * 256 + 4 * BH * keep * 256
     assert bm["prune"] >= BH * keep * (256 + 16 + 128)
+
+
+def test_traffic_record_matches_source():
+    """The committed ncu record is reported only for the kernel source it
+    was taken on, with its DRAM bytes and issue/pipe counters."""
+    rec = bench._traffic_record("prune_kernel", "long")
+    if rec is None:
+        pytest.skip("prune.cu changed since the committed capture")
+    assert rec["bytes_per_launch"] > 0
+    c = rec["ncu_counters"]
+    assert 0 < c["issue_active_pct"] <= 100 and c["warp_inst_per_token_head"] > 0
+    assert bench._traffic_record("no_such_kernel", "long") is None
