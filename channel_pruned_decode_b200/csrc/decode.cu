@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         ws.tabq = ws.pT + G * kWT;
         ws.tabc = ws.tabq + kD * G;
         ws.pdup = ws.tabc + kD;
-        ws.qc = ws.pdup + kWT * G * 2;
+        ws.qc = ws.pdup + dec_pdup_bytes(G, es) / sizeof(float);
         ws.bars = reinterpret_cast<uint64_t *>(ws.qc + 16);
         ws.stages = base + dec_table_bytes(G, es);
         ws.vstage_off = (uint32_t)dec_stage_bytes(a.T, es);
@@ -1028,10 +1028,11 @@ DecodeGeom decode_geometry(long BH, int S, int T, int Tv, int es, int G, int num
         const size_t wb = (table + ns * stage + 127) / 128 * 128;
         return (int)std::min<size_t>(max_w, budget / wb);
     };
-    // a 4-deep ring if all warps still fit, else 3 deep with >= 3/4 of them,
-    // else 2 deep with as many warps as fit
+    // a 4-deep ring if all warps still fit, else 3 deep with >= 3/4 of them
+    // unless 2 deep fits more warps (at T = 64: 11 warps of 2 stages ran
+    // 4-7 % faster than 9 of 3), else 2 deep with as many warps as fit
     if (warps_for(4) >= max_w) g.nstage = 4;
-    else if (warps_for(3) >= max_w * 3 / 4) g.nstage = 3;
+    else if (warps_for(3) >= max_w * 3 / 4 && warps_for(3) >= warps_for(2)) g.nstage = 3;
     else g.nstage = 2;
     g.nwarp = std::max(1, warps_for(g.nstage));
     g.warp_bytes = (table + g.nstage * stage + 127) / 128 * 128;

@@ -77,13 +77,15 @@ __host__ __device__ inline size_t dec_stage_bytes(int T, int es) {
 }
 
 // Per-warp tables: bf16 values add a swizzled V tile [kWT][kD] (8 KB); then
-// p as [G][kWT] fp32, q' [kD][G], c [kD], p as duplicated pairs [kWT][G][2]
-// (fp32 values), Qc [16] and the ring's mbarriers; rounded to 128 bytes so
-// that the stages start aligned.
+// p as [G][kWT] fp32, q' [kD][G], c [kD], for fp32 values p as duplicated
+// pairs [kWT][G][2] (the CUDA-core P.V; bf16 values take p from the first
+// table), Qc [16] and the ring's mbarriers; rounded to 128 bytes so that the
+// stages start aligned.
 __host__ __device__ inline size_t dec_vtile_bytes(int es) { return es == 2 ? (size_t)kWT * kD * 2 : 0; }
+__host__ __device__ inline size_t dec_pdup_bytes(int G, int es) { return es == 2 ? 0 : (size_t)kWT * G * 8; }
 __host__ __device__ inline size_t dec_table_bytes(int G, int es) {
     const size_t b = dec_vtile_bytes(es) + (size_t)G * kWT * 4 + (size_t)kD * G * 4 + kD * 4 +
-                     (size_t)kWT * G * 8 + 64 + kMaxStagesW * 8;
+                     dec_pdup_bytes(G, es) + 64 + kMaxStagesW * 8;
     return (b + 127) / 128 * 128;
 }
 
