@@ -30,11 +30,6 @@ static size_t snapkv_workspace(long BH, int S, int W) {
     return kWsHeader + (size_t)BH * (size_t)(S - W) * 8 + snapkv_partials_bytes(BH);
 }
 
-static int elem_size(int dtype) {
-    return dtype == SPARK_F32 ? 4 : (dtype == SPARK_BF16 ? 2 : 0);
-}
-
-static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -44,22 +39,6 @@ static int num_sms() {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
         return 148;
     return n;
-}
-
-// shape checks shared by prune and decode; returns SPARK_OK or an error
-static int check_cache(const spark_kcache *kc) {
-    if (!kc) return SPARK_ERR_ARG;
-    if (kc->B < 0 || kc->Hkv < 0 || kc->S < 0) return SPARK_ERR_ARG;
-    if (elem_size(kc->dtype) == 0) return SPARK_ERR_ARG;
-    if (kc->D != kD) return SPARK_ERR_UNSUPPORTED;
-    if (kc->T < 0 || kc->T > kc->D) return SPARK_ERR_ARG;
-    if ((long)kc->B * kc->Hkv == 0) return SPARK_OK;
-    if (!kc->qn || !kc->stats || !aligned16(kc->qn) || !aligned16(kc->stats)) return SPARK_ERR_ARG;
-    if (kc->S > 0) {
-        if (!kc->mask || !aligned16(kc->mask)) return SPARK_ERR_ARG;
-        if (kc->T > 0 && (!kc->vals || !aligned16(kc->vals))) return SPARK_ERR_ARG;
-    }
-    return SPARK_OK;
 }
 
 // Self-test of the bounded-wait path: one warp waits on an mbarrier that
@@ -142,17 +121,25 @@ size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D, int T,
 
 int spark_prune(const void *k, const void *q_obs, int G, int W, const spark_kcache *out,
                 void *workspace, size_t ws_bytes, void *stream) {
-    int rc = check_cache(out);
+    const int rc = check_prune_args(k, q_obs, G, W, out);
     if (rc != SPARK_OK) return rc;
-    if (G < 1 || W < 1) return SPARK_ERR_ARG;
     const long BH = (long)out->B * out->Hkv;
     if (BH == 0) return SPARK_OK;
-    if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
-    if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
     if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
     if (ws_bytes < prune_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
     cudaError_t e = launch_prune(k, q_obs, G, W, *out, workspace, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_group_budget(int D, int g, const float *rates, int *Tg) {
+    if (!rates || !Tg || D <= 0 || g < 1 || g > kMaxGroups || g > D) return SPARK_ERR_ARG;
+    for (int q = 0; q < g; ++q)
+        if (!(rates[q] >= 0.0f && rates[q] <= 1.0f)) return SPARK_ERR_ARG;
+    for (int q = 0; q < g; ++q) {
+        const int size = (q + 1) * D / g - q * D / g;
+        Tg[q] = (int)llround((1.0 - (double)rates[q]) * (double)size);
+    }
+    return SPARK_OK;
 }
 
 int spark_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups, const int *group_T,

@@ -1051,19 +1051,15 @@ cudaError_t launch_prune_topp(const void *k, const void *q_obs, int G, int W, fl
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB on every device
 static __device__ __align__(256) unsigned char g_prune_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-static void *g_prune_scratch_addr[kMaxDevices];  // device address per device id
-
-// Device address of the scratch array on `dev` (the current device).  Host
-// code cannot use the symbol itself: in host code it names a host-side
-// stand-in.  Looked up once per device; racing first calls store the same
-// value.
-static void *prune_scratch(int dev) {
-    if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    void *p = __atomic_load_n(&g_prune_scratch_addr[dev], __ATOMIC_ACQUIRE);
-    if (p) return p;
-    if (cudaGetSymbolAddress(&p, g_prune_scratch) != cudaSuccess || !p) return nullptr;
-    __atomic_store_n(&g_prune_scratch_addr[dev], p, __ATOMIC_RELEASE);
+// Device address of the scratch array in the current context.  Host code
+// cannot use the symbol itself: there it names a host-side stand-in.  The
+// address is looked up on every call rather than cached: after a device
+// reset, or under another context of the same device, the module is loaded
+// again and the array can sit elsewhere.  The first lookup in a context loads
+// the module (set-up); later ones read the runtime's table.
+static void *prune_scratch() {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_prune_scratch) != cudaSuccess) return nullptr;
     return p;
 }
 
@@ -1072,26 +1068,13 @@ static void *prune_scratch(int dev) {
 extern "C" SPARK_API int spark_prune_noalloc(const void *k, const void *q_obs, int G, int W,
                                              const spark_kcache *out, void *stream) {
     using namespace spark;
-    if (!out) return SPARK_ERR_ARG;
-    if (out->B < 0 || out->Hkv < 0 || out->S < 0) return SPARK_ERR_ARG;
-    if (out->dtype != SPARK_F32 && out->dtype != SPARK_BF16) return SPARK_ERR_ARG;
-    if (out->D != kD) return SPARK_ERR_UNSUPPORTED;
-    if (out->T < 0 || out->T > out->D || G < 1 || W < 1) return SPARK_ERR_ARG;
+    const int rc = check_prune_args(k, q_obs, G, W, out);
+    if (rc != SPARK_OK) return rc;
     const long BH = (long)out->B * out->Hkv;
     if (BH == 0) return SPARK_OK;
-    auto a16 = [](const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    if (!a16(q_obs) || !a16(out->qn) || !a16(out->stats)) return SPARK_ERR_ARG;
-    if (out->S > 0 && (!a16(k) || !a16(out->mask))) return SPARK_ERR_ARG;
-    if (out->S > 0 && out->T > 0 && !a16(out->vals)) return SPARK_ERR_ARG;
     if (prune_workspace(BH, out->S) > kNoAllocScratchBytes) return SPARK_ERR_WORKSPACE;
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SPARK_ERR_CUDA;
-    void *ws = prune_scratch(dev);
+    void *ws = prune_scratch();
     if (!ws) return SPARK_ERR_CUDA;
     cudaError_t e = launch_prune(k, q_obs, G, W, *out, ws, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
-
-namespace spark {
-
-}  // namespace spark

@@ -16,6 +16,41 @@ constexpr int kMaskWords = kD / 32;   // 128-bit channel mask per token
 constexpr int kWsHeader = 256;        // status word + padding at workspace start
 constexpr uint32_t kDevTimeout = 1u;  // status bit: a bounded wait ran out
 
+// ------------------------------------------------------- argument checks
+inline int elem_size(int dtype) { return dtype == SPARK_F32 ? 4 : (dtype == SPARK_BF16 ? 2 : 0); }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape and pointer checks of a cache descriptor shared by every entry point
+// that reads or writes one; returns SPARK_OK or the error status.
+inline int check_cache(const spark_kcache *kc) {
+    if (!kc) return SPARK_ERR_ARG;
+    if (kc->B < 0 || kc->Hkv < 0 || kc->S < 0) return SPARK_ERR_ARG;
+    if (elem_size(kc->dtype) == 0) return SPARK_ERR_ARG;
+    if (kc->D != kD) return SPARK_ERR_UNSUPPORTED;
+    if (kc->T < 0 || kc->T > kc->D) return SPARK_ERR_ARG;
+    if ((long)kc->B * kc->Hkv == 0) return SPARK_OK;
+    if (!kc->qn || !kc->stats || !aligned16(kc->qn) || !aligned16(kc->stats)) return SPARK_ERR_ARG;
+    if (kc->S > 0) {
+        if (!kc->mask || !aligned16(kc->mask)) return SPARK_ERR_ARG;
+        if (kc->T > 0 && (!kc->vals || !aligned16(kc->vals))) return SPARK_ERR_ARG;
+    }
+    return SPARK_OK;
+}
+
+// Every check of spark_prune's arguments except the workspace: the cache
+// descriptor, the window sizes and the input pointers.  spark_prune and its
+// allocation-free variant differ only in where the scratch comes from.
+inline int check_prune_args(const void *k, const void *q_obs, int G, int W, const spark_kcache *out) {
+    const int rc = check_cache(out);
+    if (rc != SPARK_OK) return rc;
+    if (G < 1 || W < 1) return SPARK_ERR_ARG;
+    if ((long)out->B * out->Hkv == 0) return SPARK_OK;
+    if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
+    if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
+    return SPARK_OK;
+}
+
 // ----------------------------------------------------------------- prune
 constexpr int kPruneThreads = 128;    // 4 lanes per token, 32 tokens per group
 constexpr int kPruneGroups = 8;       // fewest 32-token groups per CTA (256 tokens)
