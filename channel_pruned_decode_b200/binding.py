@@ -10,7 +10,6 @@ import ctypes
 import os
 from dataclasses import dataclass
 
-import numpy as np
 import torch
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspark.so")
@@ -33,7 +32,7 @@ SPARK_OP_THINK = 3
 SPARK_OP_TOPP = 4
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
-           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_prune_values", "spark_prune_think", "spark_prune_topp", "spark_decode_attn",
+           "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_group_budget", "spark_prune_values", "spark_prune_think", "spark_prune_topp", "spark_decode_attn",
            "spark_decode_attn_topp",
            "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_selftest_wait_timeout", "spark_tail_append", "spark_device_status",
            "spark_status_str", "spark_snapkv_evict")
@@ -77,6 +76,8 @@ def lib():
         L.spark_prune_noalloc.restype = I
         L.spark_prune_grouped.argtypes = [P, P, I, I, I, ctypes.POINTER(I), ctypes.POINTER(spark_kcache), P, Z, P]
         L.spark_prune_grouped.restype = I
+        L.spark_group_budget.argtypes = [I, I, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(I)]
+        L.spark_group_budget.restype = I
         L.spark_prune_values.argtypes = [P, ctypes.POINTER(spark_kcache), P, Z, P]
         L.spark_prune_values.restype = I
         L.spark_prune_think.argtypes = [P, P, I, I, ctypes.POINTER(spark_kcache), P, Z, P]
@@ -280,15 +281,14 @@ def spark_workspace_bytes_kv(B: int, Hkv: int, G: int, S: int, D: int, T: int, T
 
 
 def spark_group_budget(D: int, rates) -> list:
-    """Per-group kept-channel budgets round((1 - rate) * group size), half
-    away from zero, for len(rates) equal-rank groups of D channels."""
+    """Per-group kept-channel budgets of SparK-g (the C library's
+    spark_group_budget): round((1 - rate) * group size), half away from zero,
+    for len(rates) equal-rank groups of D channels."""
     g = len(rates)
-    out = []
-    for q, r in enumerate(rates):
-        size = (q + 1) * D // g - q * D // g
-        x = (1.0 - float(np.float32(r))) * size
-        out.append(int(np.floor(x + 0.5)) if x >= 0 else -int(np.floor(-x + 0.5)))
-    return out
+    arr = (ctypes.c_float * max(g, 1))(*[float(r) for r in rates])
+    out = (ctypes.c_int * max(g, 1))()
+    _check(lib().spark_group_budget(D, g, arr, out), "spark_group_budget")
+    return [int(out[q]) for q in range(g)]
 
 
 def spark_decode_attn(q: torch.Tensor, kc: KCache, v: torch.Tensor, k_tail, v_tail, tail_cap: int,

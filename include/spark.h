@@ -17,8 +17,10 @@
  *
  * Conventions shared by every entry point
  *   - All tensor arguments are DEVICE pointers owned by the caller; the
- *     library never allocates, frees, synchronises or prints.  Every launch
- *     is asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *     library never allocates, frees or prints, and no entry point
+ *     synchronises except spark_device_status, which waits for `stream` so
+ *     that it can read the status word.  Every launch is asynchronous on
+ *     `stream` (a cudaStream_t; NULL = legacy default).
  *   - Tensors are dense row-major; pointers must be 16-byte aligned.
  *   - dtype: SPARK_F32 (fp32) or SPARK_BF16 (bf16) for keys, values and
  *     queries.  D must be 128.  Saliency, norms and attention arithmetic run
@@ -159,6 +161,22 @@ SPARK_API int spark_prune(const void *k, const void *q_obs, int G, int W,
  * unchanged.  With pruning rates r_q, group_T[q] = round((1 - r_q) * |group q|)
  * (half away from zero).  Returns SPARK_ERR_ARG on bad budgets.
  */
+/*
+ * SparK-g budgets ([W] 5.2: g groups, each with its own pruning rate, e.g.
+ * g = 4 with rates (0.25, 0.5, 0.75, 1.0)).  With the groups of
+ * spark_prune_grouped (group q holds the ranks [q*D/g, (q+1)*D/g), integer
+ * division), writes Tg[q] = round((1 - rates[q]) * |group q|) for q < g,
+ * halves away from zero, computed in fp64 from the fp32 rate.  The sum of Tg
+ * is the out->T that spark_prune_grouped expects.
+ *   D      channels per head, D > 0 (the pruning entry points need 128)
+ *   g      number of groups, 1 <= g <= min(8, D)
+ *   rates  host array of g pruning rates, each in [0, 1]
+ *   Tg     host array of g ints, written only on success
+ * Returns SPARK_ERR_ARG on a NULL array, g or D out of range, or a rate
+ * outside [0, 1] (NaN included).  Host arithmetic only; launches nothing.
+ */
+SPARK_API int spark_group_budget(int D, int g, const float *rates, int *Tg);
+
 SPARK_API int spark_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_groups,
                                   const int *group_T, const spark_kcache *out, void *workspace,
                                   size_t ws_bytes, void *stream);
@@ -262,8 +280,10 @@ SPARK_API int spark_prune_think(const void *k, const void *q_obs, int G, int W, 
  * 256 + 16 * B * Hkv * ceil(S / 256) bytes of it and returns
  * SPARK_ERR_WORKSPACE (launching nothing) when that exceeds 4 MiB, i.e.
  * when B * Hkv * ceil(S / 256) > 262128.
- * The first call on a device looks up the array's device address with
- * cudaGetSymbolAddress (that device must be current); make that first call
+ * Every call looks up the array's device address in the current context
+ * with cudaGetSymbolAddress, so the entry point stays valid after a device
+ * reset or under another context of the device.  The first call in a context
+ * also loads the library's device code there (set-up); make that first call
  * before any stream capture.  All calls share the array and it keeps the
  * last call's contents (every value a call reads it writes first), so calls
  * whose kernels overlap on the GPU -- on different streams, or from several

@@ -186,6 +186,68 @@ def test_prune_grouped_rejects_bad_budgets(L):
 def test_group_budget_matches_oracle():
     for rates in ([0.25, 0.5, 0.75, 1.0], [0.5] * 5, [0.1, 0.3, 0.5, 0.7, 0.9], [0.0] * 8, [1.0] * 3, [0.33] * 7):
         assert B.spark_group_budget(128, rates) == oracle.group_budget(128, rates)
+    # the pages' g = 4 rates over 128 channels: groups of 32 keep 24, 16, 8, 0
+    assert B.spark_group_budget(128, [0.25, 0.5, 0.75, 1.0]) == [24, 16, 8, 0]
+
+
+def test_group_budget_rejects_bad_args(L):
+    F, I = ctypes.c_float, ctypes.c_int
+    rates, out = (F * 9)(*([0.5] * 9)), (I * 9)(*([-7] * 9))
+    assert L.spark_group_budget(128, 0, rates, out) == B.SPARK_ERR_ARG        # no groups
+    assert L.spark_group_budget(128, 9, rates, out) == B.SPARK_ERR_ARG        # more than 8
+    assert L.spark_group_budget(2, 4, rates, out) == B.SPARK_ERR_ARG          # more groups than channels
+    assert L.spark_group_budget(0, 1, rates, out) == B.SPARK_ERR_ARG
+    assert L.spark_group_budget(128, 4, None, out) == B.SPARK_ERR_ARG
+    assert L.spark_group_budget(128, 4, rates, None) == B.SPARK_ERR_ARG
+    for bad in (-0.01, 1.01, float("nan")):
+        r = (F * 4)(0.5, bad, 0.5, 0.5)
+        assert L.spark_group_budget(128, 4, r, out) == B.SPARK_ERR_ARG
+    assert list(out) == [-7] * 9                                             # untouched on error
+
+
+C_PROGRAM = r"""
+#include <math.h>
+#include <stdio.h>
+#include "spark.h"
+
+int main(void) {
+    /* lambda -> T and the cache / workspace sizes are host arithmetic */
+    if (spark_lambda_to_T(0.8f, 128) != 26 || spark_lambda_to_T(1.5f, 128) != -1) return 1;
+    size_t sizes[4];
+    const size_t total = spark_cache_sizes(1, 8, 32768, 128, 64, SPARK_BF16, sizes);
+    if (total == 0 || sizes[0] != (size_t)8 * 32768 * 16) return 2;
+    if (spark_cache_bytes(1, 8, 32768, 128, 64, SPARK_BF16) != total) return 3;
+    if (spark_workspace_bytes(SPARK_OP_PRUNE, 1, 8, 4, 32768, 128, 64, 0) == 0) return 4;
+    if (spark_workspace_bytes(SPARK_OP_PRUNE, 1, 8, 4, 32768, 64, 64, 0) != 0) return 5;
+    const float rates[4] = {0.25f, 0.5f, 0.75f, 1.0f};
+    int Tg[4];
+    if (spark_group_budget(128, 4, rates, Tg) != SPARK_OK) return 6;
+    if (Tg[0] != 24 || Tg[1] != 16 || Tg[2] != 8 || Tg[3] != 0) return 7;
+    /* argument errors come back before anything is launched */
+    if (spark_prune(NULL, NULL, 4, 32, NULL, NULL, 0, NULL) != SPARK_ERR_ARG) return 8;
+    spark_kcache kc = {1, 8, 32768, 96, 64, SPARK_BF16, NULL, NULL, NULL, NULL};
+    if (spark_prune(NULL, NULL, 4, 32, &kc, NULL, 0, NULL) != SPARK_ERR_UNSUPPORTED) return 9;
+    if (spark_status_str(SPARK_ERR_ARG) == NULL) return 10;
+    printf("ok %zu\n", total);
+    return 0;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(L, tmp_path):
+    # a C11 caller: the header must be valid C on its own, and the calls above
+    # must link against and run with libspark.so (host arithmetic and argument
+    # errors only, so no GPU is needed)
+    src = tmp_path / "caller.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(B._LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lspark",
+                    f"-Wl,-rpath,{libdir}", "-lm"], check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith("ok ")
 
 
 def test_value_pruning_entry_points_reject_bad_args(L):
