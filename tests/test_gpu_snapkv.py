@@ -100,15 +100,28 @@ def test_evict_then_prune_then_decode_256_steps():
     np.testing.assert_allclose(_gpu_scores(ws, BH, S - W)[sel], sc_o, rtol=2e-4, atol=1e-7)
     pooled = oracle.snapkv_pool(sc_o, wl.pool)
     idx_o = oracle.snapkv_select(pooled, S, W, keep)
-    swaps = _check_selection(idx.reshape(BH, keep).cpu().numpy()[sel], idx_o, pooled, keep, W)
+    idx_g = idx.reshape(BH, keep).cpu().numpy()
+    swaps = _check_selection(idx_g[sel], idx_o, pooled, keep, W)
     assert swaps <= max(1, 1e-4 * len(sel) * (keep - W))
+    # the gather on every one of the 256 heads: kept K and V rows are the
+    # source rows at the kept indices, bit for bit
+    ig = idx.reshape(BH, keep).long()
+    for src, dst in ((pre["k"], k_out), (pre["v"], v_out)):
+        want = torch.gather(src.reshape(BH, S, D), 1, ig[..., None].expand(-1, -1, D))
+        assert torch.equal(dst.reshape(BH, keep, D), want)
 
-    # stacked: prune the compacted keys with the same window queries
+    # stacked: prune the compacted keys with the same window queries.  The
+    # oracle's side gathers the keys at the oracle's own kept indices, on the
+    # sampled heads whose kept set agrees with the GPU's
+    agree = np.array([np.array_equal(idx_g[b], idx_o[i]) for i, b in enumerate(sel)])
+    assert agree.sum() >= len(sel) - 1
+    sel, idx_o, k_np = sel[agree], idx_o[agree], k_np[agree]
+    q_np = q_np.reshape(-1, G, W, D)[agree].reshape(-1, W, D)
     T = spark_lambda_to_T(wl.lam)
     kc = run_prune(k_out, pre["q_obs"], G, W, T)
     torch.cuda.synchronize()
     selt = torch.as_tensor(sel, device=DEV)
-    kc_np = to_np(k_out.reshape(BH, keep, D)[selt])
+    kc_np = np.take_along_axis(k_np, idx_o[..., None].astype(np.int64), axis=1)
     qn_o = oracle.qnorm(q_np, G)
     m_o, v_o, st_o = oracle.prune(kc_np, qn_o, T)
     m_g = mask_np(kc)[sel]
@@ -120,7 +133,8 @@ def test_evict_then_prune_then_decode_256_steps():
     wsd = workspace(spark_workspace_bytes(SPARK_OP_DECODE, wl.rows, wl.Hkv, G, keep, D, T, cap))
     out = torch.empty((wl.rows, wl.Hq, D), dtype=torch.float32, device=DEV)
     qsel = torch.as_tensor(np.concatenate([np.arange(b * G, (b + 1) * G) for b in sel]), device=DEV)
-    vv_np = to_np(v_out.reshape(BH, keep, D)[selt])
+    v_src = to_np(pre["v"].reshape(BH, S, D)[selt])
+    vv_np = np.take_along_axis(v_src, idx_o[..., None].astype(np.int64), axis=1)
     for step in range(wl.steps):
         stp = make_decode_step(wl, step, DEV)
         spark_tail_append(stp["k_new"], stp["v_new"], kt, vt, wl.rows, wl.Hkv, D, cap, step)
