@@ -157,45 +157,19 @@ void oracle_prune(const float *k, const float *qn, long BH, long S, int D,
  * the token's total.  Reading R19 (the pages fix neither the arithmetic of
  * the cumulative sum nor the storage):
  *   - channels are taken in the greedy order of [W] 3.1 (saliency desc,
- *     lower channel first on ties, R3); the kept set is the shortest prefix
- *     of that order whose mass reaches the target;
- *   - the mass of a channel set is an fp32 sum in one fixed order: within
- *     each block of 32 channels in ascending channel order starting from
- *     +0, then the block sums pairwise, adjacent blocks first
- *     ((B0 + B1) + (B2 + B3) for D = 128); channels outside the set add
- *     nothing;
- *   - target = fp32(p * mass(all channels)); "reaches" is >=, so a token
- *     whose saliencies are all 0 keeps nothing;
+ *     lower channel first on ties, R3); the cumulative saliency of the first
+ *     n channels of that order is P(n), accumulated in fp64 in that order
+ *     (fp32 saliencies, so P(n) is the exact sum up to fp64 rounding: a
+ *     relative error below 2^-46 for D = 128);
+ *   - total = P(D); target = p * total in fp64; the kept set is the shortest
+ *     prefix with P(n) >= target ("reaches" is >=, so a token whose
+ *     saliencies are all 0, or p = 0, keeps nothing);
  *   - the cache has a capacity of Tcap values per token: a longer prefix is
  *     cut to its first Tcap channels.  vals keeps the kept values in
  *     ascending channel order in the first slots of the token's Tcap slots,
  *     zeros after;
  *   - statistics over the pruned entries as in oracle_prune.
  */
-
-/* fp32 mass of the channels with in[j] != 0 (order of R19). */
-static float topp_mass(const float *w, const unsigned char *in, int D)
-{
-    float blk[64];
-    int nb = 0;
-    for (int b0 = 0; b0 < D; b0 += 32) {
-        float acc = 0.0f;
-        for (int j = b0; j < D && j < b0 + 32; ++j)
-            if (in[j])
-                acc = acc + w[j];
-        blk[nb++] = acc;
-    }
-    while (nb > 1) {
-        int m = 0;
-        for (int i = 0; i + 1 < nb; i += 2)
-            blk[m++] = blk[i] + blk[i + 1];
-        if (nb & 1)
-            blk[m++] = blk[nb - 1];
-        nb = m;
-    }
-    return nb ? blk[0] : 0.0f;
-}
-
 void oracle_prune_topp(const float *k, const float *qn, long BH, long S, int D, float p, int Tcap,
                        uint32_t *mask, float *vals, double *stats)
 {
@@ -213,22 +187,19 @@ void oracle_prune_topp(const float *k, const float *qn, long BH, long S, int D, 
                 order[j].j = j;
             }
             qsort(order, (size_t)D, sizeof(chan_score), by_saliency_desc);
-            memset(in, 1, (size_t)D);
-            const float target = p * topp_mass(w, in, D);
-            /* shortest prefix: the mass of a prefix never decreases as it
-             * grows (each rounding is monotone), so bisect on its length */
-            int lo = 0, hi = D;  /* mass(prefix hi) >= target always holds */
-            while (lo < hi) {
-                const int mid = lo + (hi - lo) / 2;
-                memset(in, 0, (size_t)D);
-                for (int r = 0; r < mid; ++r)
-                    in[order[r].j] = 1;
-                if (topp_mass(w, in, D) >= target)
-                    hi = mid;
-                else
-                    lo = mid + 1;
+            double total = 0.0;
+            for (int r = 0; r < D; ++r)
+                total += (double)order[r].w;
+            const double target = (double)p * total;
+            /* the shortest greedy prefix whose cumulative saliency reaches
+             * the target (P(0) = 0) */
+            int n = 0;
+            double cum = 0.0;
+            while (n < D && cum < target) {
+                cum += (double)order[n].w;
+                n += 1;
             }
-            const int n_keep = lo < Tcap ? lo : Tcap;
+            const int n_keep = n < Tcap ? n : Tcap;
             memset(in, 0, (size_t)D);
             for (int r = 0; r < n_keep; ++r)
                 in[order[r].j] = 1;

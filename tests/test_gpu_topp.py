@@ -1,9 +1,14 @@
 """GPU parity of SparK-p (spark_prune_topp / spark_decode_attn_topp) against
-the oracle's prune_topp on the same seeded inputs.  The mass of a channel set
-is defined in fp32 in one fixed order on both sides, so masks, kept values
-(zero padding included) and the pruned count are compared bit for bit, the
-saliency sums to fp32-partial rounding, and decode within the attention
-tolerance.  Full-size heads are checked on sampled tokens."""
+the oracle's prune_topp on the same seeded inputs.  The oracle sums the
+cumulative saliency in fp64 (reading R19); the GPU may decide a token's
+boundary in other arithmetic, so a token's kept set may differ from the
+oracle's only at a counted near-tie: the GPU's set is still a greedy prefix
+and the exact cumulative saliency at the differing boundary lies within fp32
+rounding of the target (2^-23 * D * total).  Such tokens must stay under
+0.01 %.  Kept values (zero padding included) are compared bit for bit on
+every other token, the pruned count and saliency sums through the
+statistics, and decode within the attention tolerance.  Full-size heads are
+checked on sampled tokens."""
 import numpy as np
 import pytest
 import torch
@@ -30,21 +35,51 @@ def run_topp(k, q_obs, G, W, p, Tcap):
     return kc
 
 
+def topp_near_ties(m_g, m_o, k_np, qn_np, p, Tcap):
+    """Tokens whose GPU kept set differs from the oracle's, and how many of
+    them are counted near-ties (see the module docstring).  A differing token
+    that is not a greedy prefix, or not near a tie, is never counted."""
+    diff = np.argwhere(np.any(m_g != m_o, axis=-1))
+    near = 0
+    for bh, t in diff:
+        w = (qn_np[bh] * np.abs(k_np[bh, t])).astype(np.float32).astype(np.float64)
+        order = sorted(range(D), key=lambda j: (-w[j], j))
+        kept = [j for j in range(D) if (int(m_g[bh, t, j // 32]) >> (j % 32)) & 1]
+        n_g = len(kept)
+        if sorted(order[:n_g]) != kept or n_g > Tcap:
+            continue
+        total = float(np.sum(w))
+        target = float(np.float32(p)) * total
+        tol = 2.0 ** -23 * D * total
+        pre = np.concatenate([[0.0], np.cumsum(w[order])])
+        n_o = int(np.searchsorted(pre >= target, True)) if total > 0 else 0
+        if n_g < min(n_o, Tcap) and target - pre[n_g] <= tol:
+            near += 1
+        elif n_g > n_o and pre[n_g - 1] - target <= tol:
+            near += 1
+    return len(diff), near
+
+
 def check_topp(kc, k_np, q_np, G, p, what):
     BH, S, Tcap = kc.B * kc.Hkv, kc.S, kc.T
     qn = oracle.qnorm(q_np.reshape(BH * G, -1, D), G)
     assert np.array_equal(kc.qn.cpu().numpy().reshape(BH, D).view(np.uint32), qn.view(np.uint32)), what
     m_o, v_o, s_o = oracle.prune_topp(k_np.reshape(BH, S, D), qn, p, Tcap)
     s_g = kc.stats.cpu().numpy().reshape(BH, 4)
-    assert np.array_equal(s_g[:, 0], s_o[:, 0]), f"{what}: pruned count"
-    np.testing.assert_allclose(s_g[:, 1:], s_o[:, 1:], rtol=STATS_RTOL, atol=0, err_msg=what)
     if S == 0:
+        assert np.array_equal(s_g[:, 0], s_o[:, 0]), f"{what}: pruned count"
         return qn, m_o, v_o, s_o
     m_g = mask_np(kc)
-    bad = np.argwhere(np.any(m_g != m_o, axis=-1))
-    assert len(bad) == 0, f"{what}: {len(bad)} tokens differ, first {bad[:4].tolist()}"
+    n_diff, near = topp_near_ties(m_g, m_o, k_np.reshape(BH, S, D), qn, p, Tcap)
+    assert n_diff == near, f"{what}: {n_diff - near} of {n_diff} differing tokens are not near-ties"
+    assert n_diff <= 1e-4 * BH * S, f"{what}: {n_diff} near-tie tokens of {BH * S}"
+    ok = np.all(m_g == m_o, axis=-1)
     if Tcap > 0:
-        assert np.array_equal(unpack_vals(kc).view(np.uint32), v_o.view(np.uint32)), f"{what}: vals"
+        v_g = unpack_vals(kc)
+        assert np.array_equal(v_g[ok].view(np.uint32), v_o[ok].view(np.uint32)), f"{what}: vals"
+    if n_diff == 0:
+        assert np.array_equal(s_g[:, 0], s_o[:, 0]), f"{what}: pruned count"
+        np.testing.assert_allclose(s_g[:, 1:], s_o[:, 1:], rtol=STATS_RTOL, atol=0, err_msg=what)
     return qn, m_o, v_o, s_o
 
 
@@ -154,11 +189,15 @@ def test_topp_full_size_sampled():
     rng = np.random.default_rng(1)
     vals_g = unpack_vals(kc)
     k_np = to_np(pre["k"]).reshape(BH, S, D)
+    n_diff = n_near = 0
     for bh in range(BH):
-        ts = np.sort(rng.choice(S, 256, replace=False))
+        ts = np.sort(rng.choice(S, 4096, replace=False))
         m_o, v_o, _ = oracle.prune_topp(k_np[bh, ts][None], qn[bh:bh + 1], 0.99, Tcap)
-        assert np.array_equal(m_g[bh, ts], m_o[0]), f"head {bh}"
-        assert np.array_equal(vals_g[bh, ts].view(np.uint32), v_o[0].view(np.uint32)), f"head {bh}"
+        d, nr = topp_near_ties(m_g[bh, ts][None], m_o, k_np[bh, ts][None], qn[bh:bh + 1], 0.99, Tcap)
+        n_diff, n_near = n_diff + d, n_near + nr
+        ok = np.all(m_g[bh, ts] == m_o[0], axis=-1)
+        assert np.array_equal(vals_g[bh, ts][ok].view(np.uint32), v_o[0][ok].view(np.uint32)), f"head {bh}"
+    assert n_diff == n_near and n_diff <= 1e-4 * BH * 4096, (n_diff, n_near)
 
 
 @pytest.mark.parametrize("G", [1, 2, 8])

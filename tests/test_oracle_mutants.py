@@ -80,15 +80,11 @@ MUTANTS = {
     "think_recovers_mean": ("stats[bh * 4 + 3] = 0.0;\n    }\n    free(ord);",
                             "stats[bh * 4 + 3] = 1.0;\n    }\n    free(ord);"),
     # SparK-p (reading R19)
-    "topp_reach_strict": ("if (topp_mass(w, in, D) >= target)", "if (topp_mass(w, in, D) > target)"),
-    "topp_p_ignored": ("const float target = p * topp_mass(w, in, D);",
-                       "const float target = topp_mass(w, in, D);"),
-    "topp_blocks_sequential": ("        for (int i = 0; i + 1 < nb; i += 2)\n            blk[m++] = blk[i] + blk[i + 1];\n"
-                               "        if (nb & 1)\n            blk[m++] = blk[nb - 1];\n",
-                               "        blk[m++] = blk[0] + blk[1];\n        for (int i = 2; i < nb; ++i)\n"
-                               "            blk[m++] = blk[i];\n"),
-    "topp_one_block": ("for (int b0 = 0; b0 < D; b0 += 32) {", "for (int b0 = 0; b0 < D; b0 += D) {"),
-    "topp_cap_off_by_one": ("const int n_keep = lo < Tcap ? lo : Tcap;", "const int n_keep = lo < Tcap ? lo : Tcap - 1;"),
+    "topp_reach_strict": ("while (n < D && cum < target) {", "while (n < D && cum <= target) {"),
+    "topp_p_ignored": ("const double target = (double)p * total;", "const double target = total;"),
+    "topp_fp32_cumulative": ("            double cum = 0.0;\n", "            float cum = 0.0f;\n"),
+    "topp_channel_order": ("                cum += (double)order[n].w;", "                cum += (double)w[n];"),
+    "topp_cap_off_by_one": ("const int n_keep = n < Tcap ? n : Tcap;", "const int n_keep = n < Tcap ? n : Tcap - 1;"),
     "topp_padding_not_zero": ("vrow[r] = 0.0f;", "vrow[r] = 1.0f;"),
     "lambda_truncates": ("return (int)llround((1.0 - (double)lambda) * (double)D);",
                          "return (int)((1.0 - (double)lambda) * (double)D);"),

@@ -1,14 +1,16 @@
 """Pins for the SparK-p oracle (per-token top-p channel selection, reading
-R19 of the oracle: the shortest greedy prefix of channels whose fp32
-saliency mass reaches fp32(p * total), capped at Tcap).
+R19 of the oracle: the shortest greedy prefix of channels whose cumulative
+saliency, summed in fp64 in greedy order, reaches p times the token's total,
+capped at Tcap).
 
 Source: "KV Cache 还能再砍一刀：SparK ..." section 5.2 (SparK-p: every token
 keeps the fewest channels whose cumulative saliency reaches 99 %), with the
 greedy order and tie rule of section 3.1.  Each pin fixes a part of the
 oracle from outside it: a brute-force minimum over all channel subsets on
 exact (integer) saliencies, closed forms for p = 0 / p = 1 / all-zero
-tokens, the cap against plain top-T pruning, hand-built cases where the
-stated summation order decides the outcome, and invariants on random data.
+tokens, the cap against plain top-T pruning, hand-built cases whose exact
+sums an fp32 accumulation would get wrong, and invariants on random data
+checked with exact rational sums.
 """
 import itertools
 
@@ -74,31 +76,35 @@ def test_closed_forms():
     assert not m.any() and st[0, 0] == 2 * D and st[0, 3] == 0.0
 
 
-def test_summation_order_within_and_across_blocks():
-    """Cases where the fixed fp32 order of the mass decides the count."""
+def test_cumulative_sums_are_exact():
+    """Hand-built tokens whose exact cumulative saliency an fp32 running sum
+    would lose: the kept count follows the exact sums."""
     D = 128
     qn = np.ones((1, D), np.float32)
-    # (a) a 1.0 and 63 saliencies of 2^-25 in channels 1..63: inside block 0
-    # each tiny term is lost against 1.0 (half an ulp of 1 is 2^-24), block 1
-    # sums its 32 exactly to 2^-20 before meeting 1.0, so the total is
-    # 1 + 8 ulp.  A prefix holding channel 0, channels 1..31 and m channels of
-    # block 1 has mass fl(1 + (m / 4) ulp): 29 give 1 + 7 ulp, 30 round (tie
-    # to even) to 1 + 8 ulp.  So 1 + 31 + 30 = 62 channels.  (One sequential
-    # pass would lose every tiny term and keep 1 channel; exact sums, 64.)
+    # (a) a 1.0 and 63 saliencies of 2^-25 (channels 1..63).  Exactly, the
+    # total is 1 + 63 * 2^-25 and with p = 1 every one of the 64 nonzero
+    # channels is needed; an fp32 running sum from 1.0 loses every 2^-25 term
+    # (half an ulp of 1 is 2^-24) and would keep one channel.
     k = np.zeros((1, 1, D), np.float32)
     k[0, 0, 0] = 1.0
     k[0, 0, 1:64] = 2.0 ** -25
     m, v, st = oracle.prune_topp(k, qn, 1.0, D)
-    assert _kept(m[0, 0], D) == list(range(62))
-    # (b) blocks combine pairwise: 1.0 in block 0, 2^-24 in blocks 2 and 3.
-    # (B0 + B1) + (B2 + B3) = 1 + 2^-23 needs both tiny channels; with the
-    # prefix {0, 64} the mass (1 + 0) + (2^-24 + 0) rounds back to 1.
+    assert _kept(m[0, 0], D) == list(range(64))
+    # (b) 1.0 in channel 0, 2^-24 in channels 64 and 96: the exact total
+    # 1 + 2^-23 needs all three; the two equal saliencies go in channel order
     k = np.zeros((1, 1, D), np.float32)
     k[0, 0, 0] = 1.0
     k[0, 0, 64] = 2.0 ** -24
     k[0, 0, 96] = 2.0 ** -24
     m, v, st = oracle.prune_topp(k, qn, 1.0, D)
     assert _kept(m[0, 0], D) == [0, 64, 96]
+    # (c) p = 0.75 with saliencies 4, 1, 1, 1, 1 (total 8, target 6): the
+    # prefix {4, 1, 1} reaches 6 exactly (>= counts equality); the three
+    # equal ones taken in channel order
+    k = np.zeros((1, 1, D), np.float32)
+    k[0, 0, [3, 10, 20, 30, 40]] = [1.0, 4.0, 1.0, 1.0, 1.0]
+    m, v, st = oracle.prune_topp(k, qn, 0.75, D)
+    assert _kept(m[0, 0], D) == [3, 10, 20]
 
 
 def test_capacity_cut_equals_top_T():
@@ -123,21 +129,10 @@ def test_capacity_cut_equals_top_T():
     assert n_cut > 0
 
 
-def _mass(w, sel):
-    """fp32 mass in the order of R19 (blocks of 32 ascending, pairwise)."""
-    blocks = []
-    for b0 in range(0, len(w), 32):
-        acc = np.float32(0.0)
-        for j in range(b0, min(b0 + 32, len(w))):
-            if sel[j]:
-                acc = np.float32(acc + w[j])
-        blocks.append(acc)
-    while len(blocks) > 1:
-        nxt = [np.float32(blocks[i] + blocks[i + 1]) for i in range(0, len(blocks) - 1, 2)]
-        if len(blocks) % 2:
-            nxt.append(blocks[-1])
-        blocks = nxt
-    return blocks[0]
+def _exact(w, idx):
+    """Exact rational sum of the fp32 values w[idx]."""
+    from fractions import Fraction
+    return sum((Fraction(float(w[j])) for j in idx), Fraction(0))
 
 
 def test_invariants_lognormal_tokens():
@@ -160,13 +155,14 @@ def test_invariants_lognormal_tokens():
             n = len(kept)
             counts.append(n)
             assert sorted(order[:n]) == kept
-            target = np.float32(np.float32(p) * _mass(w, np.ones(D, bool)))
-            sel = np.zeros(D, bool)
-            sel[order[:n]] = True
-            assert _mass(w, sel) >= target
+            # with exact sums: the prefix reaches p of the total and one
+            # channel less does not (the fp64 sums of the oracle agree with
+            # the exact ones away from 1e-12 relative near-ties, none here)
+            from fractions import Fraction
+            target = Fraction(float(np.float32(p))) * _exact(w, range(D))
+            assert _exact(w, order[:n]) >= target
             if n > 0:
-                sel[order[n - 1]] = False
-                assert _mass(w, sel) < target
+                assert _exact(w, order[:n - 1]) < target
             assert np.array_equal(v[b, t, :n].view(np.uint32), k[b, t, kept].view(np.uint32))
             assert not v[b, t, n:].any()
             sw += float(np.sum(w.astype(np.float64)[[j for j in range(D) if j not in kept]]))
