@@ -688,12 +688,15 @@ cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W,
 // ---------------------------------------------------------------------------
 // SparK-p ("KV Cache 还能再砍一刀：SparK ..." section 5.2): every token keeps
 // the fewest channels, taken in the greedy order of section 3.1 (saliency
-// desc, lower channel first), whose saliency mass reaches p of its total,
-// at most Tcap of them.  The library's arithmetic for the mass of a channel
-// set (the pages leave it open): each lane adds its 32 channels in
-// ascending order in fp32 from +0, then the quad adds
-// (lane 0 + lane 1) + (lane 2 + lane 3); fp32 addition is commutative, so
-// every lane of the quad holds the same bits.  target = fp32(p * total).
+// desc, lower channel first), whose cumulative saliency reaches p of its
+// total, at most Tcap of them.  The decision is taken on fp64 sums of the
+// fp32 saliencies (the pages leave the arithmetic open).  The search below
+// first finds the boundary with fp32 masses: each lane adds its 32 channels
+// in ascending order in fp32 from +0, then the quad adds
+// (lane 0 + lane 1) + (lane 2 + lane 3) (fp32 addition is commutative, so
+// every lane of the quad holds the same bits), target = fp32(p * total).  An
+// fp64 check then moves the boundary where fp32 rounding put it on the wrong
+// side.
 //
 // A set {16-bit key >= P} is a threshold set of the exact keys (the 16-bit
 // key is monotone in them), hence a greedy prefix, and its mass M(P) does
@@ -904,6 +907,77 @@ __global__ void __launch_bounds__(kPruneThreads, 3)
                 if (open && (M >= target || wc >= 4 * kD)) open = false;
             }
             m = band ? mA : m;
+        }
+        // The fp32 search above finds a greedy prefix whose fp32 mass reaches
+        // the fp32 target.  The boundary itself is decided on the cumulative
+        // saliency in fp64 (each fp32 key is exact in fp64, sums of 128 keys
+        // round at 2^-46 relative): the prefix must reach target64 and, less
+        // its last channel in greedy order, fall short of it.  Tokens that
+        // fail (near-ties of the fp32 arithmetic) move the boundary one
+        // channel at a time in greedy order.
+        {
+            double tot64 = 0.0, m64 = 0.0;
+            float wl = __int_as_float(0x7f800000);  // smallest kept saliency
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float x = __uint_as_float(key[i]);
+                const bool in = (m >> i) & 1u;
+                tot64 = __dadd_rn(tot64, (double)x);
+                m64 = in ? __dadd_rn(m64, (double)x) : m64;
+                wl = in ? fminf(wl, x) : wl;
+            }
+#pragma unroll
+            for (int o = 1; o <= 2; o <<= 1) {
+                tot64 = __dadd_rn(tot64, __shfl_xor_sync(0xffffffffu, tot64, o));
+                m64 = __dadd_rn(m64, __shfl_xor_sync(0xffffffffu, m64, o));
+                wl = fminf(wl, __shfl_xor_sync(0xffffffffu, wl, o));
+            }
+            const double target64 = __dmul_rn((double)p, tot64);
+            const bool act64 = valid && target64 > 0.0 && Tcap > 0;
+            const bool some = quad_sum(__popc(m)) > 0;
+            if (!act64) m = 0u;  // p = 0 or no saliency: nothing to keep
+            bool open = act64 && (m64 < target64 || (some && __dsub_rn(m64, (double)wl) >= target64));
+            for (int it = 0; it < 2 * kD && __any_sync(0xffffffffu, open); ++it) {
+                // greedy-next channel outside the set: (key desc, channel asc);
+                // greedy-last inside it: (key asc, channel desc)
+                uint32_t nk = 0u, lk = 0xffffffffu;
+                int ni = -1, li = -1;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool in = (m >> i) & 1u;
+                    const bool tn = !in && (ni < 0 || key[i] > nk);
+                    nk = tn ? key[i] : nk;
+                    ni = tn ? i : ni;
+                    const bool tl2 = in && (li < 0 || key[i] <= lk);
+                    lk = tl2 ? key[i] : lk;
+                    li = tl2 ? i : li;
+                }
+                int nc = ni < 0 ? -1 : 32 * s + ni, lc = li < 0 ? -1 : 32 * s + li;
+#pragma unroll
+                for (int o = 1; o <= 2; o <<= 1) {
+                    const uint32_t onk = __shfl_xor_sync(0xffffffffu, nk, o);
+                    const int onc = __shfl_xor_sync(0xffffffffu, nc, o);
+                    const bool bn = onc >= 0 && (nc < 0 || onk > nk || (onk == nk && onc < nc));
+                    nk = bn ? onk : nk;
+                    nc = bn ? onc : nc;
+                    const uint32_t olk = __shfl_xor_sync(0xffffffffu, lk, o);
+                    const int olc = __shfl_xor_sync(0xffffffffu, lc, o);
+                    const bool bl = olc >= 0 && (lc < 0 || olk < lk || (olk == lk && olc > lc));
+                    lk = bl ? olk : lk;
+                    lc = bl ? olc : lc;
+                }
+                if (open) {
+                    if (m64 < target64 && nc >= 0) {
+                        if ((nc >> 5) == s) m |= 1u << (nc & 31);
+                        m64 = __dadd_rn(m64, (double)__uint_as_float(nk));
+                    } else if (lc >= 0 && __dsub_rn(m64, (double)__uint_as_float(lk)) >= target64) {
+                        if ((lc >> 5) == s) m &= ~(1u << (lc & 31));
+                        m64 = __dsub_rn(m64, (double)__uint_as_float(lk));
+                    } else {
+                        open = false;
+                    }
+                }
+            }
         }
         const int n_keep = quad_sum(__popc(m));
         if (active) tau = gi == 0 ? b.lo : (uint32_t)((int)tau + (((int)b.lo - (int)tau) >> 1));

@@ -188,12 +188,13 @@ SPARK_API int spark_prune_grouped(const void *k, const void *q_obs, int G, int W
  *   p     fraction in [0, 1] (SPARK_ERR_ARG otherwise, NaN included)
  *   out   out->T is the capacity Tcap: the number of value slots per token
  * Per token, channels are ordered by (w desc, channel asc); the kept set is
- * the shortest prefix of that order whose mass reaches fp32(p * total), cut
- * to its first Tcap channels when longer.  The library's arithmetic for the
- * mass of a channel set (the pages leave it open): an fp32 sum, within each
- * block of 32 channels in ascending channel order from +0, then
- * (B0 + B1) + (B2 + B3); "reaches" is >=, so a token whose saliencies are
- * all 0 (or p = 0) keeps nothing.  The mask holds the kept channels (at most
+ * the shortest prefix of that order whose cumulative saliency reaches
+ * p * total, cut to its first Tcap channels when longer.  The library's
+ * arithmetic (the pages leave it open): the cumulative saliency and the
+ * total are sums of the fp32 saliencies taken in fp64 and p * total is an
+ * fp64 product, so the boundary is the exact one up to fp64 rounding
+ * (2^-46 relative); "reaches" is >=, so a token whose saliencies are all 0
+ * (or p = 0) keeps nothing.  The mask holds the kept channels (at most
  * Tcap bits); the kept values fill the first slots of the token's Tcap slots
  * in ascending channel order (layout of spark_kcache with T = Tcap), the
  * other slots are 0.  stats: N = number of pruned entries (data-dependent),
