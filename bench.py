@@ -403,6 +403,11 @@ def run_gpu(args):
               "snapkv": "CUDA events around spark_snapkv_evict on its stream: both score passes, the "
                         "select and the gather (the bytes are those of the whole entry point)"}[dom]
 
+    # decode alone, called back to back for ~0.6 s (sustained load: the
+    # power cap may engage, unlike inside the step where decode alternates
+    # with the ALU-bound prune)
+    sustained = run_decode_sustained(job, wl, stream, bm["decode"], peak, peak_kind) if rank == 0 else None
+
     variants = None
     if not args.no_variants:
         variants = run_variants(job, wl, stream, peak, peak_kind)
@@ -417,7 +422,16 @@ def run_gpu(args):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": UNIT,
+            # the metric's own quantities, per step of the same timed region:
+            # the decode-attention call alone and the prune call alone
+            "decode_token_heads_per_s": world * token_heads / (decode_ms / 1e3),
+            "decode_us": decode_ms * 1e3, "decode_gbs": decode_gbs,
+            "decode_frac_8tbs": decode_gbs / NOMINAL_HBM_GBS, f"decode_frac_{peak_kind}": decode_gbs / peak,
+            "prune_gbs": prune_gbs, f"prune_frac_{peak_kind}": prune_gbs / peak,
+            "value_is": "whole-step throughput: prompt token-heads (+ the tail token) per second of prune + "
+                        "tail append + decode",
+            "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
             "data": "synthetic (seeded N(0,1) x per-channel LogNormal(0,1) outlier scales)",
@@ -440,16 +454,59 @@ def run_gpu(args):
             "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "limiter": limiter,
+                         "traffic_source": ("committed ncu capture of the same kernel source "
+                                            "(profiles/traffic.json), not measured in this run") if rec else None,
                          "bytes_per_launch": bm[dom], "entry": {"prune": "spark_prune",
                                                                 "decode": "spark_decode_attn",
                                                                 "snapkv": "spark_snapkv_evict"}[dom],
                          "timing": timing},
+            "decode_sustained": sustained,
             "variants": variants,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": job.launches_per_step * args.steps,
         }
         print(json.dumps(line), flush=True)
     sd.finalize()
+
+
+def run_decode_sustained(job, wl, stream, nbytes, peak, peak_kind, seconds=0.6):
+    """spark_decode_attn alone, back to back for about `seconds` of device
+    time on the launching stream (after the timed step loop), with the clocks
+    sampled meanwhile: the decode figure under sustained load."""
+    sp = job.sp
+
+    def call():
+        sp.spark_decode_attn(job.q, job.kc, job.v_ev if wl.keep else job.v, job.kt, job.vt, job.cap, 1, wl.G,
+                             job.out, job.wsd, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    n = max(10, int(seconds * 1e3 / max(e0.elapsed_time(e1), 1e-3)))
+    sampler = ClockSampler(job.dev.index)
+    sampler.start()
+    time.sleep(0.2)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n):
+            call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if sp.spark_device_status(job.wsd) != 0:
+        raise RuntimeError("device status after the sustained decode calls")
+    us = e0.elapsed_time(e1) / n * 1e3
+    gbs = nbytes / (us / 1e6) / 1e9
+    return {"calls": n, "us_per_call": us, "gbs": gbs, "frac_8tbs": gbs / NOMINAL_HBM_GBS,
+            f"frac_{peak_kind}": gbs / peak, "clocks": clocks,
+            "timing": "CUDA events around n back-to-back spark_decode_attn calls on the launching stream"}
 
 
 def run_variants(job, wl, stream, peak, peak_kind, iters=5):
