@@ -561,7 +561,7 @@ def run_variants(job, wl, stream, peak, peak_kind, iters=5):
     del kt_, wst, wsd_t
     # SparK-p at the pages' p = 0.99, full capacity (no cut): prune + decode
     Tcap = wl.D
-    kp_ = sp.KCache.empty(wl.rows, wl.Hkv, S, wl.D, Tcap, wl.torch_dtype, device=job.dev)
+    kp_ = sp.KCache.empty_topp(wl.rows, wl.Hkv, S, wl.D, Tcap, wl.torch_dtype, device=job.dev)
     wsp_p = sp.workspace(sp.spark_workspace_bytes(sp.SPARK_OP_TOPP, wl.rows, wl.Hkv, wl.G, S, wl.D, Tcap, 0),
                          job.dev)
     us_pp = timed(lambda: sp.spark_prune_topp(k, job.q_obs, wl.G, wl.W, 0.99, kp_, wsp_p, stream))
@@ -574,9 +574,13 @@ def run_variants(job, wl, stream, peak, peak_kind, iters=5):
                                                     stream=stream))
     if sp.spark_device_status(wsd_p) != 0:
         raise RuntimeError("device status after the SparK-p decode")
-    nb_pp = wl.BH * S * (wl.D * es + 16 + Tcap * es)
-    nb_pd = wl.BH * S * (16 + Tcap * es + wl.D * es)
+    # the compact value stream: each 32-token group holds its longest kept set
+    used = sp.spark_topp_vals_used(kp_, stream)
+    ng = (S + 31) // 32
+    nb_pp = wl.BH * S * (2 * wl.D * es + 16) + used + (wl.BH * ng + 1) * 4  # K read twice
+    nb_pd = wl.BH * S * (16 + wl.D * es) + used + (wl.BH * ng + 1) * 4
     out["spark_p"] = {"p": 0.99, "Tcap": Tcap, "mean_kept": mean_kept, "mean_prune_rate": 1 - mean_kept / wl.D,
+                      "vals_bytes": used, "vals_bytes_per_token_head": used / max(wl.BH * S, 1),
                       "prune_us": us_pp, "prune_bytes": nb_pp, "prune_gbs": nb_pp / (us_pp / 1e6) / 1e9,
                       "decode_us": us_pd, "decode_bytes": nb_pd, "decode_gbs": nb_pd / (us_pd / 1e6) / 1e9,
                       "timing": "CUDA events on the stream, outside the step; no tail"}

@@ -33,7 +33,7 @@ SPARK_OP_TOPP = 4
 
 EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark_workspace_bytes",
            "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_group_budget", "spark_prune_values", "spark_prune_think", "spark_prune_topp", "spark_decode_attn",
-           "spark_decode_attn_topp",
+           "spark_decode_attn_topp", "spark_topp_offsets_bytes", "spark_topp_vals_used",
            "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_selftest_wait_timeout", "spark_tail_append", "spark_device_status",
            "spark_status_str", "spark_snapkv_evict")
 
@@ -47,7 +47,8 @@ class SparkError(RuntimeError):
 class spark_kcache(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("S", ctypes.c_int), ("D", ctypes.c_int),
                 ("T", ctypes.c_int), ("dtype", ctypes.c_int), ("mask", ctypes.c_void_p),
-                ("vals", ctypes.c_void_p), ("qn", ctypes.c_void_p), ("stats", ctypes.c_void_p)]
+                ("vals", ctypes.c_void_p), ("qn", ctypes.c_void_p), ("stats", ctypes.c_void_p),
+                ("goff", ctypes.c_void_p)]
 
 
 _lib = None
@@ -87,6 +88,10 @@ def lib():
         L.spark_decode_attn_topp.argtypes = [P, ctypes.POINTER(spark_kcache), P, P, P, I, I, I, I,
                                              ctypes.c_ulonglong, P, P, Z, P]
         L.spark_decode_attn_topp.restype = I
+        L.spark_topp_offsets_bytes.argtypes = [I, I, I]
+        L.spark_topp_offsets_bytes.restype = Z
+        L.spark_topp_vals_used.argtypes = [ctypes.POINTER(spark_kcache), ctypes.POINTER(Z), P]
+        L.spark_topp_vals_used.restype = I
         L.spark_selftest_wait_timeout.argtypes = [P, I, P]
         L.spark_selftest_wait_timeout.restype = I
         L.spark_decode_attn_kv.argtypes = [P, ctypes.POINTER(spark_kcache), ctypes.POINTER(spark_kcache), P, P, I,
@@ -171,6 +176,7 @@ class KCache:
     vals: torch.Tensor    # [B, Hkv, S32 * T] interleaved by 32-token groups
     qn: torch.Tensor      # fp32 [B, Hkv, D]
     stats: torch.Tensor   # fp64 [B, Hkv, 4]
+    goff: torch.Tensor = None  # SparK-p only: int32 [B * Hkv * S32 / 32 + 1] first value row per group
 
     @staticmethod
     def empty(B, Hkv, S, D, T, dtype, device="cuda") -> "KCache":
@@ -181,9 +187,19 @@ class KCache:
                       torch.empty((B, Hkv, D), dtype=torch.float32, device=device),
                       torch.empty((B, Hkv, 4), dtype=torch.float64, device=device))
 
+    @staticmethod
+    def empty_topp(B, Hkv, S, D, Tcap, dtype, device="cuda") -> "KCache":
+        """A SparK-p cache: masks, a value stream with room for Tcap slots per
+        token (the most spark_prune_topp can write) and the group offsets."""
+        kc = KCache.empty(B, Hkv, S, D, Tcap, dtype, device)
+        kc.vals = kc.vals.reshape(-1)
+        kc.goff = torch.empty((B * Hkv * ((S + 31) // 32) + 1,), dtype=torch.int32, device=device)
+        return kc
+
     def struct(self) -> spark_kcache:
         return spark_kcache(self.B, self.Hkv, self.S, self.D, self.T, _dtype_code(self.dtype),
-                            _ptr(self.mask), _ptr(self.vals), _ptr(self.qn), _ptr(self.stats))
+                            _ptr(self.mask), _ptr(self.vals), _ptr(self.qn), _ptr(self.stats),
+                            _ptr(self.goff) if self.goff is not None else None)
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in (self.mask, self.vals, self.qn, self.stats))
@@ -241,6 +257,18 @@ def spark_prune_topp(k: torch.Tensor, q_obs: torch.Tensor, G: int, W: int, p: fl
     rc = lib().spark_prune_topp(_ptr(k), _ptr(q_obs), G, W, ctypes.c_float(p), ctypes.byref(s), _ptr(ws),
                                 ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_prune_topp")
+
+
+def spark_topp_offsets_bytes(B: int, Hkv: int, S: int) -> int:
+    return int(lib().spark_topp_offsets_bytes(B, Hkv, S))
+
+
+def spark_topp_vals_used(kc: KCache, stream=None) -> int:
+    """Bytes of kc.vals the last spark_prune_topp used (synchronises the stream)."""
+    s = kc.struct()
+    n = ctypes.c_size_t(0)
+    _check(lib().spark_topp_vals_used(ctypes.byref(s), ctypes.byref(n), _stream(stream)), "spark_topp_vals_used")
+    return int(n.value)
 
 
 def spark_decode_attn_topp(q: torch.Tensor, kc: KCache, v: torch.Tensor, k_tail, v_tail, tail_cap: int,

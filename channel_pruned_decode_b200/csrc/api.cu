@@ -12,7 +12,8 @@ cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W,
                                  const int *group_T, const spark_kcache &kc, void *ws, cudaStream_t st);
 cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const spark_kcache *vc,
                           const void *k_tail, const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
-                          unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st);
+                          unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st,
+                          bool topp = false);
 cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws, cudaStream_t st);
 cudaError_t launch_prune_topp(const void *k, const void *q_obs, int G, int W, float p, const spark_kcache &kc,
                               void *ws, cudaStream_t st);
@@ -174,6 +175,9 @@ int spark_prune_topp(const void *k, const void *q_obs, int G, int W, float p, co
     if (!(p >= 0.0f && p <= 1.0f)) return SPARK_ERR_ARG;
     const long BH = (long)out->B * out->Hkv;
     if (BH == 0) return SPARK_OK;
+    if (!out->goff || (reinterpret_cast<uintptr_t>(out->goff) & 3u)) return SPARK_ERR_ARG;
+    // value rows are counted in 32 bits
+    if ((double)BH * (double)((out->S + 31) / 32) * (double)out->T >= 4294967295.0) return SPARK_ERR_UNSUPPORTED;
     if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
     if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
     if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
@@ -182,13 +186,34 @@ int spark_prune_topp(const void *k, const void *q_obs, int G, int W, float p, co
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 
+size_t spark_topp_offsets_bytes(int B, int Hkv, int S) {
+    if (B < 0 || Hkv < 0 || S < 0) return 0;
+    return ((size_t)B * Hkv * (((size_t)S + 31) / 32) + 1) * sizeof(uint32_t);
+}
+
+int spark_topp_vals_used(const spark_kcache *kc, size_t *bytes, void *stream) {
+    if (!kc || !bytes || !kc->goff || kc->B < 0 || kc->Hkv < 0 || kc->S < 0) return SPARK_ERR_ARG;
+    const int es = elem_size(kc->dtype);
+    if (es == 0) return SPARK_ERR_ARG;
+    const size_t n = (size_t)kc->B * kc->Hkv * (((size_t)kc->S + 31) / 32);
+    uint32_t rows = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&rows, kc->goff + n, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return SPARK_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SPARK_ERR_CUDA;
+    *bytes = (size_t)rows * 32 * (size_t)es;
+    return SPARK_OK;
+}
+
 // argument checks and launch shared by spark_decode_attn and
 // spark_decode_attn_topp; `f` is the kernel's recovery selector
 static int decode_entry(const void *q, const spark_kcache *kc, const void *v, const void *k_tail,
                         const void *v_tail, int tail_cap, int n_tail, int G, int recovery, int f,
-                        unsigned long long seed, float *out, void *workspace, size_t ws_bytes, void *stream) {
+                        unsigned long long seed, float *out, void *workspace, size_t ws_bytes, void *stream,
+                        bool topp = false) {
     int rc = check_cache(kc);
     if (rc != SPARK_OK) return rc;
+    if (topp && (!kc->goff || (reinterpret_cast<uintptr_t>(kc->goff) & 3u))) return SPARK_ERR_ARG;
     if (G != 1 && G != 2 && G != 4 && G != 8) return G < 1 ? SPARK_ERR_ARG : SPARK_ERR_UNSUPPORTED;
     if (recovery != SPARK_F_DEGENERATE && recovery != SPARK_F_GAUSSIAN && recovery != SPARK_F_EXPONENTIAL)
         return SPARK_ERR_ARG;
@@ -205,7 +230,7 @@ static int decode_entry(const void *q, const spark_kcache *kc, const void *v, co
     if (BH * (long)geo.units >= (1L << 31)) return SPARK_ERR_UNSUPPORTED;  // 32-bit item indices
     if (ws_bytes < decode_workspace(BH, geo, G)) return SPARK_ERR_WORKSPACE;
     cudaError_t e = launch_decode(q, *kc, v, nullptr, k_tail, v_tail, tail_cap, n_tail, G, f, seed, out,
-                                  workspace, geo, static_cast<cudaStream_t>(stream));
+                                  workspace, geo, static_cast<cudaStream_t>(stream), topp);
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 
@@ -225,7 +250,7 @@ int spark_decode_attn_topp(const void *q, const spark_kcache *kc, const void *v,
     // order, which already handles fewer kept channels than slots
     const int f = recovery == SPARK_F_DEGENERATE ? kRecoveryDegVar : recovery;
     return decode_entry(q, kc, v, k_tail, v_tail, tail_cap, n_tail, G, recovery, f, seed, out, workspace,
-                        ws_bytes, stream);
+                        ws_bytes, stream, true);
 }
 
 size_t spark_workspace_bytes_kv(int B, int Hkv, int G, int S, int D, int T, int Tv, int n_tail) {

@@ -56,6 +56,7 @@ struct DecArgs {
     const void *q;
     const uint32_t *mask;
     const void *vals;
+    const uint32_t *goff;   // SparK-p cache: first value row of each group (else NULL)
     const uint32_t *vmask;  // pruned value cache (packed-V kernels only)
     const void *vvals;
     int Tv;
@@ -612,13 +613,22 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         const long t1 = min((long)a.S, (long)u * a.chunk + a.chunk);
         const int n = (int)min((long)kWT, t1 - t0);
         const uint32_t mb = (uint32_t)n * 16u;
-        const uint32_t vb = (uint32_t)kWT * (uint32_t)a.T * (uint32_t)es;  // one whole 32-token group
+        // one whole 32-token group of kept values: T slots, or for a SparK-p
+        // cache the group's own slot count, found through goff
+        uint32_t vb = (uint32_t)kWT * (uint32_t)a.T * (uint32_t)es;
+        const E *vsrc = gvals + (size_t)bh * a.S32 * a.T + (size_t)t0 * a.T;
+        if (a.goff) {
+            const long gi = bh * (a.S32 / kWT) + t0 / kWT;
+            const uint32_t r0 = a.goff[gi], r1 = a.goff[gi + 1];
+            vb = (r1 - r0) * (uint32_t)kWT * (uint32_t)es;
+            vsrc = gvals + (size_t)r0 * kWT;
+        }
         const uint32_t bar = smem_u32(ws.bars + st);
         unsigned char *dst = ws.stages + (size_t)st * ws.stage_bytes;
         const uint32_t vvb = kPV ? (uint32_t)kWT * (uint32_t)a.Tv * (uint32_t)es : 0u;
         mbar_expect_tx(bar, mb + vb + (kPV ? mb + vvb : 0u));
         bulk_g2s(smem_u32(dst), a.mask + ((size_t)bh * a.S + t0) * kMaskWords, mb, bar);
-        if (vb) bulk_g2s(smem_u32(dst + kWT * 16), gvals + (size_t)bh * a.S32 * a.T + (size_t)t0 * a.T, vb, bar);
+        if (vb) bulk_g2s(smem_u32(dst + kWT * 16), vsrc, vb, bar);
         if constexpr (kPV) {
             bulk_g2s(smem_u32(dst + ws.vstage_off), a.vmask + ((size_t)bh * a.S + t0) * kMaskWords, mb, bar);
             if (vvb)
@@ -1121,13 +1131,15 @@ static cudaError_t dispatch_f(const DecArgs &a, const DecodeGeom &geo, int G, in
 
 cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, const spark_kcache *vc,
                           const void *k_tail, const void *v_tail, int tail_cap, int n_tail, int G, int recovery,
-                          unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st) {
+                          unsigned long long seed, float *out, void *ws, const DecodeGeom &geo, cudaStream_t st,
+                          bool topp) {
     const long BH = (long)kc.B * kc.Hkv;
     if (BH == 0) return cudaSuccess;
     DecArgs a{};
     a.q = q;
     a.mask = kc.mask;
     a.vals = kc.vals;
+    a.goff = topp ? kc.goff : nullptr;
     a.qn = kc.qn;
     a.stats = kc.stats;
     a.v = v;

@@ -775,10 +775,8 @@ __device__ __forceinline__ void topp_full_range(TopPBracket &b) {
 template <typename E>
 __global__ void __launch_bounds__(kPruneThreads, 3)
     prune_topp_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
-                      E *__restrict__ vals, double *__restrict__ partial, int S, int Tcap, int n_chunks, int gpc,
-                      float p) {
-    using Raw = typename RawT<E>::type;
-    __shared__ __align__(16) Raw vtile[kPruneThreads / 32][kD * 8];
+                      uint32_t *__restrict__ tg, double *__restrict__ partial, int S, int Tcap, int n_chunks,
+                      int gpc, float p) {
     __shared__ double red[3][kPruneThreads / 32];
     __shared__ uint32_t qmax[kPruneThreads / 32];
     __shared__ __align__(16) float qs[4 * 36];
@@ -812,12 +810,11 @@ __global__ void __launch_bounds__(kPruneThreads, 3)
     }
     const float2 scale2 = make_float2(scale, scale);
 
-    Raw *vt = vtile[warp];
     uint32_t tau = 0u;  // running estimate of the quad's mass level
     double acc_w = 0.0, acc_w2 = 0.0, acc_n = 0.0;
     const long g_first = (long)chunk * gpc;
+    const long ng = S32 / 32;
     const E *krow = k + ((size_t)bh * S + g_first * 32 + tl) * kD + 32 * s;
-    E *gvals = vals + (size_t)bh * S32 * Tcap + (size_t)g_first * 32 * Tcap;
 
     auto group = [&](int gi, KSlice<E> &cur, KSlice<E> &nxt) {
         const long t = (g_first + gi) * 32 + tl;
@@ -992,21 +989,17 @@ __global__ void __launch_bounds__(kPruneThreads, 3)
         }
         if (valid) mask[((size_t)bh * S + t) * kMaskWords + s] = m;
 
-        // zero the warp's Tcap staging rows, then stage the kept values
-        {
-            constexpr int kRowB = 8 * (int)sizeof(Raw);  // bytes of one staging row
-            uint4 *z = reinterpret_cast<uint4 *>(vt);
-            for (int c = lane; c < Tcap * kRowB / 16; c += 32) z[c] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        __syncwarp();
-        Raw *dst = vt + quad_excl_scan(__popc(m), s) * 8 + tq;
+        // the group's slot count: the largest kept count of its tokens (the
+        // four warps of the CTA each bring their 8 tokens)
+        const int kept = quad_sum(__popc(m));  // every lane shuffles; m = 0 on padding tokens
+        const int wmax = __reduce_max_sync(0xffffffffu, kept);
+        if (lane == 0 && wmax > 0) atomicMax(tg + (size_t)bh * ng + g_first + gi, (unsigned)wmax);
+
+        // pruned-saliency sums: fp32 over this lane's 32 channels
         float sw = 0.f, sw2 = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            if ((m >> i) & 1u) {
-                *dst = (Raw)cur.raw(i);
-                dst += 8;
-            } else {
+            if (!((m >> i) & 1u)) {
                 const float w = __uint_as_float(key[i]);
                 sw = __fadd_rn(sw, w);
                 sw2 = __fmaf_rn(w, w, sw2);
@@ -1017,16 +1010,6 @@ __global__ void __launch_bounds__(kPruneThreads, 3)
             acc_w2 = __dadd_rn(acc_w2, (double)sw2);
             acc_n = __dadd_rn(acc_n, (double)(32 - __popc(m)));
         }
-        __syncwarp();
-        constexpr int kParts = (int)sizeof(E) / 2;
-        unsigned char *g = reinterpret_cast<unsigned char *>(gvals + (size_t)gi * 32 * Tcap + warp * 8);
-        const unsigned char *src = reinterpret_cast<const unsigned char *>(vt);
-        for (int c = lane; c < Tcap * kParts; c += 32) {
-            const int row = c / kParts, part = c % kParts;
-            __stcs(reinterpret_cast<uint4 *>(g + (size_t)row * 32 * sizeof(E) + part * 16),
-                   *reinterpret_cast<const uint4 *>(src + row * 8 * sizeof(E) + part * 16));
-        }
-        __syncwarp();
     };
 
     KSlice<E> ka, kb;
@@ -1091,20 +1074,193 @@ __global__ void stats_topp_kernel(const double *__restrict__ partial, int n_chun
     }
 }
 
+// ---- SparK-p value layout.  The selection kernel leaves tg[i] = the largest
+// kept count of group i (zeroed before it runs).  Three small launches turn
+// the counts into group offsets in rows of 32 elements -- per-head totals, a
+// scan of the head totals, per-head scans plus the head bases -- integer
+// sums, so the offsets are the same on every run.  topp_gather_kernel then
+// reads the key rows a second time and writes each group's kept values.
+constexpr int kScanThreads = 1024;
+
+// exclusive prefix of v over the CTA (kScanThreads threads); *tot = the sum
+__device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, uint32_t *sh, uint32_t &tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) sh[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = sh[lane];  // kScanThreads / 32 == 32 warp totals
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        sh[32 + lane] = w;
+    }
+    __syncthreads();
+    tot = sh[63];
+    const uint32_t r = (warp > 0 ? sh[32 + warp - 1] : 0u) + x - v;
+    __syncthreads();  // sh is reused by the caller's next round
+    return r;
+}
+
+// rows of each head: the sum of its groups' slot counts
+__global__ void __launch_bounds__(kScanThreads) topp_head_rows_kernel(const uint32_t *__restrict__ tg, long ng,
+                                                                      uint32_t *__restrict__ hrows) {
+    __shared__ uint32_t sh[64];
+    const long bh = blockIdx.x;
+    uint32_t acc = 0u;
+    for (long g = threadIdx.x; g < ng; g += kScanThreads) acc += tg[bh * ng + g];
+    uint32_t tot;
+    (void)cta_excl_scan(acc, sh, tot);
+    if (threadIdx.x == 0) hrows[bh] = tot;
+}
+
+// first row of each head (exclusive scan of the head totals, one CTA), and
+// the total rows into the last entry of goff
+__global__ void __launch_bounds__(kScanThreads) topp_head_base_kernel(const uint32_t *__restrict__ hrows, long BH,
+                                                                      uint32_t *__restrict__ hbase,
+                                                                      uint32_t *__restrict__ goff_end) {
+    __shared__ uint32_t sh[64];
+    uint32_t carry = 0u;
+    for (long b0 = 0; b0 < BH; b0 += kScanThreads) {
+        const long bh = b0 + threadIdx.x;
+        const uint32_t v = bh < BH ? hrows[bh] : 0u;
+        uint32_t tot;
+        const uint32_t ex = cta_excl_scan(v, sh, tot);
+        if (bh < BH) hbase[bh] = carry + ex;
+        carry += tot;
+    }
+    if (threadIdx.x == 0) *goff_end = carry;
+}
+
+// goff of each group: its head's base plus the exclusive scan of the head's
+// slot counts
+__global__ void __launch_bounds__(kScanThreads) topp_goff_kernel(const uint32_t *__restrict__ tg, long ng,
+                                                                 const uint32_t *__restrict__ hbase,
+                                                                 uint32_t *__restrict__ goff) {
+    __shared__ uint32_t sh[64];
+    const long bh = blockIdx.x;
+    uint32_t carry = hbase[bh];
+    for (long g0 = 0; g0 < ng; g0 += kScanThreads) {
+        const long g = g0 + threadIdx.x;
+        const uint32_t v = g < ng ? tg[bh * ng + g] : 0u;
+        uint32_t tot;
+        const uint32_t ex = cta_excl_scan(v, sh, tot);
+        if (g < ng) goff[bh * ng + g] = carry + ex;
+        carry += tot;
+    }
+}
+
+// Kept values of the SparK-p cache: one warp per 32-token group.  The
+// group's key rows arrive by one bulk copy; then lane = token, and every
+// lane runs the group's T_g slots from the top (the same slot j for the
+// whole warp, so each slot of the 32 tokens is one coalesced store): slot j
+// takes the token's j-th kept channel in ascending order -- found by walking
+// the mask bits from the top channel down -- or 0 past the token's count.
+constexpr int kGatherWarps = 4;
+
+template <typename E>
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    topp_gather_kernel(const E *__restrict__ k, const uint32_t *__restrict__ mask, const uint32_t *__restrict__ goff,
+                       E *__restrict__ vals, uint32_t *__restrict__ status, int S, long ng, long n_groups) {
+    using Raw = typename RawT<E>::type;
+    constexpr int kRowB = kD * (int)sizeof(E);
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ uint64_t bars[kGatherWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long idx = (long)blockIdx.x * kGatherWarps + warp;
+    if (idx >= n_groups) return;
+    const long bh = idx / ng, g = idx % ng;
+    const long t0 = g * 32;
+    const int rows = (int)min(32L, (long)S - t0);
+    unsigned char *tile = smem_raw + (size_t)warp * 32 * kRowB;
+    const uint32_t bar = smem_u32(&bars[warp]);
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_expect_tx(bar, (uint32_t)rows * (uint32_t)kRowB);
+        bulk_g2s(smem_u32(tile), k + ((size_t)bh * S + t0) * kD, (uint32_t)rows * (uint32_t)kRowB, bar);
+    }
+    __syncwarp();
+    const bool valid = lane < rows;
+    uint4 mw = make_uint4(0u, 0u, 0u, 0u);
+    if (valid) mw = *reinterpret_cast<const uint4 *>(mask + ((size_t)bh * S + t0 + lane) * kMaskWords);
+    const int n = __popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w);
+    const uint32_t r0 = goff[idx];
+    const int Tg = (int)(goff[idx + 1] - r0);
+    const bool ok = mbar_wait_bounded(bar, 0u);
+    if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) {
+            atomicOr(status, kDevTimeout);
+            (void)mbar_wait_bounded(bar, 0u);  // let the copy in flight land before the warp exits
+        }
+        __syncwarp();
+        return;
+    }
+    // the non-empty mask words, top first
+    uint32_t q0 = mw.w, q1 = mw.z, q2 = mw.y, q3 = mw.x;
+    int b0 = 96, b1 = 64, b2 = 32, b3 = 0;
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+        if (q2 == 0u) { q2 = q3; b2 = b3; q3 = 0u; }
+        if (q1 == 0u) { q1 = q2; b1 = b2; q2 = q3; b2 = b3; q3 = 0u; }
+        if (q0 == 0u) { q0 = q1; b0 = b1; q1 = q2; b1 = b2; q2 = q3; b2 = b3; q3 = 0u; }
+    }
+    const Raw *row = reinterpret_cast<const Raw *>(tile + lane * kRowB);
+    Raw *out = reinterpret_cast<Raw *>(vals) + (size_t)r0 * 32 + lane;
+    for (int j = Tg - 1; j >= 0; --j) {
+        Raw v = (Raw)0;
+        if (j < n) {
+            uint32_t b;
+            asm("bfind.u32 %0, %1;" : "=r"(b) : "r"(q0));
+            v = row[(b0 + (int)b) & (kD - 1)];
+            q0 &= ~(1u << b);
+            if (q0 == 0u) { q0 = q1; b0 = b1; q1 = q2; b1 = b2; q2 = q3; b2 = b3; }
+        }
+        out[(size_t)j * 32] = v;
+    }
+}
+
 template <typename E>
 static cudaError_t launch_prune_topp_t(const void *k, const void *q_obs, int G, int W, float p,
                                        const spark_kcache &kc, void *ws, cudaStream_t st) {
     const long BH = (long)kc.B * kc.Hkv;
     if (BH == 0) return cudaSuccess;
-    double *partial = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
+    const long ng = ((long)kc.S + 31) / 32;
+    const ToppWs tw = topp_ws_layout(ws, BH, kc.S);
     qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn);
     const int gpc = prune_groups_per_cta(BH, kc.S);
     const int nch = prune_chunks(kc.S, gpc);
-    if (nch > 0)
+    if (ng > 0) {
+        cudaError_t e = cudaMemsetAsync(tw.tg, 0, (size_t)BH * ng * sizeof(uint32_t), st);
+        if (e != cudaSuccess) return e;
         prune_topp_kernel<E><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
-            static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T, nch, gpc,
-            p);
-    stats_topp_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.stats);
+            static_cast<const E *>(k), kc.qn, kc.mask, tw.tg, tw.partial, kc.S, kc.T, nch, gpc, p);
+    }
+    stats_topp_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(tw.partial, nch, BH, kc.stats);
+    // group offsets (the last entry, the total, also when there are no groups)
+    if (ng > 0) topp_head_rows_kernel<<<(unsigned)BH, kScanThreads, 0, st>>>(tw.tg, ng, tw.hrows);
+    else {
+        cudaError_t e = cudaMemsetAsync(tw.hrows, 0, (size_t)BH * sizeof(uint32_t), st);
+        if (e != cudaSuccess) return e;
+    }
+    topp_head_base_kernel<<<1, kScanThreads, 0, st>>>(tw.hrows, BH, tw.hbase, kc.goff + BH * ng);
+    if (ng > 0) {
+        topp_goff_kernel<<<(unsigned)BH, kScanThreads, 0, st>>>(tw.tg, ng, tw.hbase, kc.goff);
+        const int smem = kGatherWarps * 32 * kD * (int)sizeof(E);
+        cudaError_t e = cudaFuncSetAttribute(topp_gather_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        const long n_groups = BH * ng;
+        topp_gather_kernel<E><<<(unsigned)((n_groups + kGatherWarps - 1) / kGatherWarps), kGatherWarps * 32, smem, st>>>(
+            static_cast<const E *>(k), kc.mask, kc.goff, static_cast<E *>(kc.vals), static_cast<uint32_t *>(ws),
+            kc.S, ng, n_groups);
+    }
     return cudaGetLastError();
 }
 

@@ -76,9 +76,38 @@ inline size_t prune_workspace(long BH, int S) {
     return kWsHeader + (size_t)BH * (size_t)prune_chunks(S) * 2 * sizeof(double);
 }
 
-// SparK-p: a third partial per chunk (the data-dependent pruned count)
+// SparK-p workspace: the prune partials with a third one per chunk (the
+// data-dependent pruned count), then per group the largest kept count, then
+// per head its rows and its first row (the value layout's scan)
+struct ToppWs {
+    double *partial;
+    uint32_t *tg;
+    uint32_t *hrows;
+    uint32_t *hbase;
+};
+
+inline size_t topp_partials_bytes(long BH, int S) {
+    return ((size_t)BH * (size_t)prune_chunks(S) * 3 * sizeof(double) + 255) / 256 * 256;
+}
+
+inline size_t topp_groups(long BH, int S) { return (size_t)BH * (((size_t)S + 31) / 32); }
+
 inline size_t topp_workspace(long BH, int S) {
-    return kWsHeader + (size_t)BH * (size_t)prune_chunks(S) * 3 * sizeof(double);
+    return kWsHeader + topp_partials_bytes(BH, S) + (topp_groups(BH, S) * 4 + 255) / 256 * 256 +
+           2 * (((size_t)BH * 4 + 255) / 256 * 256);
+}
+
+inline ToppWs topp_ws_layout(void *ws, long BH, int S) {
+    char *p = static_cast<char *>(ws) + kWsHeader;
+    ToppWs t;
+    t.partial = reinterpret_cast<double *>(p);
+    p += topp_partials_bytes(BH, S);
+    t.tg = reinterpret_cast<uint32_t *>(p);
+    p += (topp_groups(BH, S) * 4 + 255) / 256 * 256;
+    t.hrows = reinterpret_cast<uint32_t *>(p);
+    p += ((size_t)BH * 4 + 255) / 256 * 256;
+    t.hbase = reinterpret_cast<uint32_t *>(p);
+    return t;
 }
 
 // ---------------------------------------------------------------- decode

@@ -18,8 +18,8 @@
  * Conventions shared by every entry point
  *   - All tensor arguments are DEVICE pointers owned by the caller; the
  *     library never allocates, frees or prints, and no entry point
- *     synchronises except spark_device_status, which waits for `stream` so
- *     that it can read the status word.  Every launch is asynchronous on
+ *     synchronises except spark_device_status and spark_topp_vals_used,
+ *     which wait for `stream` so that they can read a device word.  Every launch is asynchronous on
  *     `stream` (a cudaStream_t; NULL = legacy default).
  *   - Tensors are dense row-major; pointers must be 16-byte aligned.
  *   - dtype: SPARK_F32 (fp32) or SPARK_BF16 (bf16) for keys, values and
@@ -87,6 +87,17 @@ typedef enum {
  *   qn    fp32 [B][Hkv][D]: window-query channel norm (see spark_prune).
  *   stats fp64 [B][Hkv][4]: {N_pruned, sum w, sum w^2, mu_pruned} over the
  *         pruned (token, channel) entries of that head; mu = 0 when N = 0.
+ *   goff  NULL for every cache above.  A SparK-p cache (spark_prune_topp)
+ *         stores its kept values compactly instead, in rows of 32 elements
+ *         (one slot of the 32 tokens of a group): goff is uint32
+ *         [B*Hkv*G32 + 1] (G32 = S32 / 32 groups per head), goff[i] the
+ *         first row of group i = (b*Hkv + h)*G32 + g, and goff[B*Hkv*G32]
+ *         the number of rows used.  Group i holds T_i = goff[i+1] - goff[i]
+ *         slots per token, interleaved as above: kept value j (ascending
+ *         channel order) of token t of the group at
+ *         vals[(goff[i] + j)*32 + t % 32]; T_i is the largest kept count of
+ *         the group's tokens, and the slots past a token's own count (and
+ *         all slots of padding tokens) hold 0.
  */
 typedef struct spark_kcache {
     int B, Hkv, S, D, T, dtype;
@@ -94,6 +105,7 @@ typedef struct spark_kcache {
     void *vals;
     float *qn;
     double *stats;
+    uint32_t *goff;
 } spark_kcache;
 
 /* Kept channels for pruning ratio lambda ([A] Table 1 caption, [W] 4.1):
@@ -186,7 +198,12 @@ SPARK_API int spark_prune_grouped(const void *k, const void *q_obs, int G, int W
  * channels whose cumulative saliency reaches p -- 99 % in [W] -- of its
  * total).  Same arguments, saliencies w and statistics as spark_prune, plus
  *   p     fraction in [0, 1] (SPARK_ERR_ARG otherwise, NaN included)
- *   out   out->T is the capacity Tcap: the number of value slots per token
+ *   out   out->T is the cap Tcap on the kept channels of a token (1..128);
+ *         out->goff (required, spark_topp_offsets_bytes bytes) receives the
+ *         group offsets and out->vals the compact value stream (see
+ *         spark_kcache), at most B*Hkv*S32*Tcap elements: allocate that
+ *         (spark_cache_sizes' vals size for T = Tcap) or reuse a buffer
+ *         sized from an earlier call's spark_topp_vals_used.
  * Per token, channels are ordered by (w desc, channel asc); the kept set is
  * the shortest prefix of that order whose cumulative saliency reaches
  * p * total, cut to its first Tcap channels when longer.  The library's
@@ -194,22 +211,33 @@ SPARK_API int spark_prune_grouped(const void *k, const void *q_obs, int G, int W
  * total are sums of the fp32 saliencies taken in fp64 and p * total is an
  * fp64 product, so the boundary is the exact one up to fp64 rounding
  * (2^-46 relative); "reaches" is >=, so a token whose saliencies are all 0
- * (or p = 0) keeps nothing.  The mask holds the kept channels (at most
- * Tcap bits); the kept values fill the first slots of the token's Tcap slots
- * in ascending channel order (layout of spark_kcache with T = Tcap), the
- * other slots are 0.  stats: N = number of pruned entries (data-dependent),
- * sum w, sum w^2 over them, mu = sum w / N.  Decode this cache with
+ * (or p = 0) keeps nothing.  The mask holds the kept channels; each 32-token
+ * group stores as many value slots per token as its longest kept set, so
+ * storage and decode traffic follow the data.  stats: N = number of pruned
+ * entries (data-dependent), sum w, sum w^2 over them, mu = sum w / N.  Reads
+ * k twice (the selection, then the kept values).  Decode this cache with
  * spark_decode_attn_topp.  Workspace: spark_workspace_bytes(SPARK_OP_TOPP,
  * ...).
  */
 SPARK_API int spark_prune_topp(const void *k, const void *q_obs, int G, int W, float p,
                                const spark_kcache *out, void *workspace, size_t ws_bytes, void *stream);
 
+/* Bytes of a SparK-p cache's goff array: 4 * (B*Hkv*ceil(S/32) + 1); 0 on
+ * bad arguments. */
+SPARK_API size_t spark_topp_offsets_bytes(int B, int Hkv, int S);
+
+/* Synchronise `stream` and write to *bytes the bytes of kc->vals that the
+ * last spark_prune_topp on this cache used (goff's last entry times 32
+ * times the element size).  Returns SPARK_ERR_ARG on a NULL or non-SparK-p cache and
+ * SPARK_ERR_CUDA if the copy fails.  Besides spark_device_status, the one
+ * entry point that synchronises. */
+SPARK_API int spark_topp_vals_used(const spark_kcache *kc, size_t *bytes, void *stream);
+
 /*
  * Decode attention over a SparK-p cache (spark_prune_topp): exactly
- * spark_decode_attn (same arguments, workspace and results), for a cache
- * whose masks may hold fewer bits than its T value slots, the kept values
- * first.  Degenerate F adds no term for the empty slots.
+ * spark_decode_attn (same arguments, workspace and results), reading each
+ * 32-token group's kept values through kc->goff (required); kc->T is the
+ * cap Tcap.  A token may keep fewer channels than its group's slots.
  */
 SPARK_API int spark_decode_attn_topp(const void *q, const spark_kcache *kc, const void *v,
                                      const void *k_tail, const void *v_tail, int tail_cap,

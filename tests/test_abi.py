@@ -225,7 +225,7 @@ int main(void) {
     if (Tg[0] != 24 || Tg[1] != 16 || Tg[2] != 8 || Tg[3] != 0) return 7;
     /* argument errors come back before anything is launched */
     if (spark_prune(NULL, NULL, 4, 32, NULL, NULL, 0, NULL) != SPARK_ERR_ARG) return 8;
-    spark_kcache kc = {1, 8, 32768, 96, 64, SPARK_BF16, NULL, NULL, NULL, NULL};
+    spark_kcache kc = {1, 8, 32768, 96, 64, SPARK_BF16, NULL, NULL, NULL, NULL, NULL};
     if (spark_prune(NULL, NULL, 4, 32, &kc, NULL, 0, NULL) != SPARK_ERR_UNSUPPORTED) return 9;
     if (spark_status_str(SPARK_ERR_ARG) == NULL) return 10;
     printf("ok %zu\n", total);
@@ -281,7 +281,7 @@ def test_prune_think_rejects_bad_args(L):
 
 
 def test_prune_topp_rejects_bad_args(L):
-    kc = _kc()
+    kc = _kc(goff=16)
 
     def f(p=0.99, k=16, G=4, c=None, ws=256, wsb=1 << 20):
         return L.spark_prune_topp(k, 16, G, 32, ctypes.c_float(p), ctypes.byref(c or kc), ws, wsb, None)
@@ -291,16 +291,31 @@ def test_prune_topp_rejects_bad_args(L):
     assert f(k=None) == B.SPARK_ERR_ARG
     assert f(ws=None) == B.SPARK_ERR_WORKSPACE
     assert f(wsb=64) == B.SPARK_ERR_WORKSPACE
-    assert f(c=_kc(T=129)) == B.SPARK_ERR_ARG
-    assert f(c=_kc(D=64)) == B.SPARK_ERR_UNSUPPORTED
+    assert f(c=_kc(T=129, goff=16)) == B.SPARK_ERR_ARG
+    assert f(c=_kc(D=64, goff=16)) == B.SPARK_ERR_UNSUPPORTED
+    assert f(c=_kc()) == B.SPARK_ERR_ARG                     # no group offsets
+    assert f(c=_kc(goff=18)) == B.SPARK_ERR_ARG              # misaligned offsets
+    # value rows counted in 32 bits: 2^20 heads x 2^11 groups x 128 slots is too many
+    assert f(c=_kc(B=1 << 10, Hkv=1 << 10, S=1 << 16, T=128, goff=16)) == B.SPARK_ERR_UNSUPPORTED
     # three fp64 partials per chunk of 256 tokens (the pruned count is the third)
     assert B.spark_workspace_bytes(B.SPARK_OP_TOPP, 1, 8, 4, 32768, 128, 128, 0) >= 256 + 8 * 128 * 24
     assert B.spark_workspace_bytes(B.SPARK_OP_TOPP, 1, 8, 4, 32768, 128, 128, 0) > \
         B.spark_workspace_bytes(B.SPARK_OP_PRUNE, 1, 8, 4, 32768, 128, 128, 0)
 
 
+def test_topp_offsets_bytes(L):
+    assert B.spark_topp_offsets_bytes(1, 8, 32768) == (8 * 1024 + 1) * 4
+    assert B.spark_topp_offsets_bytes(2, 3, 33) == (2 * 3 * 2 + 1) * 4
+    assert B.spark_topp_offsets_bytes(1, 1, 0) == 4
+    assert B.spark_topp_offsets_bytes(-1, 1, 5) == 0
+    n = ctypes.c_size_t(7)
+    assert L.spark_topp_vals_used(ctypes.byref(_kc()), ctypes.byref(n), None) == B.SPARK_ERR_ARG  # no goff
+    assert L.spark_topp_vals_used(None, ctypes.byref(n), None) == B.SPARK_ERR_ARG
+    assert n.value == 7
+
+
 def test_decode_topp_rejects_bad_args(L):
-    kc = _kc()
+    kc = _kc(goff=16)
     call = lambda **k: L.spark_decode_attn_topp(
         k.get("q", 16), ctypes.byref(kc), k.get("v", 16), k.get("kt", 16), k.get("vt", 16),
         k.get("cap", 8), k.get("n", 0), k.get("G", 4), k.get("rec", 0), 0, k.get("out", 16),
@@ -311,3 +326,5 @@ def test_decode_topp_rejects_bad_args(L):
     assert call(q=None) == B.SPARK_ERR_ARG
     assert call(kt=None) == B.SPARK_ERR_ARG
     assert call(ws=None) == B.SPARK_ERR_WORKSPACE
+    kc.goff = None
+    assert call() == B.SPARK_ERR_ARG  # a SparK-p decode needs the group offsets

@@ -15,10 +15,10 @@ import torch
 
 import oracle
 from channel_pruned_decode_b200 import (KCache, spark_decode_attn, spark_decode_attn_topp, spark_device_status,
-                                        spark_prune_topp, spark_workspace_bytes, workspace, SPARK_F_GAUSSIAN,
-                                        SPARK_OP_DECODE, SPARK_OP_TOPP)
+                                        spark_prune_topp, spark_topp_vals_used, spark_workspace_bytes, workspace,
+                                        SPARK_F_GAUSSIAN, SPARK_OP_DECODE, SPARK_OP_TOPP)
 from channel_pruned_decode_b200.synth import WORKLOADS, make_decode_step, make_prefill, scaled
-from tests._parity import assert_out_close, mask_np, run_prune, to_np, unpack_vals
+from tests._parity import assert_out_close, mask_np, run_prune, to_np
 from tests.test_gpu_parity import STATS_RTOL
 
 pytestmark = pytest.mark.gpu
@@ -28,11 +28,39 @@ DEV = "cuda"
 
 def run_topp(k, q_obs, G, W, p, Tcap):
     R, Hkv, S, _ = k.shape
-    kc = KCache.empty(R, Hkv, S, D, Tcap, k.dtype, device=k.device)
+    kc = KCache.empty_topp(R, Hkv, S, D, Tcap, k.dtype, device=k.device)
     ws = workspace(spark_workspace_bytes(SPARK_OP_TOPP, R, Hkv, G, S, D, Tcap, 0))
     spark_prune_topp(k, q_obs, G, W, p, kc, ws)
     torch.cuda.synchronize()
+    assert spark_device_status(ws) == 0
     return kc
+
+
+def unpack_topp(kc):
+    """The compact SparK-p value stream (group offsets in 32-element rows) as
+    [B*Hkv, S, Tcap] fp32, zero past each token's kept values; also checks
+    the layout: each group's slot count is its longest kept set, unused
+    slots hold 0, and the last offset is the number of rows used."""
+    BH, S, Tcap = kc.B * kc.Hkv, kc.S, kc.T
+    ng = (S + 31) // 32
+    goff = kc.goff.cpu().numpy().view(np.uint32).astype(np.int64)
+    assert goff.shape == (BH * ng + 1,) and goff[0] == 0 and np.all(np.diff(goff) >= 0)
+    vals = kc.vals.reshape(-1)[: int(goff[-1]) * 32].float().cpu().numpy()
+    m = mask_np(kc)
+    cnt = np.zeros((BH, ng * 32), np.int64)
+    if S:
+        cnt[:, :S] = np.unpackbits(np.ascontiguousarray(m).view(np.uint8), axis=-1).sum(-1)
+    out = np.zeros((BH, ng * 32, Tcap), np.float32)
+    for i in range(BH * ng):
+        bh, g = divmod(i, ng)
+        r0, r1 = int(goff[i]), int(goff[i + 1])
+        c = cnt[bh, g * 32:(g + 1) * 32]
+        assert r1 - r0 == c.max(), (i, r1 - r0, c.max())
+        blk = vals[r0 * 32:r1 * 32].reshape(r1 - r0, 32).T
+        slot = np.arange(r1 - r0)[None, :]
+        assert not np.any(blk[slot >= c[:, None]]), f"group {i}: nonzero unused slots"
+        out[bh, g * 32:(g + 1) * 32, :r1 - r0] = blk
+    return out[:, :S]
 
 
 def topp_near_ties(m_g, m_o, k_np, qn_np, p, Tcap):
@@ -74,8 +102,8 @@ def check_topp(kc, k_np, q_np, G, p, what):
     assert n_diff == near, f"{what}: {n_diff - near} of {n_diff} differing tokens are not near-ties"
     assert n_diff <= 1e-4 * BH * S, f"{what}: {n_diff} near-tie tokens of {BH * S}"
     ok = np.all(m_g == m_o, axis=-1)
+    v_g = unpack_topp(kc)
     if Tcap > 0:
-        v_g = unpack_vals(kc)
         assert np.array_equal(v_g[ok].view(np.uint32), v_o[ok].view(np.uint32)), f"{what}: vals"
     if n_diff == 0:
         assert np.array_equal(s_g[:, 0], s_o[:, 0]), f"{what}: pruned count"
@@ -121,6 +149,30 @@ def test_topp_extreme_tokens():
     for p, Tcap in ((0.99, 128), (0.999, 50), (1.0, 128)):
         kc = run_topp(k, pre["q_obs"], G, wl.W, p, Tcap)
         check_topp(kc, to_np(k), to_np(pre["q_obs"]), G, p, f"extreme p={p} Tcap={Tcap}")
+        # the groups whose tokens keep one channel or none take 1 or 0 slots
+        goff = kc.goff.cpu().numpy().view(np.uint32).astype(np.int64)
+        assert goff[1] - goff[0] == 0 and goff[2] - goff[1] == 1
+        assert spark_topp_vals_used(kc) < Hkv * S * Tcap * 2
+
+
+def test_topp_concentrated_saliency_stores_less():
+    """Keys whose saliency sits in a few channels per token (the concentrated
+    case SparK-p is made for): the compact stream holds about the kept
+    values, far below the capacity layout, and still matches the oracle."""
+    G, S, Hkv = 4, 4096, 2
+    wl = scaled(WORKLOADS["tiny"], S=S, G=G, Hkv=Hkv, dtype="bf16", seed=93)
+    pre = make_prefill(wl, DEV)
+    g = torch.Generator(device=DEV).manual_seed(93)
+    k = pre["k"].float() * 1e-3
+    hot = torch.randint(0, D, (1, Hkv, S, 6), generator=g, device=DEV)
+    k.scatter_(-1, hot, torch.randn(hot.shape, generator=g, device=DEV) * 10)
+    k = k.to(torch.bfloat16)
+    kc = run_topp(k, pre["q_obs"], G, wl.W, 0.99, 128)
+    check_topp(kc, to_np(k), to_np(pre["q_obs"]), G, 0.99, "concentrated")
+    used = spark_topp_vals_used(kc)
+    m = mask_np(kc)
+    kept = int(np.unpackbits(np.ascontiguousarray(m).view(np.uint8), axis=-1).sum())
+    assert kept * 2 <= used <= 4 * kept * 2 and used < Hkv * S * 128 * 2 / 8
 
 
 def test_topp_decode_gaussian_and_tail():
@@ -157,6 +209,9 @@ def test_topp_decode_equals_plain_decode_on_full_masks(dtype, T, G):
     pre = make_prefill(wl, DEV)
     kc = run_prune(pre["k"], pre["q_obs"], wl.G, wl.W, T)
     q = make_decode_step(wl, 0, DEV)["q"]
+    # the plain cache read through group offsets that give every group T slots
+    BH, ng = wl.rows * wl.Hkv, (wl.S + 31) // 32
+    kc.goff = (torch.arange(BH * ng + 1, device=DEV, dtype=torch.int64) * T).to(torch.int32)
     outs = []
     for fn in (spark_decode_attn, spark_decode_attn_topp):
         out = torch.empty((wl.rows, wl.Hkv * wl.G, D), dtype=torch.float32, device=DEV)
@@ -171,7 +226,8 @@ def test_topp_decode_equals_plain_decode_on_full_masks(dtype, T, G):
 def test_topp_full_size_sampled():
     """One layer of the long-context workload (8 heads x 131072 tokens) in
     the launch configuration of the benchmark: sampled tokens against the
-    oracle, every mask within the capacity."""
+    oracle, every mask within the capacity, and the compact value stream
+    smaller than the capacity layout."""
     wl = scaled(WORKLOADS["long"], L=1)
     pre = make_prefill(wl, DEV)
     Tcap = 96
@@ -187,7 +243,7 @@ def test_topp_full_size_sampled():
     st = kc.stats.cpu().numpy().reshape(BH, 4)
     assert np.array_equal(st[:, 0], (D - pc).sum(1).astype(np.float64))
     rng = np.random.default_rng(1)
-    vals_g = unpack_vals(kc)
+    vals_g = unpack_topp(kc)
     k_np = to_np(pre["k"]).reshape(BH, S, D)
     n_diff = n_near = 0
     for bh in range(BH):
@@ -198,6 +254,10 @@ def test_topp_full_size_sampled():
         ok = np.all(m_g[bh, ts] == m_o[0], axis=-1)
         assert np.array_equal(vals_g[bh, ts][ok].view(np.uint32), v_o[0][ok].view(np.uint32)), f"head {bh}"
     assert n_diff == n_near and n_diff <= 1e-4 * BH * 4096, (n_diff, n_near)
+    # the compact stream: each group holds its longest kept set (here nearly
+    # every group has a token cut at the cap, so it is close to the capacity)
+    used = spark_topp_vals_used(kc)
+    assert used == int(kc.goff[-1].item()) * 32 * 2 and used <= BH * S * Tcap * 2
 
 
 @pytest.mark.parametrize("G", [1, 2, 8])
