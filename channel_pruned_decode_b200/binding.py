@@ -35,7 +35,7 @@ EXPORTS = ("spark_lambda_to_T", "spark_cache_sizes", "spark_cache_bytes", "spark
            "spark_prune", "spark_prune_noalloc", "spark_prune_grouped", "spark_group_budget", "spark_prune_values", "spark_prune_think", "spark_prune_topp", "spark_decode_attn",
            "spark_decode_attn_topp", "spark_topp_offsets_bytes", "spark_topp_vals_used",
            "spark_decode_attn_kv", "spark_workspace_bytes_kv", "spark_selftest_wait_timeout", "spark_tail_append", "spark_device_status",
-           "spark_status_str", "spark_snapkv_evict")
+           "spark_status_str", "spark_snapkv_evict", "spark_snapkv_evict_rows", "spark_pyramid_keep")
 
 
 class SparkError(RuntimeError):
@@ -48,7 +48,7 @@ class spark_kcache(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hkv", ctypes.c_int), ("S", ctypes.c_int), ("D", ctypes.c_int),
                 ("T", ctypes.c_int), ("dtype", ctypes.c_int), ("mask", ctypes.c_void_p),
                 ("vals", ctypes.c_void_p), ("qn", ctypes.c_void_p), ("stats", ctypes.c_void_p),
-                ("goff", ctypes.c_void_p)]
+                ("goff", ctypes.c_void_p), ("lens", ctypes.c_void_p)]
 
 
 _lib = None
@@ -104,6 +104,10 @@ def lib():
         L.spark_decode_attn.restype = I
         L.spark_snapkv_evict.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P, Z, P]
         L.spark_snapkv_evict.restype = I
+        L.spark_snapkv_evict_rows.argtypes = [P, P, P, I, I, I, I, I, I, P, I, I, I, P, P, P, P, Z, P]
+        L.spark_snapkv_evict_rows.restype = I
+        L.spark_pyramid_keep.argtypes = [I, I, ctypes.c_float, I, I, ctypes.POINTER(I)]
+        L.spark_pyramid_keep.restype = I
         L.spark_tail_append.argtypes = [P, P, P, P, I, I, I, I, I, I, P]
         L.spark_tail_append.restype = I
         L.spark_device_status.argtypes = [P, ctypes.POINTER(I), I, P]
@@ -177,6 +181,7 @@ class KCache:
     qn: torch.Tensor      # fp32 [B, Hkv, D]
     stats: torch.Tensor   # fp64 [B, Hkv, 4]
     goff: torch.Tensor = None  # SparK-p only: int32 [B * Hkv * S32 / 32 + 1] first value row per group
+    lens: torch.Tensor = None  # optional int32 [B] prompt tokens per row (S is then the row stride)
 
     @staticmethod
     def empty(B, Hkv, S, D, T, dtype, device="cuda") -> "KCache":
@@ -199,7 +204,8 @@ class KCache:
     def struct(self) -> spark_kcache:
         return spark_kcache(self.B, self.Hkv, self.S, self.D, self.T, _dtype_code(self.dtype),
                             _ptr(self.mask), _ptr(self.vals), _ptr(self.qn), _ptr(self.stats),
-                            _ptr(self.goff) if self.goff is not None else None)
+                            _ptr(self.goff) if self.goff is not None else None,
+                            _ptr(self.lens) if self.lens is not None else None)
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in (self.mask, self.vals, self.qn, self.stats))
@@ -339,6 +345,26 @@ def spark_snapkv_evict(k: torch.Tensor, v: torch.Tensor, q_obs: torch.Tensor, G:
                                   _dtype_code(k.dtype), _ptr(k_out), _ptr(v_out), _ptr(idx_out), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "spark_snapkv_evict")
+
+
+def spark_snapkv_evict_rows(k: torch.Tensor, v: torch.Tensor, q_obs: torch.Tensor, G: int, W: int,
+                            keep_rows: torch.Tensor, keep_cap: int, pool: int, k_out: torch.Tensor,
+                            v_out: torch.Tensor, idx_out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    """SnapKV-style eviction with one budget per row (keep_rows: int32 [B] on
+    the device); outputs with row stride keep_cap (see spark.h)."""
+    B, Hkv, S, D = k.shape
+    rc = lib().spark_snapkv_evict_rows(_ptr(k), _ptr(v), _ptr(q_obs), B, Hkv, S, D, G, W, _ptr(keep_rows),
+                                       keep_cap, pool, _dtype_code(k.dtype), _ptr(k_out), _ptr(v_out),
+                                       _ptr(idx_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "spark_snapkv_evict_rows")
+
+
+def spark_pyramid_keep(L: int, M: int, beta: float, W: int, S: int) -> list:
+    """PyramidKV-style layer budgets around the mean M (the library's linear
+    reading, see spark.h)."""
+    out = (ctypes.c_int * max(L, 1))()
+    _check(lib().spark_pyramid_keep(L, M, ctypes.c_float(beta), W, S, out), "spark_pyramid_keep")
+    return [int(out[i]) for i in range(L)]
 
 
 def spark_tail_append(k_new, v_new, k_tail, v_tail, B, Hkv, D, tail_cap, slot, stream=None) -> None:

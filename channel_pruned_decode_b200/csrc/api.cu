@@ -21,7 +21,8 @@ cudaError_t launch_think(const void *k, const void *q_obs, int G, int W, const s
                          cudaStream_t st);
 size_t think_workspace(long BH, int S);
 cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
-                          int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st);
+                          int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st,
+                          const int32_t *keep_rows = nullptr, int Hkv = 1, int keep_cap = 0);
 
 size_t snapkv_partials_bytes(long BH);
 
@@ -171,6 +172,7 @@ int spark_prune_topp(const void *k, const void *q_obs, int G, int W, float p, co
                      void *workspace, size_t ws_bytes, void *stream) {
     int rc = check_cache(out);
     if (rc != SPARK_OK) return rc;
+    if (out->lens) return SPARK_ERR_UNSUPPORTED;
     if (G < 1 || W < 1) return SPARK_ERR_ARG;
     if (!(p >= 0.0f && p <= 1.0f)) return SPARK_ERR_ARG;
     const long BH = (long)out->B * out->Hkv;
@@ -214,6 +216,7 @@ static int decode_entry(const void *q, const spark_kcache *kc, const void *v, co
     int rc = check_cache(kc);
     if (rc != SPARK_OK) return rc;
     if (topp && (!kc->goff || (reinterpret_cast<uintptr_t>(kc->goff) & 3u))) return SPARK_ERR_ARG;
+    if (topp && kc->lens) return SPARK_ERR_UNSUPPORTED;
     if (G != 1 && G != 2 && G != 4 && G != 8) return G < 1 ? SPARK_ERR_ARG : SPARK_ERR_UNSUPPORTED;
     if (recovery != SPARK_F_DEGENERATE && recovery != SPARK_F_GAUSSIAN && recovery != SPARK_F_EXPONENTIAL)
         return SPARK_ERR_ARG;
@@ -264,6 +267,7 @@ int spark_prune_think(const void *k, const void *q_obs, int G, int W, const spar
                       size_t ws_bytes, void *stream) {
     int rc = check_cache(out);
     if (rc != SPARK_OK) return rc;
+    if (out->lens) return SPARK_ERR_UNSUPPORTED;
     if (G < 1 || W < 1) return SPARK_ERR_ARG;
     const long BH = (long)out->B * out->Hkv;
     if (BH == 0) return SPARK_OK;
@@ -332,6 +336,38 @@ int spark_snapkv_evict(const void *k, const void *v, const void *q_obs, int B, i
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
 }
 
+int spark_snapkv_evict_rows(const void *k, const void *v, const void *q_obs, int B, int Hkv, int S, int D, int G,
+                            int W, const int32_t *keep_rows, int keep_cap, int pool, int dtype, void *k_out,
+                            void *v_out, int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream) {
+    if (B < 0 || Hkv < 0 || S < 0 || G < 1 || W < 1 || elem_size(dtype) == 0) return SPARK_ERR_ARG;
+    if (D != kD || dtype != SPARK_BF16) return SPARK_ERR_UNSUPPORTED;
+    if ((G * W) % 16 != 0 || G * W > 128) return SPARK_ERR_UNSUPPORTED;
+    if (keep_cap < W || W > S || pool < 1 || (pool & 1) == 0) return SPARK_ERR_ARG;
+    const long BH = (long)B * Hkv;
+    if (BH == 0) return SPARK_OK;
+    if (!keep_rows || (reinterpret_cast<uintptr_t>(keep_rows) & 3u)) return SPARK_ERR_ARG;
+    if (!k || !v || !q_obs || !k_out || !v_out || !idx_out) return SPARK_ERR_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(q_obs) || !aligned16(k_out) || !aligned16(v_out) ||
+        !aligned16(idx_out))
+        return SPARK_ERR_ARG;
+    if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < snapkv_workspace(BH, S, W)) return SPARK_ERR_WORKSPACE;
+    cudaError_t e = launch_snapkv(k, v, q_obs, BH, S, G, W, W, pool, k_out, v_out, idx_out, workspace,
+                                  static_cast<cudaStream_t>(stream), keep_rows, Hkv, keep_cap);
+    return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;
+}
+
+int spark_pyramid_keep(int L, int M, float beta, int W, int S, int *keep) {
+    if (L < 1 || W < 1 || M < W || S < M || !(beta >= 0.0f && beta < 1.0f) || !keep) return SPARK_ERR_ARG;
+    for (int l = 0; l < L; ++l) {
+        const double f = L > 1 ? (double)(L - 1 - 2 * l) / (double)(L - 1) : 0.0;
+        long x = llround((double)M * (1.0 + (double)beta * f));
+        x = x < W ? W : (x > S ? S : x);
+        keep[l] = (int)x;
+    }
+    return SPARK_OK;
+}
+
 int spark_tail_append(const void *k_new, const void *v_new, void *k_tail, void *v_tail, int B, int Hkv,
                       int D, int tail_cap, int slot, int dtype, void *stream) {
     const int es = elem_size(dtype);
@@ -365,7 +401,7 @@ int spark_device_status(void *workspace, int *status, int clear, void *stream) {
     if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return SPARK_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return SPARK_ERR_CUDA;
-    *status = (word & kDevTimeout) ? SPARK_ERR_TIMEOUT : SPARK_OK;
+    *status = (word & kDevTimeout) ? SPARK_ERR_TIMEOUT : ((word & kDevBadArg) ? SPARK_ERR_ARG : SPARK_OK);
     if (clear && word) {
         if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return SPARK_ERR_CUDA;
         if (cudaStreamSynchronize(st) != cudaSuccess) return SPARK_ERR_CUDA;

@@ -57,6 +57,8 @@ struct DecArgs {
     const uint32_t *mask;
     const void *vals;
     const uint32_t *goff;   // SparK-p cache: first value row of each group (else NULL)
+    const int32_t *lens;    // prompt tokens per row (else NULL: S for every row)
+    int Hkv;
     const uint32_t *vmask;  // pruned value cache (packed-V kernels only)
     const void *vvals;
     int Tv;
@@ -577,11 +579,14 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
     auto item_head = [&](int item) -> int { return item < n_prompt ? item / a.n_pre : item - n_prompt; };
     auto item_unit = [&](int item) -> int { return item < n_prompt ? item % a.n_pre : a.n_pre; };
 
+    // prompt tokens of head bh (S is the row stride when rows have lengths)
+    auto head_len = [&](int bh) -> int { return row_len(a.lens, bh, a.Hkv, a.S, nullptr); };
+
     // ---- tile stream of this warp: prompt tiles of its items, in order
-    auto item_tiles = [&](int u) -> int {
+    auto item_tiles = [&](int bh, int u) -> int {
         if (u >= a.n_pre) return 0;  // dense-tail items are not streamed
         const long t0 = (long)u * a.chunk;
-        const long t1 = min((long)a.S, t0 + a.chunk);
+        const long t1 = min((long)head_len(bh), t0 + a.chunk);
         return t1 > t0 ? (int)((t1 - t0 + kWT - 1) / kWT) : 0;
     };
     // issue cursor: the next prompt tile to copy, with its item decoded once
@@ -593,7 +598,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         if (c.item < n_items) {
             c.bh = item_head(c.item);
             c.u = item_unit(c.item);
-            c.ntiles = item_tiles(c.u);
+            c.ntiles = item_tiles(c.bh, c.u);
         } else {
             c.ntiles = 0;
         }
@@ -610,7 +615,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         const long bh = c.bh;
         const int u = c.u;
         const long t0 = (long)u * a.chunk + (long)c.tile * kWT;
-        const long t1 = min((long)a.S, (long)u * a.chunk + a.chunk);
+        const long t1 = min((long)head_len((int)bh), (long)u * a.chunk + a.chunk);
         const int n = (int)min((long)kWT, t1 - t0);
         const uint32_t mb = (uint32_t)n * 16u;
         // one whole 32-token group of kept values: T slots, or for a SparK-p
@@ -748,9 +753,9 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
         }
 
         // ---- prompt tokens of this item, one 32-token tile at a time
-        const int ntiles = item_tiles(u);
+        const int ntiles = item_tiles(bh, u);
         const long t_item = (long)u * a.chunk;
-        const long t_end = min((long)a.S, t_item + a.chunk);
+        const long t_end = min((long)head_len(bh), t_item + a.chunk);
         const E *vbase = gv + (size_t)bh * a.S * kD;
         for (int tile = 0; tile < ntiles; ++tile) {
             const long t0 = t_item + (long)tile * kWT;
@@ -1140,6 +1145,8 @@ cudaError_t launch_decode(const void *q, const spark_kcache &kc, const void *v, 
     a.mask = kc.mask;
     a.vals = kc.vals;
     a.goff = topp ? kc.goff : nullptr;
+    a.lens = kc.lens;
+    a.Hkv = kc.Hkv;
     a.qn = kc.qn;
     a.stats = kc.stats;
     a.v = v;

@@ -333,7 +333,7 @@ template <typename E, bool kGrouped>
 __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
                  E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks, int gpc,
-                 GroupArgs ga) {
+                 GroupArgs ga, const int32_t *__restrict__ lens, int Hkv, uint32_t *__restrict__ status) {
     using Raw = typename RawT<E>::type;
     // per-warp staging of the kept values: [kept index][8 tokens of the warp]
     __shared__ __align__(16) Raw vtile[kPruneThreads / 32][kD * 8];
@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     const int tq = lane >> 2;               // token within the warp's 8
     const int tl = warp * 8 + tq;           // token within the 32-token group
     const long S32 = ((long)S + 31) / 32 * 32;
+    const int Sb = row_len(lens, bh, Hkv, S, tid == 0 ? status : nullptr);  // tokens of this row (S: its stride)
 
     // the 16-bit keys are fp16(key * scale), scale = 2^-floor(log2 max_j qn_j),
     // so the largest window-query norm maps into [1, 2) and the keys of
@@ -422,8 +423,8 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     // slice; the next group's slice is loaded into `nxt` first.
     auto group = [&](int gi, KSlice<E> &cur, KSlice<E> &nxt) {
         const long t = (g_first + gi) * 32 + tl;
-        const bool valid = t < S;
-        if (gi + 1 < gpc && t + 32 < S) nxt.load(krow + (size_t)(gi + 1) * 32 * kD);
+        const bool valid = t < Sb;
+        if (gi + 1 < gpc && t + 32 < Sb) nxt.load(krow + (size_t)(gi + 1) * 32 * kD);
         else nxt.zero();
 
         // exact fp32 saliency keys w_j = qn_j * |k_j| (packed fp32 multiplies,
@@ -556,12 +557,12 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     };
 
     KSlice<E> ka, kb;
-    if (g_first * 32 + tl < S) ka.load(krow);
+    if (g_first * 32 + tl < Sb) ka.load(krow);
     else ka.zero();
     for (int gi = 0; gi < gpc; gi += 2) {
-        if ((g_first + gi) * 32 >= S) break;  // uniform across the CTA
+        if ((g_first + gi) * 32 >= Sb) break;  // uniform across the CTA
         group(gi, ka, kb);
-        if ((g_first + gi + 1) * 32 >= S) break;
+        if ((g_first + gi + 1) * 32 >= Sb) break;
         group(gi + 1, kb, ka);
     }
 
@@ -590,7 +591,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
 // One warp per (row, kv head): lanes sum the chunk partials in a fixed order,
 // then a fixed xor tree.
 __global__ void stats_kernel(const double *__restrict__ partial, int n_chunks, long BH, int S, int T,
-                             double *__restrict__ stats) {
+                             double *__restrict__ stats, const int32_t *__restrict__ lens, int Hkv) {
     const long bh = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (bh >= BH) return;
@@ -605,7 +606,7 @@ __global__ void stats_kernel(const double *__restrict__ partial, int n_chunks, l
         b = __dadd_rn(b, __shfl_xor_sync(0xffffffffu, b, o));
     }
     if (lane == 0) {
-        const double n = (double)S * (double)(kD - T);
+        const double n = (double)row_len(lens, bh, Hkv, S, nullptr) * (double)(kD - T);
         stats[bh * 4 + 0] = n;
         stats[bh * 4 + 1] = a;
         stats[bh * 4 + 2] = b;
@@ -626,13 +627,14 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
         if (ga)
             prune_kernel<E, true><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-                nch, gpc, *ga);
+                nch, gpc, *ga, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
         else
             prune_kernel<E, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-                nch, gpc, GroupArgs{});
+                nch, gpc, GroupArgs{}, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
     }
-    stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.S, kc.T, kc.stats);
+    stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.S, kc.T, kc.stats, kc.lens,
+                                                           kc.Hkv);
     return cudaGetLastError();
 }
 
@@ -666,13 +668,14 @@ cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws,
         if (vc.dtype == SPARK_BF16)
             prune_kernel<__nv_bfloat16, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16 *>(v), vc.qn, vc.mask, static_cast<__nv_bfloat16 *>(vc.vals),
-                partial, vc.S, vc.T, nch, gpc, GroupArgs{});
+                partial, vc.S, vc.T, nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws));
         else
             prune_kernel<float, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const float *>(v), vc.qn, vc.mask, static_cast<float *>(vc.vals), partial, vc.S, vc.T,
-                nch, gpc, GroupArgs{});
+                nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws));
     }
-    stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, vc.S, vc.T, vc.stats);
+    stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, vc.S, vc.T, vc.stats, vc.lens,
+                                                           vc.Hkv);
     return cudaGetLastError();
 }
 

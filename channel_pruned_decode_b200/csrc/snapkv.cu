@@ -87,17 +87,25 @@ __device__ __forceinline__ int block_excl_scan(int v, int *wsum, int &total) {
 
 __global__ void __launch_bounds__(kSelThreads)
     snap_select_kernel(const float *__restrict__ scores, uint32_t *__restrict__ pooled, int S, int W, int keep,
-                       int pool, int *__restrict__ idx) {
+                       int pool, int *__restrict__ idx, const int32_t *__restrict__ keep_rows, int Hkv,
+                       int keep_cap, uint32_t *__restrict__ status) {
     __shared__ int hist[256];
     __shared__ int wsum[32];
     __shared__ uint32_t sel[3];  // prefix, remaining rank, digit
     const long bh = blockIdx.x;
     const int tid = threadIdx.x;
     const long P = (long)S - W;
+    if (keep_rows) {  // a budget per row (uniform over the CTA)
+        keep = keep_rows[bh / Hkv];
+        if (keep < W || keep > S || keep > keep_cap) {
+            if (tid == 0) atomicOr(status, kDevBadArg);
+            return;
+        }
+    }
     const int kp = keep - W;
     const float *sc = scores + (size_t)bh * P;
     uint32_t *pk = pooled + (size_t)bh * P;
-    int *out = idx + (size_t)bh * keep;
+    int *out = idx + (size_t)bh * keep_cap;
     const int h = pool / 2;
 
     // max-pool; scores are >= 0 so the fp32 bit pattern orders them
@@ -192,15 +200,20 @@ __global__ void __launch_bounds__(kSelThreads)
 }
 
 __global__ void snap_gather_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
-                                   const int *__restrict__ idx, int S, int keep, int row_vec,
-                                   uint4 *__restrict__ k_out, uint4 *__restrict__ v_out) {
+                                   const int *__restrict__ idx, int S, int W, int keep, int row_vec,
+                                   uint4 *__restrict__ k_out, uint4 *__restrict__ v_out,
+                                   const int32_t *__restrict__ keep_rows, int Hkv, int keep_cap) {
     const long bh = blockIdx.y;
     const long i = (long)blockIdx.x * (blockDim.x / row_vec) + threadIdx.x / row_vec;
     const int c = threadIdx.x % row_vec;
+    if (keep_rows) {
+        keep = keep_rows[bh / Hkv];
+        if (keep < W || keep > S || keep > keep_cap) return;  // recorded by the select kernel
+    }
     if (i >= keep) return;
-    const long t = idx[bh * keep + i];
-    k_out[((size_t)bh * keep + i) * row_vec + c] = k[((size_t)bh * S + t) * row_vec + c];
-    v_out[((size_t)bh * keep + i) * row_vec + c] = v[((size_t)bh * S + t) * row_vec + c];
+    const long t = idx[bh * keep_cap + i];
+    k_out[((size_t)bh * keep_cap + i) * row_vec + c] = k[((size_t)bh * S + t) * row_vec + c];
+    v_out[((size_t)bh * keep_cap + i) * row_vec + c] = v[((size_t)bh * S + t) * row_vec + c];
 }
 
 // ---------------------------------------------------------------------------
@@ -599,7 +612,8 @@ static bool make_key_map(CUtensorMap *tm, const void *k, long BH, int S) {
 }
 
 cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long BH, int S, int G, int W, int keep,
-                          int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st) {
+                          int pool, void *k_out, void *v_out, int *idx_out, void *ws, cudaStream_t st,
+                          const int32_t *keep_rows, int Hkv, int keep_cap) {
     const long P = (long)S - W;
     float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeader);
     uint32_t *pooled = reinterpret_cast<uint32_t *>(scores + (size_t)BH * P);
@@ -618,12 +632,15 @@ cudaError_t launch_snapkv(const void *k, const void *v, const void *q_obs, long 
     if (!make_key_map(&tmap, k, BH, S)) return cudaErrorInvalidValue;
     snap_tc_kernel<0><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(tmap, qb, S, G, W, ns, ml, scores, status);
     snap_tc_kernel<1><<<(unsigned)(BH * ns), kTcThreads, smem, st>>>(tmap, qb, S, G, W, ns, ml, scores, status);
-    snap_select_kernel<<<(unsigned)BH, kSelThreads, 0, st>>>(scores, pooled, S, W, keep, pool, idx_out);
+    if (!keep_rows) keep_cap = keep;
+    snap_select_kernel<<<(unsigned)BH, kSelThreads, 0, st>>>(scores, pooled, S, W, keep, pool, idx_out, keep_rows,
+                                                              Hkv, keep_cap, status);
     const int row_vec = kD * 2 / 16;  // bf16 rows
     const int rows_per_cta = 256 / row_vec;
-    snap_gather_kernel<<<dim3((unsigned)((keep + rows_per_cta - 1) / rows_per_cta), (unsigned)BH), 256, 0, st>>>(
-        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), idx_out, S, keep, row_vec,
-        static_cast<uint4 *>(k_out), static_cast<uint4 *>(v_out));
+    snap_gather_kernel<<<dim3((unsigned)((keep_cap + rows_per_cta - 1) / rows_per_cta), (unsigned)BH), 256, 0,
+                         st>>>(static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), idx_out, S, W, keep,
+                               row_vec, static_cast<uint4 *>(k_out), static_cast<uint4 *>(v_out), keep_rows, Hkv,
+                               keep_cap);
     return cudaGetLastError();
 }
 

@@ -15,6 +15,7 @@ constexpr int kD = 128;               // head dimension the kernels are built fo
 constexpr int kMaskWords = kD / 32;   // 128-bit channel mask per token
 constexpr int kWsHeader = 256;        // status word + padding at workspace start
 constexpr uint32_t kDevTimeout = 1u;  // status bit: a bounded wait ran out
+constexpr uint32_t kDevBadArg = 2u;   // status bit: a device-side length or budget was out of range
 
 // ------------------------------------------------------- argument checks
 inline int elem_size(int dtype) { return dtype == SPARK_F32 ? 4 : (dtype == SPARK_BF16 ? 2 : 0); }
@@ -29,6 +30,7 @@ inline int check_cache(const spark_kcache *kc) {
     if (elem_size(kc->dtype) == 0) return SPARK_ERR_ARG;
     if (kc->D != kD) return SPARK_ERR_UNSUPPORTED;
     if (kc->T < 0 || kc->T > kc->D) return SPARK_ERR_ARG;
+    if (kc->lens && (reinterpret_cast<uintptr_t>(kc->lens) & 3u)) return SPARK_ERR_ARG;
     if ((long)kc->B * kc->Hkv == 0) return SPARK_OK;
     if (!kc->qn || !kc->stats || !aligned16(kc->qn) || !aligned16(kc->stats)) return SPARK_ERR_ARG;
     if (kc->S > 0) {
@@ -172,6 +174,19 @@ template <> struct Elem<__nv_bfloat16> {
     static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
     static constexpr int size = 2;
 };
+
+// Prompt tokens of head bh: S, or the row's entry of a per-row length array
+// (row = bh / Hkv), clamped to [0, S]; an out-of-range entry is recorded in
+// the status word.
+__device__ __forceinline__ int row_len(const int32_t *lens, long bh, int Hkv, int S, uint32_t *status) {
+    if (!lens) return S;
+    const int n = lens[bh / Hkv];
+    if (n < 0 || n > S) {
+        if (status) atomicOr(status, kDevBadArg);
+        return n < 0 ? 0 : S;
+    }
+    return n;
+}
 
 // ------------------------------------------------------------- PTX glue
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -98,6 +98,18 @@ typedef enum {
  *         vals[(goff[i] + j)*32 + t % 32]; T_i is the largest kept count of
  *         the group's tokens, and the slots past a token's own count (and
  *         all slots of padding tokens) hold 0.
+ *   lens  NULL when every row holds S prompt tokens.  Otherwise int32 [B]
+ *         in device memory: row b holds lens[b] <= S tokens (its first
+ *         lens[b] token slots; S is then the row stride, e.g. the capacity
+ *         of an eviction with per-row budgets).  spark_prune,
+ *         spark_prune_grouped, spark_prune_values, spark_prune_noalloc and
+ *         the decodes spark_decode_attn and spark_decode_attn_kv honour it;
+ *         the statistics count N = lens[b] * (D - T); mask and value slots
+ *         past a row's length are left untouched.  A length outside
+ *         [0, S] is clamped into it and raises SPARK_ERR_ARG in the device
+ *         status word.  spark_prune_think, spark_prune_topp and
+ *         spark_decode_attn_topp return SPARK_ERR_UNSUPPORTED when it is
+ *         set.
  */
 typedef struct spark_kcache {
     int B, Hkv, S, D, T, dtype;
@@ -106,6 +118,7 @@ typedef struct spark_kcache {
     float *qn;
     double *stats;
     uint32_t *goff;
+    const int32_t *lens;
 } spark_kcache;
 
 /* Kept channels for pruning ratio lambda ([A] Table 1 caption, [W] 4.1):
@@ -377,6 +390,41 @@ SPARK_API int spark_snapkv_evict(const void *k, const void *v, const void *q_obs
                                  size_t ws_bytes, void *stream);
 
 /*
+ * SnapKV-style eviction with a budget per batch row (the PyramidKV base of
+ * [W] 4.1 / 4.2 stacks SparK on layer-wise budgets; callers with L layers
+ * pass B*L rows, row = l*B + b, so a row's budget is its layer's).  As
+ * spark_snapkv_evict, except that
+ *   keep_rows  int32 [B] in device memory: row b keeps keep_rows[b] tokens,
+ *              W <= keep_rows[b] <= min(S, keep_cap)
+ *   keep_cap   the row stride of the outputs: k_out, v_out
+ *              [B][Hkv][keep_cap][D], idx_out int32 [B][Hkv][keep_cap]
+ * Row b's kept tokens fill its first keep_rows[b] slots (ascending); the
+ * slots after them are left untouched.  Prune and decode the result with
+ * kc.S = keep_cap and kc.lens = keep_rows.  A budget outside its range
+ * evicts nothing for that row and raises SPARK_ERR_ARG in the device status
+ * word (read with spark_device_status).  Workspace:
+ * spark_workspace_bytes(SPARK_OP_SNAPKV, ...) for S.
+ */
+SPARK_API int spark_snapkv_evict_rows(const void *k, const void *v, const void *q_obs, int B, int Hkv,
+                                      int S, int D, int G, int W, const int32_t *keep_rows, int keep_cap,
+                                      int pool, int dtype, void *k_out, void *v_out, int32_t *idx_out,
+                                      void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * PyramidKV-style layer budgets (the pages name PyramidKV as the eviction
+ * base SparK is stacked on, [W] 4.1 / 4.2, but give no schedule).  The
+ * library's reading: a budget falling linearly with depth around the mean
+ * budget M (the "KV-size"),
+ *   keep[l] = round(M * (1 + beta * (L - 1 - 2 l) / (L - 1)))   (L > 1),
+ * i.e. M (1 + beta) for the first layer, M (1 - beta) for the last, mean M
+ * before rounding (halves away from zero, fp64), then clamped to [W, S];
+ * keep[0] = M for L = 1.  beta in [0, 1).  Writes keep[0..L-1] (host).
+ * Returns SPARK_ERR_ARG for L < 1, W < 1, M < W, S < M, beta outside [0, 1)
+ * or a NULL keep.  Host arithmetic only.
+ */
+SPARK_API int spark_pyramid_keep(int L, int M, float beta, int W, int S, int *keep);
+
+/*
  * Append one unpruned decode-time key/value per (row, kv head) into the
  * dense tail at row `slot` (configs that "append unpruned new keys").
  *   k_new, v_new [B][Hkv][D] dtype;  k_tail, v_tail [B][Hkv][tail_cap][D].
@@ -387,8 +435,10 @@ SPARK_API int spark_tail_append(const void *k_new, const void *v_new, void *k_ta
                       int slot, int dtype, void *stream);
 
 /* Synchronise `stream`, read the device status word at the start of
- * `workspace` into *status (SPARK_OK or SPARK_ERR_TIMEOUT) and, when
- * clear != 0, reset it to zero.  Returns SPARK_ERR_CUDA if a copy fails. */
+ * `workspace` into *status (SPARK_OK, SPARK_ERR_TIMEOUT when a bounded wait
+ * ran out, SPARK_ERR_ARG when a device-side length or budget was out of
+ * range) and, when clear != 0, reset it to zero.  Returns SPARK_ERR_CUDA if
+ * a copy fails. */
 SPARK_API int spark_device_status(void *workspace, int *status, int clear, void *stream);
 
 /*

@@ -78,6 +78,8 @@ def _bind(lib):
     lib.oracle_group_of_channel.restype = None
     lib.oracle_group_budget.argtypes = [I, I, P, P]
     lib.oracle_group_budget.restype = None
+    lib.oracle_pyramid_keep.argtypes = [I, I, ctypes.c_double, I, I, P]
+    lib.oracle_pyramid_keep.restype = None
     lib.oracle_prune_grouped.argtypes = [P, P, L, L, I, I, P, P, P, P]
     lib.oracle_prune_grouped.restype = None
     lib.oracle_recover_values.argtypes = [P, P, L, L, I, I, P]
@@ -166,6 +168,15 @@ def group_of_channel(qn, g: int, lib=None) -> np.ndarray:
     gid = np.zeros((BH, D), np.int32)
     lib.oracle_group_of_channel(_ptr(qn), BH, D, g, _ptr(gid))
     return gid
+
+
+def pyramid_keep(L: int, M: int, beta: float, W: int, S: int, lib=None) -> list:
+    """PyramidKV-style layer budgets (reading R20); beta is taken as the
+    fp32 value the C library receives."""
+    lib = lib or load()
+    out = np.zeros(max(L, 1), np.int32)
+    lib.oracle_pyramid_keep(L, M, float(np.float32(beta)), W, S, _ptr(out))
+    return [int(x) for x in out[:L]]
 
 
 def group_budget(D: int, rates, lib=None) -> list:

@@ -765,3 +765,29 @@ void oracle_decode_f(const float *q, const uint32_t *mask, const float *vals, co
     free(s);
     free(acc);
 }
+
+/*
+ * PyramidKV layer budgets (reading R20).  [W] 4.1 and 4.2 stack SparK on
+ * PyramidKV, a token eviction whose budget differs per layer, but give no
+ * schedule.  The reading: the budget of layer l of L falls linearly with
+ * depth around the mean budget M ("KV-size"), from M (1 + beta) at the first
+ * layer to M (1 - beta) at the last, rounded half away from zero, then
+ * clamped to [W, S]; a single layer keeps M.
+ */
+void oracle_pyramid_keep(int L, int M, double beta, int W, int S, int *keep)
+{
+    for (int l = 0; l < L; ++l) {
+        double frac = 0.0;  /* +1 at the first layer, -1 at the last */
+        if (L > 1)
+            frac = 1.0 - 2.0 * (double)l / (double)(L - 1);
+        double x = (double)M + (double)M * beta * frac;
+        long r = (long)floor(fabs(x) + 0.5);
+        if (x < 0.0)
+            r = -r;
+        if (r < W)
+            r = W;
+        if (r > S)
+            r = S;
+        keep[l] = (int)r;
+    }
+}

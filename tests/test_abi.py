@@ -225,7 +225,8 @@ int main(void) {
     if (Tg[0] != 24 || Tg[1] != 16 || Tg[2] != 8 || Tg[3] != 0) return 7;
     /* argument errors come back before anything is launched */
     if (spark_prune(NULL, NULL, 4, 32, NULL, NULL, 0, NULL) != SPARK_ERR_ARG) return 8;
-    spark_kcache kc = {1, 8, 32768, 96, 64, SPARK_BF16, NULL, NULL, NULL, NULL, NULL};
+    spark_kcache kc = {0};
+    kc.B = 1; kc.Hkv = 8; kc.S = 32768; kc.D = 96; kc.T = 64; kc.dtype = SPARK_BF16;
     if (spark_prune(NULL, NULL, 4, 32, &kc, NULL, 0, NULL) != SPARK_ERR_UNSUPPORTED) return 9;
     if (spark_status_str(SPARK_ERR_ARG) == NULL) return 10;
     printf("ok %zu\n", total);

@@ -18,7 +18,8 @@ PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_group_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_vprune_pins.py"),
         os.path.join(ROOT, "tests", "test_oracle_think_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_topp_pins.py")]
+        os.path.join(ROOT, "tests", "test_oracle_topp_pins.py"),
+        os.path.join(ROOT, "tests", "test_oracle_pyramid_pins.py")]
 
 MUTANTS = {
     "tie_rule_reversed": ("return (a->j > b->j) - (a->j < b->j);",
@@ -86,6 +87,12 @@ MUTANTS = {
     "topp_channel_order": ("                cum += (double)order[n].w;", "                cum += (double)w[n];"),
     "topp_cap_off_by_one": ("const int n_keep = n < Tcap ? n : Tcap;", "const int n_keep = n < Tcap ? n : Tcap - 1;"),
     "topp_padding_not_zero": ("vrow[r] = 0.0f;", "vrow[r] = 1.0f;"),
+    # PyramidKV budgets (reading R20)
+    "pyramid_increasing": ("frac = 1.0 - 2.0 * (double)l / (double)(L - 1);",
+                           "frac = 2.0 * (double)l / (double)(L - 1) - 1.0;"),
+    "pyramid_denominator_L": ("frac = 1.0 - 2.0 * (double)l / (double)(L - 1);",
+                              "frac = 1.0 - 2.0 * (double)l / (double)L;"),
+    "pyramid_truncates": ("long r = (long)floor(fabs(x) + 0.5);", "long r = (long)floor(fabs(x));"),
     "lambda_truncates": ("return (int)llround((1.0 - (double)lambda) * (double)D);",
                          "return (int)((1.0 - (double)lambda) * (double)D);"),
 }
