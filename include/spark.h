@@ -107,7 +107,8 @@ typedef enum {
  *         the statistics count N = lens[b] * (D - T); mask and value slots
  *         past a row's length are left untouched.  A length outside
  *         [0, S] is clamped into it and raises SPARK_ERR_ARG in the device
- *         status word.  spark_prune_think, spark_prune_topp and
+ *         status word (spark_prune_noalloc has no workspace to report it
+ *         in: there the clamp is silent).  spark_prune_think, spark_prune_topp and
  *         spark_decode_attn_topp return SPARK_ERR_UNSUPPORTED when it is
  *         set.
  */
