@@ -29,8 +29,12 @@
 //   stats_kernel   fixed-order fp64 sum of the CTA partials per head, then
 //                  N = S*(D-T) and mu_pruned = sum w / N.
 // All reductions have a fixed order, so reruns are bit-identical.  SparK-g
-// uses prune_kernel with per-group selections; SparK-p (per-token top-p
-// selection) has its own kernel, prune_topp_kernel, described with it below.
+// uses prune_kernel with per-group selections: with four groups of 32
+// channels the quad's lanes exchange their 16-bit keys through shared memory
+// so that lane s searches group s, all four groups at once, with per-lane
+// tensor-core counts; other group counts search the groups one after the
+// other over the whole quad.  SparK-p (per-token top-p selection) has its own
+// kernel, prune_topp_kernel, described with it below.
 #include "spark_internal.cuh"
 
 #include <cuda_fp16.h>
@@ -151,15 +155,29 @@ __device__ __forceinline__ void mma_f16(uint32_t &d0, uint32_t &d1, uint32_t a0,
 // keys of one token, and rows r and r + 8 (the two accumulator registers)
 // together cover all 128 channels.  Which channel sits in which column is
 // irrelevant to a sum.  Every lane of the quad receives the count.
-__device__ __forceinline__ __half count_ge16(const uint32_t (&kp)[16], uint32_t p2) {
-    constexpr uint32_t kOne2 = 0x3c003c00u;  // fp16 (1, 1)
+//
+// With bsel in place of the all-ones operand (see own_count_operand) each
+// lane instead receives the count of its own 32 keys.
+constexpr uint32_t kOne2 = 0x3c003c00u;  // fp16 (1, 1)
+
+__device__ __forceinline__ __half count_ge16(const uint32_t (&kp)[16], uint32_t p2, uint32_t bsel = kOne2) {
     uint32_t d0 = 0u, d1 = 0u;
 #pragma unroll
     for (int m = 0; m < 4; ++m)
         mma_f16(d0, d1, hge2_one(kp[4 * m + 0], p2), hge2_one(kp[4 * m + 1], p2), hge2_one(kp[4 * m + 2], p2),
-                hge2_one(kp[4 * m + 3], p2), kOne2, kOne2);
+                hge2_one(kp[4 * m + 3], p2), bsel, bsel);
     const __half2 c = __hadd2(*reinterpret_cast<const __half2 *>(&d0), *reinterpret_cast<const __half2 *>(&d1));
     return __low2half(c);
+}
+
+// B operand that makes count_ge16 a per-lane count.  Columns k = 2s, 2s+1,
+// 2s+8, 2s+9 of an A row come from position s of the row's quad; B column
+// 2s is one on exactly those rows and every odd column is zero, so output
+// column 2s, which lands in the low half of the quad's position-s lane,
+// counts that lane's keys alone.  B rows 2s', 2s'+1, 2s'+8, 2s'+9 of column n
+// sit in the lane at quad n, position s'.
+__device__ __forceinline__ uint32_t own_count_operand(int lane) {
+    return (lane >> 2) == 2 * (lane & 3) ? kOne2 : 0u;
 }
 
 // Number of the quad's keys >= mid among the channels of `gm` (bit i =
@@ -179,40 +197,41 @@ constexpr uint32_t kTop16 = 0x7c01u;  // above +inf: no key reaches it, never pr
 constexpr uint32_t kGallop16 = 256u;  // first gallop step of the fallback search, fp16 units
 constexpr int kLift = 11;             // search window 2^11 fp16 units (2 octaves) around the estimate
 constexpr int kLiftCold = 12;         // first token of a quad: 2^12 units (4 octaves) below its top key
+// one lane per group of 32 channels: the threshold of a few of 32 keys moves
+// more from token to token, so the window spans 2 octaves on each side
+constexpr int kLiftLane = 12;
 
-// Mask word (32 channels) of this lane's quarter of the token: the T largest
-// exact fp32 keys over the quad, ties to the lower channel index.  0 < T < 128.
+// Phase 1 of the selection: the fp16 threshold lo of the T largest 16-bit
+// keys.  kp[i] holds the keys of two channels (which two does not matter to
+// the counts); the keys are the fp32 keys scaled by a power of two and
+// rounded to fp16, which is monotone in the key.  With kOwn false the keys of
+// the quad's four lanes are counted together (one token, 128 channels); with
+// kOwn true each lane counts its own 32 keys.
 //
-// kp[i] holds the 16-bit keys of channels i (low half) and i + 16 (high
-// half): the fp32 keys scaled by a power of two and rounded to fp16, which is
-// monotone in the key.  Phase 1 finds the fp16 threshold by binary lifting
-// over the window [base, base + 2^K): assuming count(>= base) >= T, after the
-// probe for bit b, lo is the largest point base + j * 2^b with
-// count(>= lo) >= T.  A probe that counts exactly T keys fixes the mask
-// (keys >= lo), and later probes keep that true, so the loop ends as soon as
-// every quad of the warp has seen one.  Otherwise the band of fp16 keys equal
-// to lo holds the boundary; if the window may not have bracketed it (lo never
-// moved, or reached the window's top) a gallop + bisection over the whole key
-// range redoes the search.  Phase 2 bisects the exact fp32 keys inside the
-// band, and a scan over the quad settles exact ties.  Every loop has a
-// warp-uniform trip count (finished quads idle), so the quad shuffles and the
-// warp-wide tensor-core counts see the full warp.  Only the channels of gm
-// take part (a SparK-g group; all ones otherwise): the caller sets the fp16
-// keys of the others negative, below every probe.
-__device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
-                                                 int s, float inv_scale, uint32_t base, int K, bool skip,
-                                                 uint32_t gm, uint32_t &tau) {
+// Binary lifting over the window [base, base + 2^K): assuming count(>= base)
+// >= T, after the probe for bit b, lo is the largest point base + j * 2^b
+// with count(>= lo) >= T.  A probe that counts exactly T keys fixes the
+// selection (keys >= lo: `exact`), and later probes keep that true, so the
+// loop ends as soon as every searcher of the warp has seen one.  Otherwise
+// the band of fp16 keys equal to lo holds the boundary and count(>= lo + 1)
+// < T; if the window may not have bracketed it (lo never moved, or reached
+// the window's top) a gallop + bisection over the whole key range redoes the
+// search.  Every loop has a warp-uniform trip count (finished searchers
+// idle), so the shuffles and the warp-wide tensor-core counts see the full
+// warp.  Keys that must not count are set negative, below every probe.
+template <bool kOwn>
+__device__ __forceinline__ void search_fp16(const uint32_t (&kp)[16], int T, uint32_t base, int K, bool skip,
+                                            uint32_t bsel, uint32_t &lo_out, bool &exact_out) {
     const __half hT = __int2half_rn(T);
     uint32_t lo = base;
-    bool exact = skip;  // lanes past the end of the keys take no part
+    bool exact = skip;  // searchers past the end of the keys take no part
     for (int b = K - 1; b >= 0; --b) {
         const uint32_t p = lo + (1u << b);
-        const __half c = count_ge16(kp, p * 0x10001u);
+        const __half c = count_ge16(kp, p * 0x10001u, kOwn ? bsel : kOne2);
         lo = __hge(c, hT) ? p : lo;
         exact = exact || __heq(c, hT);
         if (__all_sync(0xffffffffu, exact)) break;
     }
-    uint32_t hi = lo + 1u;
     const bool suspect = !exact && (lo == base || lo == base + (1u << K) - 1u);
     if (__any_sync(0xffffffffu, suspect)) {
         // count(>= glo) >= T > count(>= ghi); gallop from lo away from the
@@ -222,7 +241,7 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
         uint32_t step = kGallop16;
         uint32_t mid = min(max(lo, 1u), kTop16 - 1u);
         while (__any_sync(0xffffffffu, !done)) {
-            const __half c = count_ge16(kp, mid * 0x10001u);
+            const __half c = count_ge16(kp, mid * 0x10001u, kOwn ? bsel : kOne2);
             const bool ge = __hge(c, hT);
             const bool act = !done;
             glo = (act && ge) ? mid : glo;
@@ -237,24 +256,28 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
             mid = up ? gal_up : (down ? gal_dn : bis);
             step <<= 1;
         }
+        // not exact: the bisection ended with ghi = glo + 1
         lo = suspect ? glo : lo;
-        hi = suspect ? ghi : hi;
     }
-    tau = lo;
+    lo_out = lo;
+    exact_out = exact;
+}
 
-    // fp16 decision: keys >= lo (exactly T of them when `exact`)
-    uint32_t m = 0u;
-    {
-        const uint32_t p2 = lo * 0x10001u;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) m |= hge2_mask(kp[i], p2) & (0x00010001u << i);
-    }
-    if (!__any_sync(0xffffffffu, !exact)) return m;
+// Phase 2: the mask word (32 channels of this lane's quarter) of the T
+// largest exact fp32 keys among the quad's channels of gm (bit i = channel i
+// of this lane's quarter takes part), ties to the lower channel index, given
+// the phase-1 result: m16 = the channels of gm whose fp16 key is >= lo, which
+// is the answer when `exact`; otherwise count(fp16 >= lo) >= T > count(fp16
+// >= lo + 1).  Warp-uniform: every lane of the warp calls it.
+__device__ __forceinline__ uint32_t refine_fp32(const uint32_t (&key)[32], int T, int s, float inv_scale,
+                                                uint32_t lo, bool exact, uint32_t gm, uint32_t m16) {
+    if (!__any_sync(0xffffffffu, !exact)) return m16;
+    const uint32_t hi = lo + 1u;
 
-    // ---- phase 2 on the exact keys.  With v = the fp16 value of lo - 1 and
-    // u that of hi = lo + 1, every key whose fp16 key is >= lo is > v / scale,
-    // and every key >= u / scale has an fp16 key >= hi, so [v / scale,
-    // u / scale) in fp32 bit patterns brackets the T-th largest key.
+    // With v = the fp16 value of lo - 1 and u that of hi = lo + 1, every key
+    // whose fp16 key is >= lo is > v / scale, and every key >= u / scale has
+    // an fp16 key >= hi, so [v / scale, u / scale) in fp32 bit patterns
+    // brackets the T-th largest key.
     uint32_t lo32 = lo == 0u ? 0u : __float_as_uint(half_bits_to_float(lo - 1u) * inv_scale);
     uint32_t hi32 = hi >= kTop16 ? 0x7f800001u : __float_as_uint(half_bits_to_float(hi) * inv_scale);
     {
@@ -320,7 +343,35 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
             }
         }
     }
-    return exact ? m : m32;
+    return exact ? m16 : m32;
+}
+
+// fp16 decision of one quarter: bit i of the word = channel i, set where the
+// channel's 16-bit key is >= its threshold.  p2[i] holds the thresholds of
+// channels (i, i + 16), the layout of kp.
+__device__ __forceinline__ uint32_t decide_fp16(const uint32_t (&kp)[16], const uint32_t (&p2)[16]) {
+    uint32_t m = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m |= hge2_mask(kp[i], p2[i]) & (0x00010001u << i);
+    return m;
+}
+
+// Mask word (32 channels) of this lane's quarter of the token: the T largest
+// exact fp32 keys over the quad's channels of gm, ties to the lower channel
+// index.  0 < T < 128.  kp[i] holds the 16-bit keys of channels i (low half)
+// and i + 16 (high half); the caller sets the keys of channels outside gm
+// negative.
+__device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
+                                                 int s, float inv_scale, uint32_t base, int K, bool skip,
+                                                 uint32_t gm, uint32_t &tau) {
+    uint32_t lo;
+    bool exact;
+    search_fp16<false>(kp, T, base, K, skip, kOne2, lo, exact);
+    tau = lo;
+    uint32_t p2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) p2[i] = lo * 0x10001u;
+    return refine_fp32(key, T, s, inv_scale, lo, exact, gm, decide_fp16(kp, p2));
 }
 
 // SparK-g groups: number of groups and each group's kept-channel budget.
@@ -329,12 +380,18 @@ struct GroupArgs {
     int T[kMaxGroups];
 };
 
-template <typename E, bool kGrouped>
+// prune_kernel modes: one top-T selection per token; SparK-g with any number
+// of groups, searched one after the other over the whole quad; SparK-g with
+// four groups of 32 channels, one group per lane of the quad.
+constexpr int kModePlain = 0, kModeGroups = 1, kModeLaneGroups = 2;
+
+template <typename E, int kMode>
 __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
                  E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks, int gpc,
                  GroupArgs ga, const int32_t *__restrict__ lens, int Hkv, uint32_t *__restrict__ status) {
     using Raw = typename RawT<E>::type;
+    constexpr bool kGrouped = kMode != kModePlain, kLane = kMode == kModeLaneGroups;
     // per-warp staging of the kept values: [kept index][8 tokens of the warp]
     __shared__ __align__(16) Raw vtile[kPruneThreads / 32][kD * 8];
     __shared__ double red[2][kPruneThreads / 32];
@@ -384,7 +441,22 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     __shared__ uint32_t gmask[kGrouped ? kMaxGroups : 1][4];
     __shared__ __align__(16) uint32_t gsel[kGrouped ? kMaxGroups : 1][4][16];
     __shared__ int gT[kGrouped ? kMaxGroups : 1];
-    __shared__ uint32_t staus[kGrouped ? kMaxGroups : 1][kPruneThreads];  // per-lane estimates
+    __shared__ uint32_t staus[kMode == kModeGroups ? kMaxGroups : 1][kPruneThreads];  // per-lane estimates
+    // Four groups: each quarter scatters its 16-bit keys into a per-warp
+    // exchange row per token in group order (group q at u16 offset kXGroup *
+    // q, a group's channels in ascending order), and lane s reads group s
+    // back with four 16-byte loads.  Rows 100 words apart put the 8 tokens of
+    // a warp in distinct bank quadruples for the scatter, and groups 24 words
+    // apart keep each 8-lane phase of the 16-byte reads free of conflicts.
+    constexpr int kXGroup = 48, kXRow = 200;  // u16 units
+    __shared__ __align__(16) uint16_t xkeys[kLane ? kPruneThreads / 32 : 1][kLane ? 8 * kXRow : 1];
+    // per lane: the shared address of each of its quarter's 32 channels in
+    // its token's exchange row, [channel / 4][thread] (conflict-free reads)
+    __shared__ __align__(16) uint4 xaddr[kLane ? 8 : 1][kLane ? kPruneThreads : 1];
+    // per quarter: byte selectors that build the threshold pair of kp[i]
+    // (groups of channels i and i + 16) from the four group thresholds
+    __shared__ __align__(16) uint32_t psel[kLane ? 4 : 1][16];
+    __shared__ uint8_t sslot[kLane ? kD : 1];
     if constexpr (kGrouped) {
         const float qj = qs[(tid >> 5) * 36 + (tid & 31)];
         int rank = 0;
@@ -408,11 +480,35 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
             for (int c = 0; c < 32; ++c) b |= (sgid[32 * qs4 + c] == q ? 1u : 0u) << c;
             gmask[q][qs4] = b;
         }
+        if constexpr (kLane) {
+            const int q = sgid[tid];
+            int j = 0;  // rank of this channel among its group's channels
+            for (int i = 0; i < tid; ++i) j += sgid[i] == q ? 1 : 0;
+            sslot[tid] = (uint8_t)(q * kXGroup + j);
+        }
         __syncthreads();
+        if constexpr (kLane) {
+            const uint32_t row = (uint32_t)__cvta_generic_to_shared(&xkeys[warp][(lane >> 2) * kXRow]);
+            const int s4 = lane & 3;
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii) {
+                uint32_t a[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) a[e] = row + 2u * sslot[32 * s4 + 4 * ii + e];
+                xaddr[ii][tid] = make_uint4(a[0], a[1], a[2], a[3]);
+            }
+            if (tid < 64) {
+                const int qs4 = tid >> 4, i = tid & 15;
+                const uint32_t ql = sgid[32 * qs4 + i], qh = sgid[32 * qs4 + i + 16];
+                psel[qs4][i] = (2u * ql) | (2u * ql + 1u) << 4 | (2u * qh) << 8 | (2u * qh + 1u) << 12;
+            }
+            __syncthreads();
+        }
     }
 
     Raw *vt = vtile[warp];
     uint32_t tau = 1u;
+    const uint32_t bsel = own_count_operand(lane);  // four-group mode: per-lane counts
     double acc_w = 0.0, acc_w2 = 0.0;
     const long g_first = (long)chunk * gpc;
     const E *krow = k + ((size_t)bh * S + g_first * 32 + tl) * kD + 32 * s;  // this lane's slice, group 0
@@ -492,6 +588,97 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
             };
             if constexpr (!kGrouped) {
                 m = select_with(kp, T, 0xffffffffu, tau);
+            } else if constexpr (kLane) {
+                // scatter this quarter's 16-bit keys into the token's exchange
+                // row, then read back group s (32 keys, two per word)
+                __syncwarp();
+#pragma unroll
+                for (int ii = 0; ii < 8; ++ii) {
+                    const uint4 a = xaddr[ii][tid];
+                    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 4 * ii + e;
+                        const uint32_t h = c < 16 ? kp[c] : (kp[c - 16] >> 16);
+                        asm volatile("st.shared.u16 [%0], %1;" ::"r"(av[e]), "h"((unsigned short)h) : "memory");
+                    }
+                }
+                __syncwarp();
+                uint32_t kg[16];
+                {
+                    const uint32_t src =
+                        (uint32_t)__cvta_generic_to_shared(&xkeys[warp][tq * kXRow + kXGroup * s]);
+#pragma unroll
+                    for (int i4 = 0; i4 < 4; ++i4)
+                        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                     : "=r"(kg[4 * i4]), "=r"(kg[4 * i4 + 1]), "=r"(kg[4 * i4 + 2]),
+                                       "=r"(kg[4 * i4 + 3])
+                                     : "r"(src + 16u * i4)
+                                     : "memory");
+                }
+                // this lane's group: top Tq of its 32 keys
+                const int Tq = gT[s];
+                const bool triv = Tq <= 0 || Tq >= 32;
+                uint32_t base;
+                int K;
+                if (gi == 0) {
+                    __half2 mx = *reinterpret_cast<const __half2 *>(&kg[0]);
+#pragma unroll
+                    for (int i = 1; i < 16; ++i) mx = __hmax2(mx, *reinterpret_cast<const __half2 *>(&kg[i]));
+                    const uint32_t mb = *reinterpret_cast<const uint32_t *>(&mx);
+                    const uint32_t m16 = max(mb & 0xffffu, mb >> 16);
+                    K = kLiftCold;
+                    base = m16 > (1u << K) - 1u ? m16 - ((1u << K) - 1u) : 0u;
+                } else {
+                    K = kLiftLane;
+                    base = tau > (1u << (K - 1)) ? tau - (1u << (K - 1)) : 0u;
+                }
+                base = min(base, kTop16 - (1u << K));
+                uint32_t lo;
+                bool ex;
+                search_fp16<true>(kg, Tq, base, K, !valid || triv, bsel, lo, ex);
+                if (!triv) tau = gi == 0 ? lo : (uint32_t)((int)tau + (((int)lo - (int)tau) >> 1));
+                tau = valid ? tau : 1u;
+                if (triv) {
+                    lo = Tq <= 0 ? kTop16 : 0u;  // kTop16 is a NaN pattern: no key compares >= it
+                    ex = true;
+                }
+                // the four groups' thresholds (bit 15: boundary inside the fp16
+                // band) to every lane of the quad, then the fp16 decision with
+                // each channel's own group threshold
+                const uint32_t v = lo | (ex ? 0u : 0x8000u);
+                const uint32_t w1 = __shfl_xor_sync(0xffffffffu, v, 1);
+                const uint32_t pr = (s & 1) ? (w1 | (v << 16)) : (v | (w1 << 16));
+                const uint32_t ot = __shfl_xor_sync(0xffffffffu, pr, 2);
+                const uint32_t P01 = (s & 2) ? ot : pr, P23 = (s & 2) ? pr : ot;
+                const uint32_t T01 = P01 & 0x7fff7fffu, T23 = P23 & 0x7fff7fffu;
+                uint32_t p2[16];
+                {
+                    const uint4 *ps = reinterpret_cast<const uint4 *>(psel[s]);
+#pragma unroll
+                    for (int i4 = 0; i4 < 4; ++i4) {
+                        const uint4 sv = ps[i4];
+                        p2[4 * i4 + 0] = __byte_perm(T01, T23, sv.x);
+                        p2[4 * i4 + 1] = __byte_perm(T01, T23, sv.y);
+                        p2[4 * i4 + 2] = __byte_perm(T01, T23, sv.z);
+                        p2[4 * i4 + 3] = __byte_perm(T01, T23, sv.w);
+                    }
+                }
+                m = decide_fp16(kp, p2);
+                // exact fp32 phase for the groups whose fp16 band holds the
+                // boundary, on the quad's channels of that group
+                const uint32_t nex =
+                    ((P01 >> 15) & 1u) | ((P01 >> 30) & 2u) | ((P23 >> 13) & 4u) | ((P23 >> 28) & 8u);
+                const uint32_t any_nex = __reduce_or_sync(0xffffffffu, nex);
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    if (!((any_nex >> q) & 1u)) continue;  // warp-uniform
+                    const uint32_t gm = gmask[q][s];
+                    const uint32_t lq = ((q < 2 ? T01 : T23) >> (16 * (q & 1))) & 0xffffu;
+                    const uint32_t mq = refine_fp32(key, gT[q], s, inv_scale, lq, !((nex >> q) & 1u), gm, m & gm);
+                    m = (m & ~gm) | mq;
+                }
+                m = valid ? m : 0u;
             } else {
                 m = 0u;
 #pragma unroll 1
@@ -559,11 +746,22 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     KSlice<E> ka, kb;
     if (g_first * 32 + tl < Sb) ka.load(krow);
     else ka.zero();
-    for (int gi = 0; gi < gpc; gi += 2) {
-        if ((g_first + gi) * 32 >= Sb) break;  // uniform across the CTA
-        group(gi, ka, kb);
-        if ((g_first + gi + 1) * 32 >= Sb) break;
-        group(gi + 1, kb, ka);
+    if constexpr (kLane) {
+        // one call site: the four-group body is large enough that a second
+        // inlined copy no longer fits the instruction cache
+#pragma unroll 1
+        for (int gi = 0; gi < gpc; ++gi) {
+            if ((g_first + gi) * 32 >= Sb) break;  // uniform across the CTA
+            group(gi, ka, kb);
+            ka = kb;
+        }
+    } else {
+        for (int gi = 0; gi < gpc; gi += 2) {
+            if ((g_first + gi) * 32 >= Sb) break;  // uniform across the CTA
+            group(gi, ka, kb);
+            if ((g_first + gi + 1) * 32 >= Sb) break;
+            group(gi + 1, kb, ka);
+        }
     }
 
     // fixed-order reduction: xor tree inside each warp, then warps in order
@@ -624,12 +822,16 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
     const int gpc = prune_groups_per_cta(BH, kc.S);
     const int nch = prune_chunks(kc.S, gpc);
     if (nch > 0) {
-        if (ga)
-            prune_kernel<E, true><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+        if (ga && ga->n == 4 && kD == 128)
+            prune_kernel<E, kModeLaneGroups><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+                static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
+                nch, gpc, *ga, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
+        else if (ga)
+            prune_kernel<E, kModeGroups><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
                 nch, gpc, *ga, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
         else
-            prune_kernel<E, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+            prune_kernel<E, kModePlain><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
                 nch, gpc, GroupArgs{}, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
     }
@@ -666,11 +868,11 @@ cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws,
     const int nch = prune_chunks(vc.S, gpc);
     if (nch > 0) {
         if (vc.dtype == SPARK_BF16)
-            prune_kernel<__nv_bfloat16, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+            prune_kernel<__nv_bfloat16, kModePlain><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16 *>(v), vc.qn, vc.mask, static_cast<__nv_bfloat16 *>(vc.vals),
                 partial, vc.S, vc.T, nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws));
         else
-            prune_kernel<float, false><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
+            prune_kernel<float, kModePlain><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const float *>(v), vc.qn, vc.mask, static_cast<float *>(vc.vals), partial, vc.S, vc.T,
                 nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws));
     }

@@ -102,6 +102,20 @@ def test_grouped_extremes(k_exp, spread):
         check_grouped(kc, to_np(k), to_np(q_obs), G, Tg, f"extremes k2^{k_exp} spread {spread} g={len(Tg)}")
 
 
+@pytest.mark.parametrize("rates", [[0.0, 0.03, 0.97, 1.0], [0.5, 0.5, 0.5, 0.5], [0.97, 0.97, 0.97, 0.97],
+                                   [0.03, 0.1, 0.2, 0.3], [1.0, 1.0, 1.0, 0.0], [0.0, 0.0, 0.0, 0.0]])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_grouped_four_groups_budgets(rates, dtype):
+    # four groups of 32 channels (one per lane of a quad): budgets from 0 to
+    # 32 per group, over several 32-token groups and a ragged tail
+    wl = scaled(WORKLOADS["tiny"], S=2083, dtype="f32" if dtype == torch.float32 else "bf16", Hkv=2,
+                seed=int(sum(rates) * 100))
+    pre = make_prefill(wl, DEV)
+    Tg = spark_group_budget(D, rates)
+    kc = run_grouped(pre["k"], pre["q_obs"], wl.G, wl.W, Tg)
+    check_grouped(kc, to_np(pre["k"]), to_np(pre["q_obs"]), wl.G, Tg, f"four groups {Tg}")
+
+
 def test_grouped_ties_integer_keys():
     # integer keys and window queries: exact saliency ties everywhere, and
     # equal window-query norms across group boundaries
