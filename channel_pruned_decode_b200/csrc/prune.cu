@@ -140,6 +140,13 @@ __device__ __forceinline__ uint32_t hge2_mask(uint32_t a, uint32_t b) {
     return d;
 }
 
+// fp16x2 a == b per half: 0xffff / 0x0000.
+__device__ __forceinline__ uint32_t heq2_mask(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("set.eq.u32.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // D += A * B for one m16n8k16 fp16 tile with fp16 accumulators.
 __device__ __forceinline__ void mma_f16(uint32_t &d0, uint32_t &d1, uint32_t a0, uint32_t a1, uint32_t a2,
                                         uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -263,15 +270,76 @@ __device__ __forceinline__ void search_fp16(const uint32_t (&kp)[16], int T, uin
     exact_out = exact;
 }
 
+constexpr int kBandPicks = 4;  // most one-at-a-time picks from an fp16 band before bisecting instead
+
 // Phase 2: the mask word (32 channels of this lane's quarter) of the T
 // largest exact fp32 keys among the quad's channels of gm (bit i = channel i
 // of this lane's quarter takes part), ties to the lower channel index, given
 // the phase-1 result: m16 = the channels of gm whose fp16 key is >= lo, which
 // is the answer when `exact`; otherwise count(fp16 >= lo) >= T > count(fp16
-// >= lo + 1).  Warp-uniform: every lane of the warp calls it.
-__device__ __forceinline__ uint32_t refine_fp32(const uint32_t (&key)[32], int T, int s, float inv_scale,
-                                                uint32_t lo, bool exact, uint32_t gm, uint32_t m16) {
+// >= lo + 1).  kp holds the 16-bit keys (channels i and i + 16 in kp[i]).
+// Warp-uniform: every lane of the warp calls it.
+//
+// The fp16 rounding is monotone, so the A keys with an fp16 key above lo are
+// all kept and the boundary lies in the band of nb keys whose fp16 key is
+// lo: of these the r = T - A largest (equal keys: lower channel first) are
+// kept.  Usually the band holds two or three keys, so the kernel picks the r
+// largest one at a time when r <= nb - r, or drops the nb - r smallest (equal
+// keys: higher channel first) otherwise, each pick a quad max or min and a
+// lowest-channel search.  A wider band, more than kBandPicks picks in any
+// quad of the warp, takes a bisection over the fp32 bit patterns instead.
+__device__ __forceinline__ uint32_t refine_fp32(const uint32_t (&key)[32], const uint32_t (&kp)[16], int T,
+                                                int s, float inv_scale, uint32_t lo, bool exact, uint32_t gm,
+                                                uint32_t m16) {
     if (!__any_sync(0xffffffffu, !exact)) return m16;
+    {
+        uint32_t band = 0u;
+        const uint32_t lo2 = lo * 0x10001u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) band |= heq2_mask(kp[i], lo2) & (0x00010001u << i);
+        band = exact ? 0u : band & gm;
+        const int above = quad_sum(__popc(m16 & ~band));
+        const int nb = quad_sum(__popc(band));
+        const int r = T - above;  // 0 < r < nb unless exact
+        const bool pmax = 2 * r <= nb;
+        const int take = exact ? 0 : (pmax ? r : nb - r);
+        const int most = __reduce_max_sync(0xffffffffu, take);
+        if (most <= kBandPicks) {
+            uint32_t cand = band, picked = 0u;
+            for (int it = 0; it < most; ++it) {
+                uint32_t mx = 0u, mn = 0xffffffffu;  // keys are non-negative: u32 order is fp32 order
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    if ((cand >> i) & 1u) {
+                        mx = max(mx, key[i]);
+                        mn = min(mn, key[i]);
+                    }
+                }
+#pragma unroll
+                for (int o = 1; o <= 2; o <<= 1) {
+                    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                }
+                const uint32_t ext = pmax ? mx : mn;
+                uint32_t eqm = 0u;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) eqm |= (key[i] == ext ? 1u : 0u) << i;
+                eqm = it < take ? eqm & cand : 0u;
+                // the pick: lowest channel of the quad for a max, highest for a min
+                const int order = pmax ? s : 3 - s;
+                int first = eqm ? order : 4;
+                first = min(first, __shfl_xor_sync(0xffffffffu, first, 1));
+                first = min(first, __shfl_xor_sync(0xffffffffu, first, 2));
+                if (eqm && order == first) {
+                    const uint32_t bit = pmax ? (eqm & (0u - eqm)) : (0x80000000u >> __clz(eqm));
+                    picked |= bit;
+                    cand &= ~bit;
+                }
+            }
+            if (exact) return m16;
+            return pmax ? ((m16 & ~band) | picked) : (m16 & ~picked);
+        }
+    }
     const uint32_t hi = lo + 1u;
 
     // With v = the fp16 value of lo - 1 and u that of hi = lo + 1, every key
@@ -371,7 +439,7 @@ __device__ __forceinline__ uint32_t select_top_t(const uint32_t (&key)[32], cons
     uint32_t p2[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) p2[i] = lo * 0x10001u;
-    return refine_fp32(key, T, s, inv_scale, lo, exact, gm, decide_fp16(kp, p2));
+    return refine_fp32(key, kp, T, s, inv_scale, lo, exact, gm, decide_fp16(kp, p2));
 }
 
 // SparK-g groups: number of groups and each group's kept-channel budget.
@@ -675,7 +743,7 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
                     if (!((any_nex >> q) & 1u)) continue;  // warp-uniform
                     const uint32_t gm = gmask[q][s];
                     const uint32_t lq = ((q < 2 ? T01 : T23) >> (16 * (q & 1))) & 0xffffu;
-                    const uint32_t mq = refine_fp32(key, gT[q], s, inv_scale, lq, !((nex >> q) & 1u), gm, m & gm);
+                    const uint32_t mq = refine_fp32(key, kp, gT[q], s, inv_scale, lq, !((nex >> q) & 1u), gm, m & gm);
                     m = (m & ~gm) | mq;
                 }
                 m = valid ? m : 0u;
