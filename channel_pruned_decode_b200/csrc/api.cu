@@ -105,7 +105,7 @@ size_t spark_cache_bytes(int B, int Hkv, int S, int D, int T, int dtype) {
 size_t spark_workspace_bytes(int op, int B, int Hkv, int G, int S, int D, int T, int n_tail) {
     if (B < 0 || Hkv < 0 || S < 0 || D != kD || T < 0 || T > D || G < 1 || n_tail < 0) return 0;
     const long BH = (long)B * Hkv;
-    if (op == SPARK_OP_PRUNE) return round256(prune_workspace(BH, S));
+    if (op == SPARK_OP_PRUNE) return round256(prune_grouped_workspace(BH, S));  // also spark_prune_grouped
     if (op == SPARK_OP_SNAPKV) return round256(snapkv_workspace(BH, S, 0));
     if (op == SPARK_OP_THINK) return round256(think_workspace(BH, S));
     if (op == SPARK_OP_TOPP) return round256(topp_workspace(BH, S));
@@ -162,7 +162,7 @@ int spark_prune_grouped(const void *k, const void *q_obs, int G, int W, int n_gr
     if (!q_obs || !aligned16(q_obs)) return SPARK_ERR_ARG;
     if (out->S > 0 && (!k || !aligned16(k))) return SPARK_ERR_ARG;
     if (!workspace || !aligned16(workspace)) return SPARK_ERR_WORKSPACE;
-    if (ws_bytes < prune_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
+    if (ws_bytes < prune_grouped_workspace(BH, out->S)) return SPARK_ERR_WORKSPACE;
     cudaError_t e = launch_prune_grouped(k, q_obs, G, W, n_groups, group_T, *out, workspace,
                                          static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SPARK_OK : SPARK_ERR_CUDA;

@@ -41,9 +41,112 @@
 
 namespace spark {
 
+// Four-group key exchange rows (u16 units): group q's 32 keys at kXGroup * q,
+// one row per token, rows kXRow apart.  Rows 100 words apart put the 8 tokens
+// of a warp in distinct bank quadruples, and groups 24 words apart keep each
+// 8-lane phase of the 16-byte reads back free of bank conflicts.
+constexpr int kXGroup = 48, kXRow = 200;
+
+// Four-group SparK-g: where each channel's key goes in the exchange row, per
+// (row, kv head), from the head's window-query norms; the groups are those of the other modes (rank by
+// qn desc, channel asc; group q holds the ranks [32q, 32q + 32)), and a
+// channel's slot is kXGroup * group + j with j < 32.  Step c of the scatter
+// writes channels c, 32 + c, 64 + c and 96 + c of the warp's 8 tokens; with
+// the row stride above it is free of bank conflicts exactly when those four
+// channels' words j / 2 differ mod 4 (call j / 2 mod 4 the slot's colour:
+// each group has 8 slots of each colour).  Colour = quarter c / 32 makes
+// every step conflict-free but may give a group more than 8 channels of a
+// colour; swaps of two channels' colours within one step (still distinct)
+// then even the groups out, each time the swap that lowers the total excess
+// most (first by step, then by pair).  Channels take their colour's slots in
+// channel order, and whatever excess is left takes the free slots.  Only the
+// bank pattern of the exchange depends on this order, not the result.
+// Called by all kD threads of a CTA, thread c holding channel c's norm in
+// q[c] (shared); writes the head's kD slots to `out`.
+__device__ __forceinline__ void build_group_slots(const float *q, uint8_t *__restrict__ out) {
+    __shared__ uint8_t gid[kD], col[kD], slot[kD];
+    __shared__ int cnt[4][4];
+    const int c = threadIdx.x;
+    if (c < 16) cnt[c >> 2][c & 3] = 0;
+    __syncthreads();
+    {
+        const float qc = q[c];
+        int rank = 0;
+        for (int i = 0; i < kD; ++i) rank += (q[i] > qc || (q[i] == qc && i < c)) ? 1 : 0;
+        gid[c] = (uint8_t)(rank >> 5);
+        col[c] = (uint8_t)(c >> 5);
+        atomicAdd(&cnt[rank >> 5][c >> 5], 1);
+    }
+    __syncthreads();
+    if (c < 32) {  // warp 0 orders the slots (warp-uniform branch); lane = step
+        const int lane = c;
+        for (int it = 0; it < 64; ++it) {
+            int best = 0, bx = 0, by = 0;
+            for (int a = 0; a < 4; ++a)
+                for (int b = a + 1; b < 4; ++b) {
+                    const int x = 32 * a + lane, y = 32 * b + lane;
+                    const int gx = gid[x], gy = gid[y], cx = col[x], cy = col[y];
+                    if (gx == gy) continue;  // same group: the counts do not change
+                    const int before = abs(cnt[gx][cx] - 8) + abs(cnt[gx][cy] - 8) + abs(cnt[gy][cy] - 8) +
+                                       abs(cnt[gy][cx] - 8);
+                    const int after = abs(cnt[gx][cx] - 9) + abs(cnt[gx][cy] - 7) + abs(cnt[gy][cy] - 9) +
+                                      abs(cnt[gy][cx] - 7);
+                    if (before - after > best) {
+                        best = before - after;
+                        bx = x;
+                        by = y;
+                    }
+                }
+            const int key = __reduce_max_sync(0xffffffffu, (best << 8) | (255 - lane));
+            if ((key >> 8) <= 0) break;  // warp-uniform
+            if (lane == 255 - (key & 255)) {
+                const int gx = gid[bx], gy = gid[by], cx = col[bx], cy = col[by];
+                --cnt[gx][cx];
+                ++cnt[gx][cy];
+                --cnt[gy][cy];
+                ++cnt[gy][cx];
+                col[bx] = (uint8_t)cy;
+                col[by] = (uint8_t)cx;
+            }
+            __syncwarp();
+        }
+        if (lane < 4) {
+            const int g = lane;
+            uint32_t used = 0u;
+            int next[4] = {0, 0, 0, 0};
+            for (int ch = 0; ch < kD; ++ch) {
+                if (gid[ch] != g) continue;
+                const int k = col[ch];
+                if (next[k] < 8) {
+                    const int i = next[k]++;
+                    const int j = 2 * k + (i & 1) + 8 * (i >> 1);  // the slots of colour k
+                    used |= 1u << j;
+                    slot[ch] = (uint8_t)(kXGroup * g + j);
+                } else {
+                    slot[ch] = 0xffu;
+                }
+            }
+            for (int ch = 0; ch < kD; ++ch) {
+                if (gid[ch] != g || slot[ch] != 0xffu) continue;
+                // a group has 32 channels, so a slot is free; NaN norms can
+                // break the ranks, and such a group's extra channels share
+                // slot 31 (the masks are then unspecified, but every slot
+                // stays in its row)
+                const int j = used == 0xffffffffu ? 31 : __ffs(~used) - 1;
+                used |= 1u << j;
+                slot[ch] = (uint8_t)(kXGroup * g + j);
+            }
+        }
+    }
+    __syncthreads();
+    out[c] = slot[c];
+}
+
+// With slots (four-group SparK-g) it also writes the head's exchange slots.
 template <typename E>
 __global__ void __launch_bounds__(kD) qnorm_kernel(const E *__restrict__ q_obs, int G, int W,
-                                                   float *__restrict__ qn) {
+                                                   float *__restrict__ qn, uint8_t *__restrict__ slots) {
+    __shared__ float qsh[kD];
     const long bh = blockIdx.x;
     const int j = threadIdx.x;
     const E *base = q_obs + (size_t)bh * G * W * kD + j;
@@ -53,7 +156,12 @@ __global__ void __launch_bounds__(kD) qnorm_kernel(const E *__restrict__ q_obs, 
             const double x = (double)Elem<E>::to_f(base[((size_t)g * W + t) * kD]);
             acc = __dadd_rn(acc, __dmul_rn(x, x));  // square of an fp32 value is exact in fp64
         }
-    qn[bh * kD + j] = __double2float_rn(sqrt(acc));
+    const float q = __double2float_rn(sqrt(acc));
+    qn[bh * kD + j] = q;
+    if (slots) {  // uniform across the CTA
+        qsh[j] = q;
+        build_group_slots(qsh, slots + bh * kD);
+    }
 }
 
 // Per-lane view of 32 consecutive channels of one key row.
@@ -457,7 +565,8 @@ template <typename E, int kMode>
 __global__ void __launch_bounds__(kPruneThreads, 4)
     prune_kernel(const E *__restrict__ k, const float *__restrict__ qn, uint32_t *__restrict__ mask,
                  E *__restrict__ vals, double *__restrict__ partial, int S, int T, int n_chunks, int gpc,
-                 GroupArgs ga, const int32_t *__restrict__ lens, int Hkv, uint32_t *__restrict__ status) {
+                 GroupArgs ga, const int32_t *__restrict__ lens, int Hkv, uint32_t *__restrict__ status,
+                 const uint8_t *__restrict__ slots) {
     using Raw = typename RawT<E>::type;
     constexpr bool kGrouped = kMode != kModePlain, kLane = kMode == kModeLaneGroups;
     // per-warp staging of the kept values: [kept index][8 tokens of the warp]
@@ -507,16 +616,12 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     // group's halves of the packed 16-bit keys.
     __shared__ uint8_t sgid[kGrouped ? kD : 1];
     __shared__ uint32_t gmask[kGrouped ? kMaxGroups : 1][4];
-    __shared__ __align__(16) uint32_t gsel[kGrouped ? kMaxGroups : 1][4][16];
+    __shared__ __align__(16) uint32_t gsel[kMode == kModeGroups ? kMaxGroups : 1][4][16];
     __shared__ int gT[kGrouped ? kMaxGroups : 1];
     __shared__ uint32_t staus[kMode == kModeGroups ? kMaxGroups : 1][kPruneThreads];  // per-lane estimates
     // Four groups: each quarter scatters its 16-bit keys into a per-warp
-    // exchange row per token in group order (group q at u16 offset kXGroup *
-    // q, a group's channels in ascending order), and lane s reads group s
-    // back with four 16-byte loads.  Rows 100 words apart put the 8 tokens of
-    // a warp in distinct bank quadruples for the scatter, and groups 24 words
-    // apart keep each 8-lane phase of the 16-byte reads free of conflicts.
-    constexpr int kXGroup = 48, kXRow = 200;  // u16 units
+    // exchange row per token in group order (the slots of build_group_slots),
+    // and lane s reads group s back with four 16-byte loads.
     __shared__ __align__(16) uint16_t xkeys[kLane ? kPruneThreads / 32 : 1][kLane ? 8 * kXRow : 1];
     // per lane: the shared address of each of its quarter's 32 channels in
     // its token's exchange row, [channel / 4][thread] (conflict-free reads)
@@ -526,33 +631,35 @@ __global__ void __launch_bounds__(kPruneThreads, 4)
     __shared__ __align__(16) uint32_t psel[kLane ? 4 : 1][16];
     __shared__ uint8_t sslot[kLane ? kD : 1];
     if constexpr (kGrouped) {
-        const float qj = qs[(tid >> 5) * 36 + (tid & 31)];
-        int rank = 0;
-        for (int i = 0; i < kD; ++i) {
-            const float qi = qs[(i >> 5) * 36 + (i & 31)];
-            rank += (qi > qj || (qi == qj && i < tid)) ? 1 : 0;
+        if constexpr (kLane) {
+            const uint8_t sl = __ldg(slots + bh * kD + tid);
+            sslot[tid] = sl;
+            sgid[tid] = (uint8_t)(sl / kXGroup);
+        } else {
+            const float qj = qs[(tid >> 5) * 36 + (tid & 31)];
+            int rank = 0;
+            for (int i = 0; i < kD; ++i) {
+                const float qi = qs[(i >> 5) * 36 + (i & 31)];
+                rank += (qi > qj || (qi == qj && i < tid)) ? 1 : 0;
+            }
+            int gq = 0;
+            for (int q = 1; q < ga.n; ++q) gq += rank >= q * kD / ga.n ? 1 : 0;
+            sgid[tid] = (uint8_t)gq;
         }
-        int gq = 0;
-        for (int q = 1; q < ga.n; ++q) gq += rank >= q * kD / ga.n ? 1 : 0;
-        sgid[tid] = (uint8_t)gq;
         if (tid < kMaxGroups) gT[tid] = tid < ga.n ? ga.T[tid] : 0;
         __syncthreads();
-        for (int e = tid; e < ga.n * 64; e += kPruneThreads) {
-            const int q = e >> 6, qs4 = (e >> 4) & 3, i = e & 15;
-            gsel[q][qs4][i] = (sgid[32 * qs4 + i] == q ? 0x0000ffffu : 0u) |
-                              (sgid[32 * qs4 + i + 16] == q ? 0xffff0000u : 0u);
+        if constexpr (!kLane) {
+            for (int e = tid; e < ga.n * 64; e += kPruneThreads) {
+                const int q = e >> 6, qs4 = (e >> 4) & 3, i = e & 15;
+                gsel[q][qs4][i] = (sgid[32 * qs4 + i] == q ? 0x0000ffffu : 0u) |
+                                  (sgid[32 * qs4 + i + 16] == q ? 0xffff0000u : 0u);
+            }
         }
         if (tid < ga.n * 4) {
             const int q = tid >> 2, qs4 = tid & 3;
             uint32_t b = 0u;
             for (int c = 0; c < 32; ++c) b |= (sgid[32 * qs4 + c] == q ? 1u : 0u) << c;
             gmask[q][qs4] = b;
-        }
-        if constexpr (kLane) {
-            const int q = sgid[tid];
-            int j = 0;  // rank of this channel among its group's channels
-            for (int i = 0; i < tid; ++i) j += sgid[i] == q ? 1 : 0;
-            sslot[tid] = (uint8_t)(q * kXGroup + j);
         }
         __syncthreads();
         if constexpr (kLane) {
@@ -886,22 +993,24 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
     const long BH = (long)kc.B * kc.Hkv;
     if (BH == 0) return cudaSuccess;
     double *partial = reinterpret_cast<double *>(static_cast<char *>(ws) + kWsHeader);
-    qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn);
+    const bool lane_groups = ga && ga->n == 4 && kD == 128;
+    uint8_t *slots = lane_groups ? static_cast<uint8_t *>(ws) + prune_slots_offset(BH, kc.S) : nullptr;
+    qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn, slots);
     const int gpc = prune_groups_per_cta(BH, kc.S);
     const int nch = prune_chunks(kc.S, gpc);
     if (nch > 0) {
-        if (ga && ga->n == 4 && kD == 128)
+        if (lane_groups) {
             prune_kernel<E, kModeLaneGroups><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-                nch, gpc, *ga, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
-        else if (ga)
+                nch, gpc, *ga, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws), slots);
+        } else if (ga)
             prune_kernel<E, kModeGroups><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-                nch, gpc, *ga, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
+                nch, gpc, *ga, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws), nullptr);
         else
             prune_kernel<E, kModePlain><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const E *>(k), kc.qn, kc.mask, static_cast<E *>(kc.vals), partial, kc.S, kc.T,
-                nch, gpc, GroupArgs{}, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws));
+                nch, gpc, GroupArgs{}, kc.lens, kc.Hkv, static_cast<uint32_t *>(ws), nullptr);
     }
     stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, kc.S, kc.T, kc.stats, kc.lens,
                                                            kc.Hkv);
@@ -911,9 +1020,9 @@ static cudaError_t launch_prune_t(const void *k, const void *q_obs, int G, int W
 cudaError_t launch_qnorm(const void *q_obs, int G, int W, long BH, int dtype, float *qn, cudaStream_t st) {
     if (BH == 0) return cudaSuccess;
     if (dtype == SPARK_BF16)
-        qnorm_kernel<__nv_bfloat16><<<(unsigned)BH, kD, 0, st>>>(static_cast<const __nv_bfloat16 *>(q_obs), G, W, qn);
+        qnorm_kernel<__nv_bfloat16><<<(unsigned)BH, kD, 0, st>>>(static_cast<const __nv_bfloat16 *>(q_obs), G, W, qn, nullptr);
     else
-        qnorm_kernel<float><<<(unsigned)BH, kD, 0, st>>>(static_cast<const float *>(q_obs), G, W, qn);
+        qnorm_kernel<float><<<(unsigned)BH, kD, 0, st>>>(static_cast<const float *>(q_obs), G, W, qn, nullptr);
     return cudaGetLastError();
 }
 
@@ -938,11 +1047,11 @@ cudaError_t launch_prune_values(const void *v, const spark_kcache &vc, void *ws,
         if (vc.dtype == SPARK_BF16)
             prune_kernel<__nv_bfloat16, kModePlain><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16 *>(v), vc.qn, vc.mask, static_cast<__nv_bfloat16 *>(vc.vals),
-                partial, vc.S, vc.T, nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws));
+                partial, vc.S, vc.T, nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws), nullptr);
         else
             prune_kernel<float, kModePlain><<<(unsigned)(BH * nch), kPruneThreads, 0, st>>>(
                 static_cast<const float *>(v), vc.qn, vc.mask, static_cast<float *>(vc.vals), partial, vc.S, vc.T,
-                nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws));
+                nch, gpc, GroupArgs{}, vc.lens, vc.Hkv, static_cast<uint32_t *>(ws), nullptr);
     }
     stats_kernel<<<(unsigned)((BH + 3) / 4), 128, 0, st>>>(partial, nch, BH, vc.S, vc.T, vc.stats, vc.lens,
                                                            vc.Hkv);
@@ -1507,7 +1616,7 @@ static cudaError_t launch_prune_topp_t(const void *k, const void *q_obs, int G, 
     if (BH == 0) return cudaSuccess;
     const long ng = ((long)kc.S + 31) / 32;
     const ToppWs tw = topp_ws_layout(ws, BH, kc.S);
-    qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn);
+    qnorm_kernel<E><<<(unsigned)BH, kD, 0, st>>>(static_cast<const E *>(q_obs), G, W, kc.qn, nullptr);
     const int gpc = prune_groups_per_cta(BH, kc.S);
     const int nch = prune_chunks(kc.S, gpc);
     if (ng > 0) {

@@ -78,6 +78,11 @@ inline size_t prune_workspace(long BH, int S) {
     return kWsHeader + (size_t)BH * (size_t)prune_chunks(S) * 2 * sizeof(double);
 }
 
+// SparK-g with four groups also keeps one byte per channel and head (the
+// channels' slots in the key exchange) after the partials
+inline size_t prune_slots_offset(long BH, int S) { return (prune_workspace(BH, S) + 255) / 256 * 256; }
+inline size_t prune_grouped_workspace(long BH, int S) { return prune_slots_offset(BH, S) + (size_t)BH * kD; }
+
 // SparK-p workspace: the prune partials with a third one per chunk (the
 // data-dependent pruned count), then per group the largest kept count, then
 // per head its rows and its first row (the value layout's scan)
