@@ -1082,7 +1082,11 @@ cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W,
 //
 // A set {16-bit key >= P} is a threshold set of the exact keys (the 16-bit
 // key is monotone in them), hence a greedy prefix, and its mass M(P) does
-// not increase with P (each rounding is monotone).  The search finds the
+// not increase with P.  The search uses the masses of the 16-bit keys
+// themselves (count_mass_ge16, on the tensor cores) against p times their
+// total; they are within fp16 rounding of the exact masses, so the search
+// may stop a channel off the exact boundary, and the fp64 step after it moves
+// the boundary from any greedy prefix.  The search finds the
 // largest level lo with M(lo) >= target by binary lifting, tracking the
 // lowest failing level hi: over [0, 2^15) for the first token of a quad
 // (M(0) is the total, nothing reaches 2^15), otherwise over a 2^11-level
@@ -1090,8 +1094,8 @@ cudaError_t launch_prune_grouped(const void *k, const void *q_obs, int G, int W,
 // did not bracket lo.  It leaves early once {key >= lo} and {key >= hi}
 // differ by one channel for every quad of the warp: that channel ends the
 // prefix.  Otherwise the band between them is added one channel at a time
-// in greedy order (exact keys desc, lower channel first) until the mass
-// reaches the target.  A prefix longer than Tcap is replaced by the top-Tcap
+// in greedy order (exact keys desc, lower channel first) until the exact
+// fp32 mass reaches the exact fp32 target.  A prefix longer than Tcap is replaced by the top-Tcap
 // set (select_top_t).
 
 // this lane's channels whose 16-bit key is >= P (bit i = channel i)
@@ -1112,6 +1116,42 @@ __device__ __forceinline__ float quad_mass(const uint32_t (&key)[32], uint32_t m
     return __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
 }
 
+// D += A * B for one m16n8k16 tile, fp16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_f32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Count and mass of the quad's 16-bit keys >= the probe p2, on the tensor
+// cores (the layout of count_ge16): the 0/1 compare results count the keys
+// in fp16, and the keys times those results (the keys of the set, exact) are
+// summed with fp32 accumulators.  The mass is that of the fp16 keys, within
+// fp16 rounding of the exact scaled mass; every lane of the quad receives
+// both.
+__device__ __forceinline__ void count_mass_ge16(const uint32_t (&kp)[16], uint32_t p2, int &cnt, float &mass) {
+    uint32_t c0 = 0u, c1 = 0u;
+    float f[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        uint32_t a[4], w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            a[e] = hge2_one(kp[4 * m + e], p2);
+            const __half2 x = __hmul2(*reinterpret_cast<const __half2 *>(&a[e]),
+                                      *reinterpret_cast<const __half2 *>(&kp[4 * m + e]));
+            w[e] = *reinterpret_cast<const uint32_t *>(&x);
+        }
+        mma_f16(c0, c1, a[0], a[1], a[2], a[3], kOne2, kOne2);
+        mma_f16_f32(f, w[0], w[1], w[2], w[3], kOne2, kOne2);
+    }
+    const __half2 c = __hadd2(*reinterpret_cast<const __half2 *>(&c0), *reinterpret_cast<const __half2 *>(&c1));
+    cnt = __half2int_rn(__low2half(c));
+    mass = __fadd_rn(f[0], f[2]);  // rows r and r + 8: the token's two halves
+}
+
 // search state of one quad: M(lo) >= target > M(hi) once both are known
 struct TopPBracket {
     uint32_t lo, hi;
@@ -1119,17 +1159,18 @@ struct TopPBracket {
     bool klo, khi;   // lo / hi established by a probe (or known bounds)
 };
 
-// Binary lifting of lo over [lo, lo + 2^K) for the active quads; every loop
-// trip is warp-uniform (the shuffles of quad_sum / quad_mass see all lanes).
-__device__ __forceinline__ void topp_lift(const uint32_t (&key)[32], const uint32_t (&kp)[16], float target,
-                                          int K, bool active, TopPBracket &b) {
+// Binary lifting of lo over [lo, lo + 2^K) for the active quads on the
+// fp16-key masses (target: p times the fp16-key total); every loop trip is
+// warp-uniform (the tensor-core counts see all lanes).
+__device__ __forceinline__ void topp_lift(const uint32_t (&kp)[16], float target, int K, bool active,
+                                          TopPBracket &b) {
     bool done = !active || (b.klo && b.khi && b.clo - b.chi <= 1);
     for (int bit = K - 1; bit >= 0; --bit) {
         if (__all_sync(0xffffffffu, done)) break;
         const uint32_t P = b.lo + (1u << bit);
-        const uint32_t m = ge16_bits(kp, P);
-        const int c = quad_sum(__popc(m));
-        const float M = quad_mass(key, m);
+        int c;
+        float M;
+        count_mass_ge16(kp, P * 0x10001u, c, M);
         if (!done) {
             if (M >= target) {
                 b.lo = P;
@@ -1228,10 +1269,20 @@ __global__ void __launch_bounds__(kPruneThreads, 3)
         }
 
         // target = p * total; a token with target 0 (p = 0 or no saliency)
-        // keeps nothing
+        // keeps nothing.  The search runs on the fp16 keys' masses (target16
+        // from their total); the band walk and the fp64 decision below use
+        // the exact keys, and the fp64 step moves the boundary to its exact
+        // place from wherever the search put it.
         const float total = quad_mass(key, 0xffffffffu);
         const float target = __fmul_rn(p, total);
         const bool active = valid && target > 0.f && Tcap > 0;
+        float target16;
+        {
+            int c_all;
+            float m_all;
+            count_mass_ge16(kp, 0u, c_all, m_all);
+            target16 = __fmul_rn(p, m_all);
+        }
 
         TopPBracket b;
         if (gi == 0) {
@@ -1243,11 +1294,11 @@ __global__ void __launch_bounds__(kPruneThreads, 3)
             b.chi = 0;
             b.klo = b.khi = false;
         }
-        topp_lift(key, kp, target, gi == 0 ? 15 : 11, active, b);
+        topp_lift(kp, target16, gi == 0 ? 15 : 11, active, b);
         const bool suspect = active && !(b.klo && b.khi);
         if (__any_sync(0xffffffffu, suspect)) {
             if (suspect) topp_full_range(b);
-            topp_lift(key, kp, target, 15, suspect, b);
+            topp_lift(kp, target16, 15, suspect, b);
         }
 
         uint32_t m = active ? ge16_bits(kp, b.lo) : 0u;
@@ -1394,14 +1445,16 @@ __global__ void __launch_bounds__(kPruneThreads, 3)
         }
     };
 
+    // one call site: a second inlined copy of the group body does not fit
+    // the instruction cache
     KSlice<E> ka, kb;
     if (g_first * 32 + tl < S) ka.load(krow);
     else ka.zero();
-    for (int gi = 0; gi < gpc; gi += 2) {
-        if ((g_first + gi) * 32 >= S) break;
+#pragma unroll 1
+    for (int gi = 0; gi < gpc; ++gi) {
+        if ((g_first + gi) * 32 >= S) break;  // uniform across the CTA
         group(gi, ka, kb);
-        if ((g_first + gi + 1) * 32 >= S) break;
-        group(gi + 1, kb, ka);
+        ka = kb;
     }
 
 #pragma unroll
@@ -1547,12 +1600,29 @@ __global__ void __launch_bounds__(kScanThreads) topp_goff_kernel(const uint32_t 
 // the mask bits from the top channel down -- or 0 past the token's count.
 constexpr int kGatherWarps = 4;
 
+// shared memory of one gather warp: 32 key rows at a stride of one row + 16
+// bytes (each lane's bulk copy lands 4 banks further on, so lanes reading
+// the same channel meet at most 4 to a bank instead of all 32), then the
+// group's value slots in their output layout, [slot][32 tokens]
+template <typename E> __host__ __device__ constexpr int gather_row_stride() { return kD * (int)sizeof(E) + 16; }
+template <typename E> __host__ __device__ constexpr int gather_warp_smem() {
+    return 32 * gather_row_stride<E>() + kD * 32 * (int)sizeof(typename RawT<E>::type);
+}
+
+// One warp per 32-token group.  Each lane brings its token's key row into
+// shared memory with one bulk copy, then every lane steps through the 128
+// channels from the top together: a kept channel's key goes to the token's
+// next slot from the end (slot n-1 for the highest kept channel, slot 0 for
+// the lowest), so the slots come out in ascending channel order; slots from
+// the token's count up to T_g are zero.  The slots are staged in the output
+// layout, and the group's T_g * 32 values, one contiguous block, are written
+// with 16-byte stores.
 template <typename E>
 __global__ void __launch_bounds__(kGatherWarps * 32)
     topp_gather_kernel(const E *__restrict__ k, const uint32_t *__restrict__ mask, const uint32_t *__restrict__ goff,
                        E *__restrict__ vals, uint32_t *__restrict__ status, int S, long ng, long n_groups) {
     using Raw = typename RawT<E>::type;
-    constexpr int kRowB = kD * (int)sizeof(E);
+    constexpr int kRowB = kD * (int)sizeof(E), kRowP = gather_row_stride<E>();
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ uint64_t bars[kGatherWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1561,52 +1631,55 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
     const long bh = idx / ng, g = idx % ng;
     const long t0 = g * 32;
     const int rows = (int)min(32L, (long)S - t0);
-    unsigned char *tile = smem_raw + (size_t)warp * 32 * kRowB;
+    unsigned char *tile = smem_raw + (size_t)warp * gather_warp_smem<E>();
+    Raw *stage = reinterpret_cast<Raw *>(tile + 32 * kRowP);
     const uint32_t bar = smem_u32(&bars[warp]);
     if (lane == 0) {
         mbar_init(bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         mbar_expect_tx(bar, (uint32_t)rows * (uint32_t)kRowB);
-        bulk_g2s(smem_u32(tile), k + ((size_t)bh * S + t0) * kD, (uint32_t)rows * (uint32_t)kRowB, bar);
     }
     __syncwarp();
     const bool valid = lane < rows;
+    if (valid) bulk_g2s(smem_u32(tile + lane * kRowP), k + ((size_t)bh * S + t0 + lane) * kD, (uint32_t)kRowB, bar);
     uint4 mw = make_uint4(0u, 0u, 0u, 0u);
     if (valid) mw = *reinterpret_cast<const uint4 *>(mask + ((size_t)bh * S + t0 + lane) * kMaskWords);
     const int n = __popc(mw.x) + __popc(mw.y) + __popc(mw.z) + __popc(mw.w);
     const uint32_t r0 = goff[idx];
-    const int Tg = (int)(goff[idx + 1] - r0);
+    const int Tg = (int)min(goff[idx + 1] - r0, (uint32_t)kD);
+    // slots past this token's count read zero (n <= T_g for a cache that
+    // spark_prune_topp wrote; a larger n only fills slots that are not copied)
+    for (int j = n; j < Tg; ++j) stage[j * 32 + lane] = (Raw)0;
     const bool ok = mbar_wait_bounded(bar, 0u);
     if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) {
             atomicOr(status, kDevTimeout);
-            (void)mbar_wait_bounded(bar, 0u);  // let the copy in flight land before the warp exits
+            (void)mbar_wait_bounded(bar, 0u);  // let the copies in flight land before the warp exits
         }
         __syncwarp();
         return;
     }
-    // the non-empty mask words, top first
-    uint32_t q0 = mw.w, q1 = mw.z, q2 = mw.y, q3 = mw.x;
-    int b0 = 96, b1 = 64, b2 = 32, b3 = 0;
+    {
+        const Raw *row = reinterpret_cast<const Raw *>(tile + lane * kRowP);
+        const uint32_t wds[4] = {mw.x, mw.y, mw.z, mw.w};
+        int j = n;
 #pragma unroll
-    for (int r = 0; r < 3; ++r) {
-        if (q2 == 0u) { q2 = q3; b2 = b3; q3 = 0u; }
-        if (q1 == 0u) { q1 = q2; b1 = b2; q2 = q3; b2 = b3; q3 = 0u; }
-        if (q0 == 0u) { q0 = q1; b0 = b1; q1 = q2; b1 = b2; q2 = q3; b2 = b3; q3 = 0u; }
-    }
-    const Raw *row = reinterpret_cast<const Raw *>(tile + lane * kRowB);
-    Raw *out = reinterpret_cast<Raw *>(vals) + (size_t)r0 * 32 + lane;
-    for (int j = Tg - 1; j >= 0; --j) {
-        Raw v = (Raw)0;
-        if (j < n) {
-            uint32_t b;
-            asm("bfind.u32 %0, %1;" : "=r"(b) : "r"(q0));
-            v = row[(b0 + (int)b) & (kD - 1)];
-            q0 &= ~(1u << b);
-            if (q0 == 0u) { q0 = q1; b0 = b1; q1 = q2; b1 = b2; q2 = q3; b2 = b3; }
+        for (int wi = 3; wi >= 0; --wi) {
+#pragma unroll
+            for (int b = 31; b >= 0; --b) {
+                if ((wds[wi] >> b) & 1u) {
+                    --j;
+                    stage[j * 32 + lane] = row[32 * wi + b];
+                }
+            }
         }
-        out[(size_t)j * 32] = v;
     }
+    __syncwarp();
+    // the group's slots: T_g rows of 32 values, contiguous in the stream
+    constexpr int kChunks = 32 * (int)sizeof(Raw) / 16;  // 16-byte pieces per slot row
+    const uint4 *src = reinterpret_cast<const uint4 *>(stage);
+    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<Raw *>(vals) + (size_t)r0 * 32);
+    for (int c = lane; c < Tg * kChunks; c += 32) __stcs(dst + c, src[c]);
 }
 
 template <typename E>
@@ -1635,7 +1708,7 @@ static cudaError_t launch_prune_topp_t(const void *k, const void *q_obs, int G, 
     topp_head_base_kernel<<<1, kScanThreads, 0, st>>>(tw.hrows, BH, tw.hbase, kc.goff + BH * ng);
     if (ng > 0) {
         topp_goff_kernel<<<(unsigned)BH, kScanThreads, 0, st>>>(tw.tg, ng, tw.hbase, kc.goff);
-        const int smem = kGatherWarps * 32 * kD * (int)sizeof(E);
+        const int smem = kGatherWarps * gather_warp_smem<E>();
         cudaError_t e = cudaFuncSetAttribute(topp_gather_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         const long n_groups = BH * ng;
