@@ -116,6 +116,44 @@ def test_grouped_four_groups_budgets(rates, dtype):
     check_grouped(kc, to_np(pre["k"]), to_np(pre["q_obs"]), wl.G, Tg, f"four groups {Tg}")
 
 
+@pytest.mark.parametrize("g", [4, 2])
+def test_grouped_row_lengths(g):
+    # per-row prompt lengths (spark_kcache.lens): each row's own tokens are
+    # pruned as if the row were that long, and nothing past it is written
+    wl = scaled(WORKLOADS["tiny"], B=3, S=700, Hkv=2, dtype="bf16", seed=71 + g)
+    pre = make_prefill(wl, DEV)
+    R, Hkv, S = wl.rows, wl.Hkv, wl.S
+    lens = [700, 333, 1]
+    Tg = spark_group_budget(D, RATES[g])
+    kc = KCache.empty(R, Hkv, S, D, sum(Tg), pre["k"].dtype, device=DEV)
+    kc.mask.fill_(0x55555555)
+    kc.lens = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    ws = workspace(spark_workspace_bytes(SPARK_OP_PRUNE, R, Hkv, wl.G, S, D, sum(Tg), 0))
+    spark_prune_grouped(pre["k"], pre["q_obs"], wl.G, wl.W, Tg, kc, ws)
+    torch.cuda.synchronize()
+    assert spark_device_status(ws) == 0
+    m_g, v_g = mask_np(kc), unpack_vals(kc)
+    s_g = kc.stats.cpu().numpy().reshape(R * Hkv, 4)
+    k3 = to_np(pre["k"]).reshape(R * Hkv, S, D)
+    q3 = to_np(pre["q_obs"]).reshape(R * Hkv * wl.G, wl.W, D)
+    qn_all = oracle.qnorm(q3, wl.G)
+    for bh in range(R * Hkv):
+        n = lens[bh // Hkv]
+        qn = qn_all[bh:bh + 1]
+        m_o, v_o, s_o = oracle.prune_grouped(k3[bh:bh + 1, :n], qn, Tg)
+        gid = oracle.group_of_channel(qn, len(Tg))[0]
+        for t in np.argwhere(np.any(m_g[bh, :n] != m_o[0], axis=-1)).ravel():
+            w = (qn[0] * np.abs(k3[bh, t])).astype(np.float32)
+            bg = ((m_g[bh, t][:, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(D)
+            bo = ((m_o[0, t][:, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(D)
+            assert _near_tie(w, gid, Tg, bg, bo), f"row head {bh}: non-tie mismatch at token {t}"
+        ok = np.all(m_g[bh, :n] == m_o[0], axis=-1)
+        assert np.array_equal(v_g[bh, :n][ok].view(np.uint32), v_o[0][ok].view(np.uint32))
+        assert s_g[bh, 0] == s_o[0, 0] == n * (D - sum(Tg))
+        np.testing.assert_allclose(s_g[bh, 1:], s_o[0, 1:], rtol=STATS_RTOL, atol=0)
+        assert np.all(m_g[bh, n:] == 0x55555555), f"row head {bh}: mask written past the row's length"
+
+
 def test_grouped_ties_integer_keys():
     # integer keys and window queries: exact saliency ties everywhere, and
     # equal window-query norms across group boundaries
