@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
     SPARK_OK = 0,
     SPARK_ERR_ARG = 1,          /* bad pointer, size, alignment or shape      */
-    SPARK_ERR_UNSUPPORTED = 2,  /* valid request this build does not run      */
+    SPARK_ERR_UNSUPPORTED = 2,  /* valid request the library does not run     */
     SPARK_ERR_CUDA = 3,         /* a CUDA call failed (launch, attribute)     */
     SPARK_ERR_TIMEOUT = 4,      /* device-side bounded wait ran out           */
     SPARK_ERR_WORKSPACE = 5     /* workspace NULL, misaligned or too small    */
@@ -368,7 +368,7 @@ SPARK_API int spark_decode_attn(const void *q, const spark_kcache *kc, const voi
 /*
  * SnapKV-style token eviction, the pre-pass SparK is stacked on ([W] 2 and
  * 4.1: SnapKV / PyramidKV bases; 3.2: the observation window).  The pages do
- * not define SnapKV; this build reads it as follows:
+ * not define SnapKV; the library reads it as follows:
  *   - the W window queries are the last W prompt positions p = S-W+w; each of
  *     the G*W (query head, window row) rows attends causally over keys 0..p
  *     (scale 1/sqrt(D)); a prefix token's score (t < S-W) is the sum of its
