@@ -871,7 +871,7 @@ __global__ void __launch_bounds__(dec_max_warps(G) * 32, 1) decode_kernel(DecArg
                 float2 s2[G / 2 > 0 ? G / 2 : 1];  // head pairs: packed fp32x2 FMAs
 #pragma unroll
                 for (int g = 0; g < (G / 2 > 0 ? G / 2 : 1); ++g) s2[g] = make_float2(0.f, 0.f);
-#pragma unroll 4
+#pragma unroll 8  // 8 measured 1-2 % faster than 4 on the long decode, 2 slower
                 for (int i = 0; i < a.T; ++i) {
                     const uint32_t pos = bit_top(cur);        // 0xffffffff when cur == 0
                     const int j = (int)((bq | pos) & (uint32_t)(kD - 1));
